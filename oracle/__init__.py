@@ -1,0 +1,31 @@
+"""CPU fp64 oracle of MILO's compressed-KV decode path.
+
+TEST INFRASTRUCTURE ONLY.  This package is the plain, slow, obviously correct
+restatement of the method that the CUDA path is checked against.  Only the
+tests, the smoke check and the benchmark's CPU-baseline leg may import it;
+the library itself never does, and it shares no code with the library.
+
+Sources (page "MILO: Efficient Many-shot In-Context Learning with Block-wise
+Low-rank Compression", a section summary of the paper):
+  §4.2  block-wise low-rank compression of keys and values, block by block;
+  §4.3  entropy-driven rank allocation under a fixed total budget;
+  §4.4  workflow: encode (partition, entropy, low-rank store), then decode.
+
+Every function states the passage it follows and the reading taken where the
+page is silent.
+"""
+from .milo import (  # noqa: F401
+    BudgetError,
+    allocate_ranks,
+    block_svd,
+    compress_layer,
+    compress_pool,
+    decode_attention,
+    decode_attention_dense,
+    rank_total,
+    reconstruct_pool,
+    spectral_entropy,
+    stored_factors,
+)
+from .hestenes import hestenes_svd  # noqa: F401
+from .tiefree import cut_gap, tiefree_taus  # noqa: F401
