@@ -1,0 +1,358 @@
+#!/usr/bin/env python
+"""Benchmark: compressed-KV decode tokens/s at the Qwen2.5-7B layer shape on B200.
+
+One step = one decode pass of the batch (rank-space scores, online softmax,
+rank-space value sum and expansion over every compressed block, the
+uncompressed suffix, and the split combine) through milo_decode_attn, on
+factors produced by milo_compress from a seeded synthetic cache.  Compression
+(Gram, Jacobi, entropy allocation, projection) is timed in the same run and
+reported as compressions/s.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl milo|reference] [--workload NAME]
+
+Prints one JSON line on rank 0.  For N > 1 launch with torch.distributed.run;
+every rank decodes its own batch (independent problems, no collective on the
+data path) and the timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "compressed-KV decode tokens/s at Qwen2.5-7B shape; achieved HBM GB/s vs peak"
+
+
+def _args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", default="milo", choices=["milo", "reference"])
+    p.add_argument("--workload", default="qwen2.5-7b-layer")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="bound of the CPU oracle sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            j = json.load(fh)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                r = subprocess.run(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                    "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
+                if r.returncode == 0 and r.stdout.strip():
+                    self.rows.append([x.strip() for x in r.stdout.strip().split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if len(r) > 5 + i and r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _to_dev(a, dt, torch):
+    if dt == "f32":
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def _algorithmic_bytes(ranks, wl, esize):
+    """Bytes one decode step must move: factors at their ranks (read once, shared by the batch),
+    the per-query suffix K and V, q and out."""
+    factors = int(ranks.sum()) * (wl.block_size + wl.head_dim) * esize
+    suffix = 2 * wl.batch * wl.kv_heads * wl.suffix * wl.head_dim * esize
+    qo = 2 * wl.batch * wl.q_heads * wl.head_dim * esize
+    return factors + suffix + qo
+
+
+def _cpu_baseline(wl, L, seconds):
+    """The fp64 oracle, as it stands, on this host: whole decode steps until `seconds` elapse."""
+    import oracle
+    from synth import from_storage
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(1)
+    except Exception:  # pragma: no cover
+        limiter = None
+    dt = wl.dtype
+    K, V = from_storage(L["K"], dt), from_storage(L["V"], dt)
+    lay = oracle.compress_layer(K, V, wl.block_size, wl.budgets[0], wl.r_min)
+    q = from_storage(L["q"], dt)
+    Ks, Vs = from_storage(L["K_suf"], dt), from_storage(L["V_suf"], dt)
+    steps = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle.decode_attention(q, lay, Ks, Vs)
+        steps += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    el = time.perf_counter() - t0
+    if limiter is not None:
+        limiter.unregister() if hasattr(limiter, "unregister") else None
+    return {"value": steps * wl.batch / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{steps} whole decode steps of {wl.name} (batch {wl.batch}) in {el:.1f} s, fp64 NumPy, "
+                      f"1 BLAS thread"}
+
+
+def run_reference(a):
+    """The oracle timed on the host cores: `steps` bounded decode steps after `warmup`."""
+    world, rank, _ = _dist()
+    if rank != 0:
+        return
+    from synth import WORKLOADS, gen_layer
+    import oracle
+    from synth import from_storage
+    wl = WORKLOADS[a.workload]
+    L = gen_layer(wl)
+    dt = wl.dtype
+    K, V = from_storage(L["K"], dt), from_storage(L["V"], dt)
+    lay = oracle.compress_layer(K, V, wl.block_size, wl.budgets[0], wl.r_min)
+    q = from_storage(L["q"], dt)
+    Ks, Vs = from_storage(L["K_suf"], dt), from_storage(L["V_suf"], dt)
+    # each step decodes a bounded sample of the batch so the whole run stays within minutes
+    per = max(1, min(wl.batch, int(os.environ.get("MILO_REF_ROWS", "2"))))
+    for w in range(a.warmup):
+        oracle.decode_attention(q[:per], lay, Ks[:per], Vs[:per])
+    t0 = time.perf_counter()
+    for s in range(a.steps):
+        i = (s * per) % wl.batch
+        sl = slice(i, min(wl.batch, i + per))
+        oracle.decode_attention(q[sl], lay, Ks[sl], Vs[sl])
+    el = time.perf_counter() - t0
+    value = a.steps * per / el
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference", "n_gpus": a.gpus,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * el / a.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "batch_per_step": per, "kv_heads": wl.kv_heads,
+                       "q_heads": wl.q_heads, "head_dim": wl.head_dim, "context": wl.context,
+                       "block_size": wl.block_size, "suffix": wl.suffix, "budget": wl.budgets[0]},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{per} of {wl.batch} queries per step, fp64 NumPy oracle"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_milo(a):
+    import torch
+    world, rank, local = _dist()
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    import decode_attention_milo_b200 as milo
+    from synth import WORKLOADS, gen_layer
+    wl = WORKLOADS[a.workload]
+    dt = wl.dtype
+    esize = 2 if dt == "bf16" else 4
+    L = gen_layer(wl)
+    dev = lambda x: _to_dev(x, dt, torch)
+    Kd, Vd = dev(L["K"]), dev(L["V"])
+    beta = wl.budgets[0]
+    S = wl.suffix
+
+    # --- compression, timed (one "compression" = the whole layer's K and V)
+    comp = []
+    for i in range(4):
+        st = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        f = milo.compress(Kd, Vd, wl.block_size, beta, wl.r_min)
+        e1.record(st)
+        torch.cuda.synchronize()
+        if i:
+            comp.append(e0.elapsed_time(e1))
+        f.close()
+
+    # --- decode inputs, rotated over enough copies that the working set exceeds 3x L2
+    probe = milo.compress(Kd, Vd, wl.block_size, beta, wl.r_min)
+    ranks = probe.ranks()
+    assert probe.status()[0] == 0
+    step_bytes = _algorithmic_bytes(ranks, wl, esize)
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    copies = max(2, math.ceil(3 * l2 / step_bytes))
+    sets = [probe]
+    for _ in range(copies - 1):
+        sets.append(milo.compress(Kd, Vd, wl.block_size, beta, wl.r_min))
+    del Kd, Vd
+    qs = [dev(L["q"]) for _ in range(copies)]
+    ks = [dev(L["K_suf"]) if S else None for _ in range(copies)]
+    vs = [dev(L["V_suf"]) if S else None for _ in range(copies)]
+    outs = [torch.empty_like(qs[0]) for _ in range(copies)]
+    for c in range(copies):  # first call per factor object builds its work list (synchronises once)
+        milo.decode_attn(qs[c], sets[c], ks[c], vs[c], out=outs[c])
+    torch.cuda.synchronize()
+    for f in sets:
+        assert f.status()[0] == 0
+
+    # capture one pass over all copies in a CUDA graph (the pages' launch-overhead remedy)
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g, stream=cap):
+            for c in range(copies):
+                milo.decode_attn(qs[c], sets[c], ks[c], vs[c], out=outs[c])
+    torch.cuda.synchronize()
+    reps_w = max(1, math.ceil(a.warmup / copies))
+    reps = max(1, math.ceil(a.steps / copies))
+    steps = reps * copies
+    for _ in range(reps_w):
+        g.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record(st)
+        for _ in range(reps):
+            g.replay()
+        e1.record(st)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / steps
+    value = world * wl.batch * steps / (ms / 1e3)
+    per_call_ms = ms_step  # every step is one milo_decode_attn call
+    kernels_per_call = sets[0].decode_launches(wl.batch, wl.q_heads, S)
+
+    # --- end to end through the public API: pinned host inputs, copies inside the timed region
+    hq = torch.from_numpy(np.ascontiguousarray(L["q"]).view(np.int16 if dt == "bf16" else np.float32)).pin_memory()
+    hk = torch.from_numpy(np.ascontiguousarray(L["K_suf"]).view(np.int16 if dt == "bf16" else np.float32)).pin_memory()
+    hv = torch.from_numpy(np.ascontiguousarray(L["V_suf"]).view(np.int16 if dt == "bf16" else np.float32)).pin_memory()
+    hout = torch.empty(qs[0].shape, dtype=torch.int16 if dt == "bf16" else torch.float32).pin_memory()
+    e2e_steps = min(steps, 500)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(st)
+    for s_ in range(e2e_steps):
+        c = s_ % copies
+        qd = qs[c].view(torch.int16 if dt == "bf16" else torch.float32)
+        qd.copy_(hq, non_blocking=True)
+        if S:
+            ks[c].view(qd.dtype).copy_(hk, non_blocking=True)
+            vs[c].view(qd.dtype).copy_(hv, non_blocking=True)
+        milo.decode_attn(qs[c], sets[c], ks[c], vs[c], out=outs[c])
+        hout.copy_(outs[c].view(hout.dtype), non_blocking=True)
+    f1.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = hq.numel() * hq.element_size() + (2 * hk.numel() * hk.element_size() if S else 0)
+    d2h = hout.numel() * hout.element_size()
+
+    peak, peak_kind = _peaks()
+    achieved = step_bytes / (per_call_ms / 1e3) / 1e9
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu = _cpu_baseline(wl, L, a.cpu_seconds)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+            "warmup": reps_w * copies, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": dt, "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "kv_heads": wl.kv_heads, "q_heads": wl.q_heads,
+                       "head_dim": wl.head_dim, "context": wl.context, "block_size": wl.block_size,
+                       "suffix": wl.suffix, "budget": beta, "r_min": wl.r_min,
+                       "ranks_total": int(ranks.sum()), "parallelism": f"replica x{world}",
+                       "l2": f"inputs rotated over {copies} copies ({copies * step_bytes / 1e6:.0f} MB > 3x L2)",
+                       "launch": "CUDA graph of one pass over the copies"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                         "bytes_per_step": step_bytes,
+                         "note": "achieved = algorithmic bytes / time of the whole milo_decode_attn call"},
+            "e2e": {"value": world * wl.batch * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "compress": {"compressions_per_s": 1e3 / statistics.median(comp), "ms": statistics.median(comp),
+                         "unit": "whole-layer compressions/s"},
+            "gpu_launches": kernels_per_call * steps,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    del g
+    for f in sets:
+        f.close()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    a = _args()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_milo(a)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,209 @@
+"""Python binding of libmilo.so: MILO compressed-KV decode attention on B200.
+
+Argument marshalling only.  Every step of the path runs in the library's CUDA
+kernels; PyTorch supplies device memory (tensors) and the current stream.
+The library must be built first (python -m decode_attention_milo_b200.build);
+importing the binding without it raises, there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+__all__ = ["F32", "BF16", "MiloError", "Factors", "compress", "decode_attn", "import_factors", "lib_path",
+           "load_library"]
+
+F32, BF16 = 0, 1
+KEEP_INTERMEDIATES = 1
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def lib_path() -> str:
+    return os.path.join(_HERE, "libmilo.so")
+
+
+class MiloError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {_status_string(code)} ({code})")
+
+
+class _Desc(ctypes.Structure):
+    _fields_ = [
+        ("num_kv_heads", ctypes.c_int32), ("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32), ("context", ctypes.c_int64), ("r_min", ctypes.c_int32),
+        ("pool_rows", ctypes.c_int32), ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("ranks", ctypes.c_void_p), ("row_offsets", ctypes.c_void_p), ("tok", ctypes.c_void_p),
+        ("dim", ctypes.c_void_p), ("eigvals", ctypes.c_void_p), ("eigvecs", ctypes.c_void_p),
+        ("entropy", ctypes.c_void_p), ("quotas", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def load_library(path: str | None = None):
+    """Loads libmilo.so (once) and declares its C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or lib_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m decode_attention_milo_b200.build`")
+    L = ctypes.CDLL(path)
+    vp, i32, i64, u32, f32, f64 = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32,
+                                   ctypes.c_float, ctypes.c_double)
+    L.milo_abi_version.restype = i32
+    L.milo_status_string.restype = ctypes.c_char_p
+    L.milo_status_string.argtypes = [i32]
+    L.milo_compress.restype = i32
+    L.milo_compress.argtypes = [vp, vp, i32, i32, i64, i32, i32, f64, i32, i32, u32, vp, ctypes.POINTER(vp)]
+    L.milo_decode_attn.restype = i32
+    L.milo_decode_attn.argtypes = [vp, i32, i32, vp, vp, vp, i32, f32, vp, vp]
+    L.milo_decode_launches.restype = i32
+    L.milo_decode_launches.argtypes = [vp, i32, i32, i32]
+    L.milo_factors_ranks.restype = i32
+    L.milo_factors_ranks.argtypes = [vp, vp]
+    L.milo_factors_describe.restype = i32
+    L.milo_factors_describe.argtypes = [vp, ctypes.POINTER(_Desc)]
+    L.milo_factors_status.restype = i32
+    L.milo_factors_status.argtypes = [vp, ctypes.POINTER(u32)]
+    L.milo_factors_import.restype = i32
+    L.milo_factors_import.argtypes = [i32, i32, i64, i32, i32, i32, vp, vp, vp, vp, ctypes.POINTER(vp)]
+    L.milo_factors_destroy.restype = None
+    L.milo_factors_destroy.argtypes = [vp]
+    if L.milo_abi_version() != 1:
+        raise RuntimeError("libmilo.so ABI version mismatch")
+    _lib = L
+    return L
+
+
+def _status_string(code: int) -> str:
+    return load_library().milo_status_string(code).decode()
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise MiloError(code, what)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _stream_ptr(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev_ptr(t, name):
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+class Factors:
+    """A compressed layer: per-block low-rank factors owned by the library."""
+
+    def __init__(self, handle: ctypes.c_void_p):
+        self._h = handle
+
+    @property
+    def handle(self):
+        if not self._h:
+            raise ValueError("factor object was destroyed")
+        return self._h
+
+    def describe(self) -> dict:
+        d = _Desc()
+        _check(load_library().milo_factors_describe(self.handle, ctypes.byref(d)), "milo_factors_describe")
+        return {name: getattr(d, name) for name, _ in _Desc._fields_}
+
+    def ranks(self) -> np.ndarray:
+        d = self.describe()
+        out = np.zeros((2 * d["num_kv_heads"], d["num_blocks"]), dtype=np.int32)
+        _check(load_library().milo_factors_ranks(self.handle, out.ctypes.data_as(ctypes.c_void_p)),
+               "milo_factors_ranks")
+        return out
+
+    def decode_launches(self, batch: int, num_q_heads: int, suffix_len: int) -> int:
+        """Kernels one decode call with this shape launches."""
+        n = load_library().milo_decode_launches(self.handle, batch, num_q_heads, suffix_len)
+        if n < 0:
+            raise MiloError(-n, "milo_decode_launches")
+        return n
+
+    def status(self) -> tuple[int, int]:
+        bits = ctypes.c_uint32(0)
+        code = load_library().milo_factors_status(self.handle, ctypes.byref(bits))
+        return code, bits.value
+
+    def close(self):
+        if self._h:
+            load_library().milo_factors_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def compress(K, V, block_size: int, budget: float, r_min: int = 4, max_sweeps: int = 0,
+             keep_intermediates: bool = False, stream=None) -> Factors:
+    """Compresses one layer's K, V [H][T][d] (CUDA tensors, float32 or bfloat16). See milo_compress."""
+    if K.shape != V.shape or K.dim() != 3 or K.dtype != V.dtype:
+        raise ValueError("K and V must both be [H][T][d] with the same dtype")
+    H, T, d = K.shape
+    h = ctypes.c_void_p()
+    flags = KEEP_INTERMEDIATES if keep_intermediates else 0
+    _check(load_library().milo_compress(_dev_ptr(K, "K"), _dev_ptr(V, "V"), _dtype_code(K), H, T, d, block_size,
+                                        float(budget), r_min, max_sweeps, flags, _stream_ptr(stream),
+                                        ctypes.byref(h)), "milo_compress")
+    return Factors(h)
+
+
+def decode_attn(q, factors: Factors, K_suf=None, V_suf=None, scale: float = 0.0, out=None, stream=None):
+    """One decode step: q [B][Hq][d] → out [B][Hq][d]. Suffix K/V [B][H][S][d] or None. See milo_decode_attn."""
+    import torch
+    if q.dim() != 3:
+        raise ValueError("q must be [batch][q_heads][d]")
+    B, Hq, d = q.shape
+    S = 0
+    if K_suf is not None:
+        if V_suf is None or K_suf.shape != V_suf.shape or K_suf.dim() != 4 or K_suf.shape[0] != B:
+            raise ValueError("K_suf and V_suf must both be [batch][kv_heads][S][d]")
+        S = K_suf.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    _check(load_library().milo_decode_attn(_dev_ptr(q, "q"), B, Hq, factors.handle,
+                                           _dev_ptr(K_suf, "K_suf") if S else None,
+                                           _dev_ptr(V_suf, "V_suf") if S else None, S, float(scale),
+                                           _dev_ptr(out, "out"), _stream_ptr(stream)), "milo_decode_attn")
+    return out
+
+
+def import_factors(dtype: int, num_kv_heads: int, context: int, head_dim: int, block_size: int, r_min: int,
+                   ranks: np.ndarray, tok: np.ndarray, dim: np.ndarray, stream=None) -> Factors:
+    """Builds a factor object from host arrays in the library's layout (tok [rows][n], dim [rows][d])."""
+    ranks = np.ascontiguousarray(ranks, dtype=np.int32)
+    tok = np.ascontiguousarray(tok)
+    dim = np.ascontiguousarray(dim)
+    h = ctypes.c_void_p()
+    _check(load_library().milo_factors_import(dtype, num_kv_heads, context, head_dim, block_size, r_min,
+                                              ranks.ctypes.data_as(ctypes.c_void_p),
+                                              tok.ctypes.data_as(ctypes.c_void_p),
+                                              dim.ctypes.data_as(ctypes.c_void_p), _stream_ptr(stream),
+                                              ctypes.byref(h)), "milo_factors_import")
+    return Factors(h)

@@ -1,0 +1,29 @@
+// Tensor-core (tcgen05) rank-space decode attention: host interface.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "internal.h"
+
+namespace milo {
+
+struct TcPlan;  // cached work list, tensor maps and scratch for one decode shape
+
+struct TcInputs {
+  const void* q;
+  const void* K_suf;
+  const void* V_suf;
+  const void* tok;
+  const void* dim;
+  uint32_t* status;
+  int pool_rows;
+  const int32_t* host_ranks;  // [2H][nb]
+};
+
+bool tc_supported(const DecodeShape& s);
+int tc_launches(const DecodeShape& s);
+cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, void* out, cudaStream_t st);
+void tc_plan_destroy(TcPlan* plan);
+
+}  // namespace milo

@@ -1,0 +1,60 @@
+// Host-side interfaces between the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace milo {
+
+struct CompressShape {
+  int H;       // KV heads
+  int64_t T;   // context
+  int d;       // head dim
+  int n;       // block size
+  int nb;      // blocks per pool
+  int R;       // total rank per pool (before capping at nb*d)
+  int pool_rows;  // min(R, nb*d)
+  int r_min;
+  int max_sweeps;
+  bool bf16;
+};
+
+struct CompressBuffers {
+  const void* K;
+  const void* V;
+  float* gram;        // [2H][nb][d][d]
+  float* eigvals;     // [2H][nb][d]
+  float* eigvecs;     // [2H][nb][d][d]
+  double* entropy;    // [2H][nb]
+  double* quotas;     // [2H][nb]
+  int32_t* ranks;     // [2H][nb]
+  int64_t* row_offsets;  // [2H][nb+1]
+  void* tok;          // [2H*pool_rows][n]
+  void* dim;          // [2H*pool_rows][d]
+  uint32_t* status;
+};
+
+cudaError_t launch_compress(const CompressShape& s, const CompressBuffers& b, cudaStream_t st);
+
+// Rank-space decode on CUDA cores (any dtype; the fp32 path and a cross-check for bf16).
+struct DecodeShape {
+  int H, nb, n, d, Bq, Hq, S;
+  bool bf16;
+  float scale;
+};
+struct DecodeBuffers {
+  const void* q;
+  const void* K_suf;
+  const void* V_suf;
+  const int32_t* ranks;
+  const int64_t* row_offsets;
+  const void* tok;
+  const void* dim;
+  float* partials;  // [(H*nb*rows) + Bq*H*G][d+2]
+  void* out;
+  uint32_t* status;
+};
+size_t simt_decode_partials_floats(const DecodeShape& s);
+cudaError_t launch_decode_simt(const DecodeShape& s, const DecodeBuffers& b, cudaStream_t st);
+
+}  // namespace milo

@@ -1,0 +1,353 @@
+// C ABI of the library (declared in include/milo.h): argument checks, the
+// factor object, scratch management and launch sequencing.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "../../include/milo.h"
+#include "common.cuh"
+#include "decode_tc.h"
+#include "internal.h"
+
+struct milo_factors {
+  int device = 0;
+  int H = 0;
+  int64_t T = 0;
+  int d = 0, n = 0, nb = 0, r_min = 0, R = 0, pool_rows = 0;
+  int dtype = 0;
+  uint32_t flags = 0;
+  int32_t* ranks = nullptr;
+  int64_t* row_offsets = nullptr;
+  void* tok = nullptr;
+  void* dim = nullptr;
+  uint32_t* status = nullptr;
+  float* eigvals = nullptr;
+  float* eigvecs = nullptr;
+  double* entropy = nullptr;
+  double* quotas = nullptr;
+  cudaEvent_t ready = nullptr;  // recorded after the factors are written
+  // decode scratch, owned here and reused by later calls
+  std::mutex mu;
+  std::vector<int32_t> host_ranks;
+  float* partials = nullptr;
+  size_t partials_floats = 0;
+  milo::TcPlan* tc_plan = nullptr;
+};
+
+namespace {
+
+size_t esize(int dtype) { return dtype == MILO_BF16 ? 2 : 4; }
+
+milo_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MILO_OK;
+  if (e == cudaErrorMemoryAllocation) return MILO_ERR_OUT_OF_MEMORY;
+  return MILO_ERR_CUDA;
+}
+
+#define MILO_CUDA(call)                                  \
+  do {                                                   \
+    cudaError_t e_ = (call);                             \
+    if (e_ != cudaSuccess) return cuda_status(e_);       \
+  } while (0)
+
+void free_all(milo_factors* f) {
+  if (!f) return;
+  cudaFree(f->ranks);
+  cudaFree(f->row_offsets);
+  cudaFree(f->tok);
+  cudaFree(f->dim);
+  cudaFree(f->status);
+  cudaFree(f->eigvals);
+  if (f->eigvecs) cudaFreeAsync(f->eigvecs, 0);
+  cudaFree(f->entropy);
+  cudaFree(f->quotas);
+  cudaFree(f->partials);
+  if (f->ready) cudaEventDestroy(f->ready);
+  milo::tc_plan_destroy(f->tc_plan);
+}
+
+bool valid_dtype(int32_t dt) { return dt == MILO_F32 || dt == MILO_BF16; }
+
+milo_status check_layer_shape(int32_t dtype, int32_t H, int64_t T, int32_t d, int32_t n, int32_t r_min) {
+  if (!valid_dtype(dtype) || H <= 0 || T <= 0 || n <= 0 || r_min < 1) return MILO_ERR_INVALID_ARGUMENT;
+  if (d != 64 && d != 128) return d > 0 ? MILO_ERR_UNSUPPORTED : MILO_ERR_INVALID_ARGUMENT;
+  if (T % n != 0 || n < d || n % 64 != 0 || r_min > d) return MILO_ERR_INVALID_ARGUMENT;
+  if (T / n > (1 << 20) || H > 1024) return MILO_ERR_INVALID_ARGUMENT;
+  return MILO_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t milo_abi_version(void) { return MILO_ABI_VERSION; }
+
+const char* milo_status_string(int32_t s) {
+  switch (s) {
+    case MILO_OK: return "ok";
+    case MILO_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case MILO_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MILO_ERR_BUDGET: return "budget below num_blocks * r_min";
+    case MILO_ERR_NO_CONVERGENCE: return "eigensolver did not converge";
+    case MILO_ERR_DEVICE_CHECK: return "device-side check failed";
+    case MILO_ERR_CUDA: return "CUDA error";
+    case MILO_ERR_OUT_OF_MEMORY: return "out of device memory";
+    default: return "unknown status";
+  }
+}
+
+milo_status milo_compress(const void* K, const void* V, int32_t dtype, int32_t num_kv_heads, int64_t context,
+                          int32_t head_dim, int32_t block_size, double budget, int32_t r_min,
+                          int32_t max_sweeps, uint32_t flags, void* stream, milo_factors** out) {
+  if (!out) return MILO_ERR_INVALID_ARGUMENT;
+  *out = nullptr;
+  if (!K || !V) return MILO_ERR_INVALID_ARGUMENT;
+  milo_status st = check_layer_shape(dtype, num_kv_heads, context, head_dim, block_size, r_min);
+  if (st != MILO_OK) return st;
+  if (!(budget > 0.0) || !isfinite(budget) || max_sweeps < 0 || (flags & ~MILO_KEEP_INTERMEDIATES))
+    return MILO_ERR_INVALID_ARGUMENT;
+  const int nb = (int)(context / block_size);
+  const double Rd = floor(budget * (double)(context * head_dim) / (double)(block_size + head_dim));
+  if (Rd < (double)nb * r_min) return MILO_ERR_BUDGET;
+  const int64_t full = (int64_t)nb * head_dim;
+  const int R = Rd >= (double)full ? (int)full : (int)Rd;
+
+  milo_factors* f = new (std::nothrow) milo_factors();
+  if (!f) return MILO_ERR_OUT_OF_MEMORY;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  f->H = num_kv_heads;
+  f->T = context;
+  f->d = head_dim;
+  f->n = block_size;
+  f->nb = nb;
+  f->r_min = r_min;
+  f->R = R;
+  f->pool_rows = R;
+  f->dtype = dtype;
+  f->flags = flags;
+  const int P = 2 * num_kv_heads;
+  const size_t rows = (size_t)P * f->pool_rows;
+  const size_t nblk = (size_t)P * nb;
+  const size_t dd = (size_t)head_dim * head_dim;
+  float* gram = nullptr;
+  cudaError_t e = cudaGetDevice(&f->device);
+  auto fail = [&](cudaError_t err) {
+    if (gram) cudaFreeAsync(gram, s);
+    cudaStreamSynchronize(s);
+    free_all(f);
+    delete f;
+    return cuda_status(err);
+  };
+  if (e != cudaSuccess) return fail(e);
+#define ALLOC(ptr, bytes)                                   \
+  do {                                                      \
+    e = cudaMalloc((void**)&(ptr), (bytes));                \
+    if (e != cudaSuccess) return fail(e);                   \
+  } while (0)
+  ALLOC(f->ranks, nblk * sizeof(int32_t));
+  ALLOC(f->row_offsets, (size_t)P * (nb + 1) * sizeof(int64_t));
+  ALLOC(f->tok, rows * block_size * esize(dtype) + 256);
+  ALLOC(f->dim, rows * head_dim * esize(dtype) + 256);
+  ALLOC(f->status, sizeof(uint32_t));
+  ALLOC(f->eigvals, nblk * head_dim * sizeof(float));
+  if ((e = cudaMallocAsync((void**)&f->eigvecs, nblk * dd * sizeof(float), s)) != cudaSuccess) return fail(e);
+  ALLOC(f->entropy, nblk * sizeof(double));
+  ALLOC(f->quotas, nblk * sizeof(double));
+  if ((e = cudaMallocAsync((void**)&gram, nblk * dd * sizeof(float), s)) != cudaSuccess) return fail(e);
+#undef ALLOC
+  if ((e = cudaMemsetAsync(f->status, 0, sizeof(uint32_t), s)) != cudaSuccess) return fail(e);
+  if ((e = cudaMemsetAsync(f->tok, 0, rows * block_size * esize(dtype) + 256, s)) != cudaSuccess) return fail(e);
+  if ((e = cudaMemsetAsync(f->dim, 0, rows * head_dim * esize(dtype) + 256, s)) != cudaSuccess) return fail(e);
+
+  milo::CompressShape cs{num_kv_heads, context, head_dim, block_size, nb, R, f->pool_rows, r_min,
+                         max_sweeps ? max_sweeps : 30, dtype == MILO_BF16};
+  milo::CompressBuffers cb{K, V, gram, f->eigvals, f->eigvecs, f->entropy, f->quotas, f->ranks,
+                           f->row_offsets, f->tok, f->dim, f->status};
+  if ((e = milo::launch_compress(cs, cb, s)) != cudaSuccess) return fail(e);
+  if ((e = cudaEventCreateWithFlags(&f->ready, cudaEventDisableTiming)) != cudaSuccess) return fail(e);
+  if ((e = cudaEventRecord(f->ready, s)) != cudaSuccess) return fail(e);
+  // The Gram scratch (and, unless kept, the eigenpairs) are released once the stream has used them.
+  cudaFreeAsync(gram, s);
+  gram = nullptr;
+  if (!(flags & MILO_KEEP_INTERMEDIATES)) {
+    cudaFreeAsync(f->eigvecs, s);
+    f->eigvecs = nullptr;
+  }
+  *out = f;
+  return MILO_OK;
+}
+
+milo_status milo_factors_import(int32_t dtype, int32_t num_kv_heads, int64_t context, int32_t head_dim,
+                                int32_t block_size, int32_t r_min, const int32_t* host_ranks,
+                                const void* host_tok, const void* host_dim, void* stream, milo_factors** out) {
+  if (!out) return MILO_ERR_INVALID_ARGUMENT;
+  *out = nullptr;
+  if (!host_ranks || !host_tok || !host_dim) return MILO_ERR_INVALID_ARGUMENT;
+  milo_status st = check_layer_shape(dtype, num_kv_heads, context, head_dim, block_size, r_min);
+  if (st != MILO_OK) return st;
+  const int nb = (int)(context / block_size);
+  const int P = 2 * num_kv_heads;
+  int pool_rows = -1;
+  for (int p = 0; p < P; ++p) {
+    int64_t sum = 0;
+    for (int b = 0; b < nb; ++b) {
+      const int r = host_ranks[(size_t)p * nb + b];
+      if (r < 1 || r > head_dim) return MILO_ERR_INVALID_ARGUMENT;
+      sum += r;
+    }
+    if (pool_rows < 0) pool_rows = (int)sum;
+    if (sum != pool_rows) return MILO_ERR_INVALID_ARGUMENT;
+  }
+  milo_factors* f = new (std::nothrow) milo_factors();
+  if (!f) return MILO_ERR_OUT_OF_MEMORY;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  f->H = num_kv_heads;
+  f->T = context;
+  f->d = head_dim;
+  f->n = block_size;
+  f->nb = nb;
+  f->r_min = r_min;
+  f->R = pool_rows;
+  f->pool_rows = pool_rows;
+  f->dtype = dtype;
+  const size_t rows = (size_t)P * pool_rows;
+  std::vector<int64_t> offs((size_t)P * (nb + 1));
+  for (int p = 0; p < P; ++p) {
+    int64_t o = (int64_t)p * pool_rows;
+    for (int b = 0; b < nb; ++b) {
+      offs[(size_t)p * (nb + 1) + b] = o;
+      o += host_ranks[(size_t)p * nb + b];
+    }
+    offs[(size_t)p * (nb + 1) + nb] = o;
+  }
+  cudaError_t e = cudaGetDevice(&f->device);
+  auto fail = [&](cudaError_t err) {
+    free_all(f);
+    delete f;
+    return cuda_status(err);
+  };
+  if (e != cudaSuccess) return fail(e);
+  const size_t tb = rows * block_size * esize(dtype), db = rows * head_dim * esize(dtype);
+  if ((e = cudaMalloc((void**)&f->ranks, (size_t)P * nb * sizeof(int32_t))) != cudaSuccess) return fail(e);
+  if ((e = cudaMalloc((void**)&f->row_offsets, offs.size() * sizeof(int64_t))) != cudaSuccess) return fail(e);
+  if ((e = cudaMalloc(&f->tok, tb + 256)) != cudaSuccess) return fail(e);
+  if ((e = cudaMalloc(&f->dim, db + 256)) != cudaSuccess) return fail(e);
+  if ((e = cudaMalloc((void**)&f->status, sizeof(uint32_t))) != cudaSuccess) return fail(e);
+  if ((e = cudaMemsetAsync(f->status, 0, sizeof(uint32_t), s)) != cudaSuccess) return fail(e);
+  if ((e = cudaMemsetAsync(f->tok, 0, tb + 256, s)) != cudaSuccess) return fail(e);
+  if ((e = cudaMemsetAsync(f->dim, 0, db + 256, s)) != cudaSuccess) return fail(e);
+  if ((e = cudaMemcpyAsync(f->ranks, host_ranks, (size_t)P * nb * sizeof(int32_t), cudaMemcpyHostToDevice, s)) !=
+      cudaSuccess)
+    return fail(e);
+  if ((e = cudaMemcpyAsync(f->row_offsets, offs.data(), offs.size() * sizeof(int64_t), cudaMemcpyHostToDevice,
+                           s)) != cudaSuccess)
+    return fail(e);
+  if ((e = cudaMemcpyAsync(f->tok, host_tok, tb, cudaMemcpyHostToDevice, s)) != cudaSuccess) return fail(e);
+  if ((e = cudaMemcpyAsync(f->dim, host_dim, db, cudaMemcpyHostToDevice, s)) != cudaSuccess) return fail(e);
+  if ((e = cudaEventCreateWithFlags(&f->ready, cudaEventDisableTiming)) != cudaSuccess) return fail(e);
+  if ((e = cudaEventRecord(f->ready, s)) != cudaSuccess) return fail(e);
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return fail(e);
+  f->host_ranks.assign(host_ranks, host_ranks + (size_t)P * nb);
+  *out = f;
+  return MILO_OK;
+}
+
+milo_status milo_factors_ranks(const milo_factors* f, int32_t* host_ranks) {
+  if (!f || !host_ranks) return MILO_ERR_INVALID_ARGUMENT;
+  MILO_CUDA(cudaEventSynchronize(f->ready));
+  MILO_CUDA(cudaMemcpy(host_ranks, f->ranks, (size_t)2 * f->H * f->nb * sizeof(int32_t), cudaMemcpyDeviceToHost));
+  return MILO_OK;
+}
+
+milo_status milo_factors_describe(const milo_factors* f, milo_factors_desc* d) {
+  if (!f || !d) return MILO_ERR_INVALID_ARGUMENT;
+  memset(d, 0, sizeof(*d));
+  d->num_kv_heads = f->H;
+  d->num_blocks = f->nb;
+  d->block_size = f->n;
+  d->head_dim = f->d;
+  d->context = f->T;
+  d->r_min = f->r_min;
+  d->pool_rows = f->pool_rows;
+  d->dtype = f->dtype;
+  d->ranks = f->ranks;
+  d->row_offsets = f->row_offsets;
+  d->tok = f->tok;
+  d->dim = f->dim;
+  const bool keep = f->flags & MILO_KEEP_INTERMEDIATES;
+  d->eigvals = keep ? f->eigvals : nullptr;
+  d->eigvecs = keep ? f->eigvecs : nullptr;
+  d->entropy = keep ? f->entropy : nullptr;
+  d->quotas = keep ? f->quotas : nullptr;
+  return MILO_OK;
+}
+
+milo_status milo_factors_status(const milo_factors* f, uint32_t* host_bits) {
+  if (!f) return MILO_ERR_INVALID_ARGUMENT;
+  MILO_CUDA(cudaDeviceSynchronize());
+  uint32_t bits = 0;
+  MILO_CUDA(cudaMemcpy(&bits, f->status, sizeof(bits), cudaMemcpyDeviceToHost));
+  if (host_bits) *host_bits = bits;
+  if (bits & milo::kStatusNoConvergence) return MILO_ERR_NO_CONVERGENCE;
+  if (bits) return MILO_ERR_DEVICE_CHECK;
+  return MILO_OK;
+}
+
+void milo_factors_destroy(milo_factors* f) {
+  if (!f) return;
+  cudaDeviceSynchronize();
+  free_all(f);
+  delete f;
+}
+
+int32_t milo_decode_launches(const milo_factors* f, int32_t batch, int32_t num_q_heads, int32_t suffix_len) {
+  if (!f || batch <= 0 || num_q_heads <= 0 || suffix_len < 0 || num_q_heads % f->H != 0)
+    return -(int32_t)MILO_ERR_INVALID_ARGUMENT;
+  milo::DecodeShape ds{f->H, f->nb, f->n, f->d, batch, num_q_heads, suffix_len, f->dtype == MILO_BF16, 1.f};
+  if (f->dtype == MILO_BF16 && milo::tc_supported(ds)) return milo::tc_launches(ds);
+  return suffix_len > 0 ? 3 : 2;
+}
+
+milo_status milo_decode_attn(const void* q, int32_t batch, int32_t num_q_heads, const milo_factors* fc,
+                             const void* K_suffix, const void* V_suffix, int32_t suffix_len, float scale,
+                             void* out, void* stream) {
+  if (!fc || !q || !out || batch <= 0 || num_q_heads <= 0 || suffix_len < 0) return MILO_ERR_INVALID_ARGUMENT;
+  milo_factors* f = const_cast<milo_factors*>(fc);
+  if (num_q_heads % f->H != 0) return MILO_ERR_INVALID_ARGUMENT;
+  if (suffix_len > 0 && (!K_suffix || !V_suffix)) return MILO_ERR_INVALID_ARGUMENT;
+  if (!(scale == scale) || isinf(scale)) return MILO_ERR_INVALID_ARGUMENT;
+  if (batch > 65535 || num_q_heads > 4096 || suffix_len > (1 << 20)) return MILO_ERR_INVALID_ARGUMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)f->d);
+  std::lock_guard<std::mutex> lock(f->mu);
+  MILO_CUDA(cudaStreamWaitEvent(s, f->ready, 0));
+  milo::DecodeShape ds{f->H, f->nb, f->n, f->d, batch, num_q_heads, suffix_len, f->dtype == MILO_BF16, sc};
+  milo::DecodeBuffers db{q, K_suffix, V_suffix, f->ranks, f->row_offsets, f->tok, f->dim, nullptr, out, f->status};
+  if (f->dtype == MILO_BF16 && milo::tc_supported(ds)) {
+    if (f->host_ranks.empty()) {
+      f->host_ranks.resize((size_t)2 * f->H * f->nb);
+      MILO_CUDA(cudaStreamSynchronize(s));
+      MILO_CUDA(cudaMemcpy(f->host_ranks.data(), f->ranks, f->host_ranks.size() * sizeof(int32_t),
+                           cudaMemcpyDeviceToHost));
+    }
+    milo::TcInputs in{q, K_suffix, V_suffix, f->tok, f->dim, f->status, f->pool_rows, f->host_ranks.data()};
+    return cuda_status(milo::tc_decode(&f->tc_plan, ds, in, out, s));
+  }
+  const size_t need = milo::simt_decode_partials_floats(ds);
+  if (need > f->partials_floats) {
+    MILO_CUDA(cudaStreamSynchronize(s));
+    cudaFree(f->partials);
+    f->partials = nullptr;
+    f->partials_floats = 0;
+    MILO_CUDA(cudaMalloc((void**)&f->partials, need * sizeof(float)));
+    f->partials_floats = need;
+  }
+  db.partials = f->partials;
+  return cuda_status(milo::launch_decode_simt(ds, db, s));
+}
+
+}  // extern "C"

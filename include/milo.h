@@ -1,0 +1,184 @@
+/*
+ * milo.h — C ABI of the B200 (sm_100a) compressed-KV decode attention library.
+ *
+ * The method is MILO (page "MILO: Efficient Many-shot In-Context Learning with
+ * Block-wise Low-rank Compression"):
+ *   §4.2  the many-shot KV cache is split into blocks of several examples and
+ *         each block's keys and values get their own low-rank approximation;
+ *   §4.3  the ranks of the blocks come from their entropy under a fixed total
+ *         rank budget;
+ *   §4.4  encoding partitions the context, analyses entropy and stores the
+ *         low-rank caches; decoding attends over them.
+ *
+ * Two calls carry the method: milo_compress (encode) and milo_decode_attn
+ * (decode).  Everything else manages the factor object they share.
+ *
+ * Conventions for every call:
+ *  - All tensors are dense, row-major, and live in device memory unless a
+ *    parameter says "host".  The library never takes ownership of a caller's
+ *    buffer and never keeps a pointer to it after the call returns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Calls are asynchronous on it unless marked "synchronises".
+ *  - Errors are reported only through the return value.  Invalid arguments
+ *    are rejected before anything is launched or allocated.  Errors found by
+ *    a kernel (non-convergence, a failed bounds check, an expired wait) are
+ *    recorded in the factor object's device status word and read back by
+ *    milo_factors_status.  No call aborts the process or traps the GPU.
+ *  - There is no CPU fallback: without an sm_100 device every compute call
+ *    returns MILO_ERR_CUDA.
+ *
+ * Layout of a factor object (one layer):
+ *   pool p = 2*h + t for KV head h and tensor t (0 = keys, 1 = values);
+ *   block b of pool p holds ranks[p*nb + b] = r rows in two row arrays that
+ *   share one row index space:
+ *     tok [rows][n]  token-side factor, transposed: row j of block b is
+ *                    column j of U_b = X_b · B_b  (X_b the n×d block)
+ *     dim [rows][d]  dimension-side factor: row j is column j of B_b
+ *   so that X_b ≈ U_b · B_bᵀ = Σ_j tok[row0+j]ᵀ · dim[row0+j].  The rows of
+ *   block b start at row_offsets[p*(nb+1) + b]; the blocks of a pool are
+ *   consecutive and pool p starts at row p * pool_rows.  Factor elements have
+ *   the dtype of the compressed cache.
+ */
+#ifndef MILO_H_
+#define MILO_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MILO_ABI_VERSION 1
+
+typedef enum {
+  MILO_OK = 0,
+  MILO_ERR_INVALID_ARGUMENT = 1, /* a shape, pointer or option is out of range  */
+  MILO_ERR_UNSUPPORTED = 2,      /* valid in principle, not built (e.g. d = 96) */
+  MILO_ERR_BUDGET = 3,           /* budget below num_blocks * r_min             */
+  MILO_ERR_NO_CONVERGENCE = 4,   /* eigensolver hit max_sweeps                  */
+  MILO_ERR_DEVICE_CHECK = 5,     /* a kernel's bounds check or bounded wait failed */
+  MILO_ERR_CUDA = 6,             /* a CUDA runtime/driver call failed           */
+  MILO_ERR_OUT_OF_MEMORY = 7
+} milo_status;
+
+typedef enum { MILO_F32 = 0, MILO_BF16 = 1 } milo_dtype;
+
+/* milo_compress flags */
+#define MILO_KEEP_INTERMEDIATES 1u /* keep fp32 eigenpairs, fp64 entropies and quotas */
+
+typedef struct milo_factors milo_factors; /* opaque, device-resident, library-owned */
+
+typedef struct {
+  int32_t num_kv_heads;  /* H */
+  int32_t num_blocks;    /* nb = context / block_size */
+  int32_t block_size;    /* n */
+  int32_t head_dim;      /* d */
+  int64_t context;       /* T */
+  int32_t r_min;
+  int32_t pool_rows;     /* rows per pool = min(R, nb*d), R = floor(budget*T*d/(n+d)) */
+  int32_t dtype;         /* milo_dtype */
+  int32_t reserved;
+  const int32_t* ranks;       /* device [2H][nb]                         */
+  const int64_t* row_offsets; /* device [2H][nb+1]                       */
+  const void* tok;            /* device [2H*pool_rows][n]                */
+  const void* dim;            /* device [2H*pool_rows][d]                */
+  /* present only with MILO_KEEP_INTERMEDIATES, else NULL: */
+  const float* eigvals;       /* device [2H][nb][d], descending (λ_i = σ_i²)           */
+  const float* eigvecs;       /* device [2H][nb][d][d], row i = eigenvector of λ_i      */
+  const double* entropy;      /* device [2H][nb], H_b                                  */
+  const double* quotas;       /* device [2H][nb], real quotas before rounding          */
+} milo_factors_desc;
+
+/*
+ * milo_compress — encode one layer's KV cache into per-block low-rank factors.
+ * Source: §4.2 (block partition, separate low-rank approximation of each
+ * block's keys and values) and §4.3 (ranks from block entropy under a total
+ * budget).  Steps, all on `stream`: per block the Gram matrix X_bᵀX_b (fp32),
+ * its eigen-decomposition by one-sided Jacobi (λ_i = σ_i², eigenvectors = the
+ * right singular vectors), the spectral entropy H_b = −Σ p_i ln p_i with
+ * p_i = λ_i/Σλ, ranks ∝ exp(H_b) summing to R = floor(budget·T·d/(n+d)) per
+ * pool (clamped to [r_min, d], largest-remainder rounding), and the
+ * projection U_b = X_b·B_b[:, :r_b].
+ *   K, V        device [H][T][d] in `dtype`; read only.
+ *   block_size  n: T % n == 0, n >= d.
+ *   head_dim    d ∈ {64, 128}.
+ *   budget      storage budget > 0 (fraction of the raw cache; > 1 allowed).
+ *   r_min       1 <= r_min <= d; MILO_ERR_BUDGET if R < nb*r_min.
+ *   max_sweeps  Jacobi sweep limit, 0 = default (30).  Hitting it sets
+ *               MILO_ERR_NO_CONVERGENCE in the status word (not the return).
+ *   flags       MILO_KEEP_INTERMEDIATES or 0.
+ *   out         receives a new factor object; destroy with milo_factors_destroy.
+ * Allocates device memory (cudaMalloc) for the factor object and its scratch;
+ * does not synchronise.
+ */
+milo_status milo_compress(const void* K, const void* V, int32_t dtype, int32_t num_kv_heads,
+                          int64_t context, int32_t head_dim, int32_t block_size, double budget,
+                          int32_t r_min, int32_t max_sweeps, uint32_t flags, void* stream,
+                          milo_factors** out);
+
+/*
+ * milo_decode_attn — one decode step of softmax attention over the compressed
+ * prefix and each query's uncompressed suffix.
+ * Source: §4.4 (inference attends over the stored low-rank caches).  Every
+ * block is attended (no selection).  Computed in rank space: per block
+ * q̃ = q·B_b, scores = scale·q̃·U_bᵀ, one online softmax over all blocks and
+ * the suffix, value sum (p·P_b)·Q_bᵀ.  Query head hq reads KV head
+ * hq / (num_q_heads / H).
+ *   q         device [batch][num_q_heads][d], dtype of the factors.
+ *   f         factor object from milo_compress or milo_factors_import.
+ *   K_suffix, V_suffix  device [batch][H][suffix_len][d]; may be NULL when
+ *             suffix_len == 0.
+ *   scale     softmax scale; <= 0 selects 1/sqrt(d).
+ *   out       device [batch][num_q_heads][d], dtype of the factors.
+ * The first call for a given (batch, num_q_heads, suffix_len) synchronises
+ * `stream` once to read the ranks and build the work list, and may allocate
+ * scratch; later calls with the same shape do neither.  Calls that share a
+ * factor object share its scratch and must be ordered on one stream.
+ */
+milo_status milo_decode_attn(const void* q, int32_t batch, int32_t num_q_heads,
+                             const milo_factors* f, const void* K_suffix, const void* V_suffix,
+                             int32_t suffix_len, float scale, void* out, void* stream);
+
+/*
+ * Number of kernels one milo_decode_attn call with these arguments launches
+ * (>= 1), or a negative milo_status for invalid arguments.  Host-only, no GPU work.
+ */
+int32_t milo_decode_launches(const milo_factors* f, int32_t batch, int32_t num_q_heads, int32_t suffix_len);
+
+/* Copies the ranks [2H][nb] to host memory. Synchronises the compress stream. */
+milo_status milo_factors_ranks(const milo_factors* f, int32_t* host_ranks);
+
+/* Fills *desc with the shape and the device pointers of f (valid until destroy). */
+milo_status milo_factors_describe(const milo_factors* f, milo_factors_desc* desc);
+
+/*
+ * Synchronises the device and returns the first error recorded by a kernel
+ * for f (MILO_OK if none).  *host_bits (optional) receives the raw bit mask:
+ * 1 = Jacobi did not converge, 2 = compress bounds check, 4 = decode bounds
+ * check, 8 = decode wait expired.
+ */
+milo_status milo_factors_status(const milo_factors* f, uint32_t* host_bits);
+
+/*
+ * Builds a factor object from host arrays in the layout above (a copy), e.g.
+ * factors computed elsewhere or saved earlier.  host_ranks [2H][nb];
+ * host_tok [2H*pool_rows][n] and host_dim [2H*pool_rows][d] in `dtype`, with
+ * pool_rows = Σ of each pool's ranks (all pools must have the same sum).
+ * Synchronises `stream`.
+ */
+milo_status milo_factors_import(int32_t dtype, int32_t num_kv_heads, int64_t context,
+                                int32_t head_dim, int32_t block_size, int32_t r_min,
+                                const int32_t* host_ranks, const void* host_tok,
+                                const void* host_dim, void* stream, milo_factors** out);
+
+/* Frees f and everything it owns (synchronises the device first). NULL is a no-op. */
+void milo_factors_destroy(milo_factors* f);
+
+const char* milo_status_string(int32_t status);
+int32_t milo_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MILO_H_ */

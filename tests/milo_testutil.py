@@ -1,0 +1,91 @@
+"""Shared helpers of the tests: storage casts, oracle-factor packing, error norms.
+
+Packing turns the oracle's per-block factors into the library's documented
+layout (ranks [2H][nb], tok [rows][n], dim [rows][d]); it is layout plumbing,
+not arithmetic of the method.
+"""
+import numpy as np
+
+import oracle
+from synth import from_storage, to_storage
+
+
+def rel_l2(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+def cast_fn(dtype):
+    return lambda x: from_storage(to_storage(x, dtype), dtype)
+
+
+def stored_layer(layer: dict, dtype: str) -> dict:
+    c = cast_fn(dtype)
+    return dict(K=[oracle.stored_factors(p, c) for p in layer["K"]],
+                V=[oracle.stored_factors(p, c) for p in layer["V"]])
+
+
+def pack_factors(layer: dict, dtype: str):
+    """Oracle layer → (ranks [2H][nb] int32, tok [rows][n], dim [rows][d]) in storage dtype."""
+    H = len(layer["K"])
+    pools = []
+    for h in range(H):
+        pools += [layer["K"][h], layer["V"][h]]
+    ranks = np.array([p["ranks"] for p in pools], dtype=np.int32)
+    tok = np.concatenate([u.T for p in pools for u in p["U"]], axis=0)
+    dim = np.concatenate([b.T for p in pools for b in p["B"]], axis=0)
+    return ranks, to_storage(tok, dtype), to_storage(dim, dtype)
+
+
+def to_torch(arr, dtype: str, device="cuda"):
+    import torch
+    if dtype == "f32":
+        return torch.from_numpy(np.ascontiguousarray(arr, dtype=np.float32)).to(device)
+    return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).to(device).view(torch.bfloat16)
+
+
+def from_torch(t) -> np.ndarray:
+    import torch
+    t = t.detach().cpu()
+    if t.dtype == torch.bfloat16:
+        return from_storage(t.view(torch.int16).numpy().view(np.uint16), "bf16")
+    return t.double().numpy()
+
+
+class _CudaArray:
+    def __init__(self, ptr, shape, typestr):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr, "data": (int(ptr), True),
+                                         "version": 3, "strides": None}
+
+
+def device_view(ptr, shape, typestr):
+    """Zero-copy torch view of library-owned device memory (read it before the owner is destroyed)."""
+    import torch
+    return torch.as_tensor(_CudaArray(ptr, shape, typestr), device="cuda")
+
+
+def factor_arrays(f) -> dict:
+    """Host copies of a factor object's arrays, as fp64 / int numpy arrays."""
+    import torch
+    d = f.describe()
+    H2, nb, n, dd, rows = 2 * d["num_kv_heads"], d["num_blocks"], d["block_size"], d["head_dim"], d["pool_rows"]
+    bf = d["dtype"] == 1
+    out = dict(desc=d)
+    out["ranks"] = device_view(d["ranks"], (H2, nb), "<i4").cpu().numpy()
+    out["row_offsets"] = device_view(d["row_offsets"], (H2, nb + 1), "<i8").cpu().numpy()
+    if bf:
+        tok = device_view(d["tok"], (H2 * rows, n), "<i2").cpu().numpy().view(np.uint16)
+        dim = device_view(d["dim"], (H2 * rows, dd), "<i2").cpu().numpy().view(np.uint16)
+        out["tok"], out["dim"] = from_storage(tok, "bf16"), from_storage(dim, "bf16")
+    else:
+        out["tok"] = device_view(d["tok"], (H2 * rows, n), "<f4").cpu().numpy().astype(np.float64)
+        out["dim"] = device_view(d["dim"], (H2 * rows, dd), "<f4").cpu().numpy().astype(np.float64)
+    if d["eigvals"]:
+        out["eigvals"] = device_view(d["eigvals"], (H2, nb, dd), "<f4").cpu().numpy().astype(np.float64)
+        out["entropy"] = device_view(d["entropy"], (H2, nb), "<f8").cpu().numpy()
+        out["quotas"] = device_view(d["quotas"], (H2, nb), "<f8").cpu().numpy()
+    if d["eigvecs"]:
+        out["eigvecs"] = device_view(d["eigvecs"], (H2, nb, dd, dd), "<f4").cpu().numpy().astype(np.float64)
+    torch.cuda.synchronize()
+    return out

@@ -1,0 +1,74 @@
+"""The C-ABI library loads, exports every symbol its header declares, and rejects bad arguments
+before touching the GPU (these calls return before any CUDA call, so they run on CPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import decode_attention_milo_b200 as milo
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", f)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(milo_\w+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = milo.load_library()
+    names = _declared()
+    assert {"milo_compress", "milo_decode_attn"} <= names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert lib.milo_abi_version() == 1
+    assert lib.milo_status_string(0) == b"ok"
+    assert lib.milo_status_string(3).startswith(b"budget")
+
+
+def _compress(lib, **kw):
+    args = dict(K=1, V=1, dtype=1, H=4, T=32768, d=128, n=512, budget=0.5, r_min=4, sweeps=0, flags=0)
+    args.update(kw)
+    out = ctypes.c_void_p(123)
+    code = lib.milo_compress(ctypes.c_void_p(args["K"]) if args["K"] else None,
+                             ctypes.c_void_p(args["V"]) if args["V"] else None,
+                             args["dtype"], args["H"], args["T"], args["d"], args["n"], args["budget"],
+                             args["r_min"], args["sweeps"], args["flags"], None, ctypes.byref(out))
+    assert out.value is None  # *out cleared on error
+    return code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(K=0), 1), (dict(dtype=7), 1), (dict(H=0), 1), (dict(d=96), 2), (dict(d=0), 1),
+    (dict(T=32769), 1), (dict(n=100), 1), (dict(n=64), 1), (dict(r_min=0), 1), (dict(r_min=129), 1),
+    (dict(budget=0.0), 1), (dict(budget=float("nan")), 1), (dict(sweeps=-1), 1), (dict(flags=8), 1),
+    (dict(budget=0.001), 3),
+])
+def test_compress_rejects_bad_arguments(kw, code):
+    assert _compress(milo.load_library(), **kw) == code
+
+
+def test_decode_rejects_null_arguments():
+    lib = milo.load_library()
+    assert lib.milo_decode_attn(None, 1, 2, None, None, None, 0, 0.0, None, None) == 1
+    assert lib.milo_factors_ranks(None, None) == 1
+    assert lib.milo_factors_status(None, None) == 1
+    lib.milo_factors_destroy(None)
+
+
+def test_import_rejects_unequal_pools():
+    import numpy as np
+    lib = milo.load_library()
+    ranks = np.array([[4, 5], [4, 4]], dtype=np.int32)  # pool sums differ
+    tok = np.zeros(64 * 512, dtype=np.uint16)
+    out = ctypes.c_void_p()
+    code = lib.milo_factors_import(1, 1, 1024, 64, 512, 4, ranks.ctypes.data_as(ctypes.c_void_p),
+                                   tok.ctypes.data_as(ctypes.c_void_p), tok.ctypes.data_as(ctypes.c_void_p),
+                                   None, ctypes.byref(out))
+    assert code == 1
