@@ -16,6 +16,8 @@ struct TcInputs {
   const void* V_suf;
   const void* tok;
   const void* dim;
+  const int32_t* ranks;        // device [2H][nb]
+  const int64_t* row_offsets;  // device [2H][nb+1]
   uint32_t* status;
   int pool_rows;
   const int32_t* host_ranks;  // [2H][nb]

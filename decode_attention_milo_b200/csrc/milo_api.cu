@@ -334,7 +334,8 @@ milo_status milo_decode_attn(const void* q, int32_t batch, int32_t num_q_heads, 
       MILO_CUDA(cudaMemcpy(f->host_ranks.data(), f->ranks, f->host_ranks.size() * sizeof(int32_t),
                            cudaMemcpyDeviceToHost));
     }
-    milo::TcInputs in{q, K_suffix, V_suffix, f->tok, f->dim, f->status, f->pool_rows, f->host_ranks.data()};
+    milo::TcInputs in{q,        K_suffix, V_suffix,     f->tok,       f->dim,
+                      f->ranks, f->row_offsets, f->status, f->pool_rows, f->host_ranks.data()};
     return cuda_status(milo::tc_decode(&f->tc_plan, ds, in, out, s));
   }
   const size_t need = milo::simt_decode_partials_floats(ds);

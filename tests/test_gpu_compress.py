@@ -65,7 +65,11 @@ def test_ranks_bit_exact_and_eckart_young(name):
             bv = got["eigvecs"][p, b, :r].T  # d × r
             err = np.linalg.norm(xb - xb @ bv @ bv.T)
             opt = math.sqrt(float(np.sum(pool["sigma"][b][r:] ** 2)))
-            assert (err - opt) / opt <= 1e-3, (p, b, err, opt)
+            if r < d:
+                assert (err - opt) / opt <= 1e-3, (p, b, err, opt)
+            else:
+                # full rank: the optimum is 0; fp32 eigenvectors are orthonormal to ~1e-6, so allow 1e-4 |X_b|
+                assert err <= 1e-4 * np.linalg.norm(xb), (p, b, err)
 
 
 def test_stored_factors_reconstruct_near_optimum_7b():
