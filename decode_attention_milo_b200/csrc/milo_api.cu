@@ -324,7 +324,11 @@ milo_status milo_decode_attn(const void* q, int32_t batch, int32_t num_q_heads, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)f->d);
   std::lock_guard<std::mutex> lock(f->mu);
-  MILO_CUDA(cudaStreamWaitEvent(s, f->ready, 0));
+  // Order after the factors were written.  Inside a stream capture the factors must already be complete
+  // (an event recorded outside the capture cannot be waited on there), so the wait is skipped.
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  MILO_CUDA(cudaStreamIsCapturing(s, &cap));
+  if (cap == cudaStreamCaptureStatusNone) MILO_CUDA(cudaStreamWaitEvent(s, f->ready, 0));
   milo::DecodeShape ds{f->H, f->nb, f->n, f->d, batch, num_q_heads, suffix_len, f->dtype == MILO_BF16, sc};
   milo::DecodeBuffers db{q, K_suffix, V_suffix, f->ranks, f->row_offsets, f->tok, f->dim, nullptr, out, f->status};
   if (f->dtype == MILO_BF16 && milo::tc_supported(ds)) {

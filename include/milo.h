@@ -132,8 +132,10 @@ milo_status milo_compress(const void* K, const void* V, int32_t dtype, int32_t n
  *   out       device [batch][num_q_heads][d], dtype of the factors.
  * The first call for a given (batch, num_q_heads, suffix_len) synchronises
  * `stream` once to read the ranks and build the work list, and may allocate
- * scratch; later calls with the same shape do neither.  Calls that share a
- * factor object share its scratch and must be ordered on one stream.
+ * scratch; later calls with the same shape do neither, so they can be captured
+ * in a CUDA graph (make one call with the shape before capturing, and let the
+ * factors be complete before the capture starts).  Calls that share a factor
+ * object share its scratch and must be ordered on one stream.
  */
 milo_status milo_decode_attn(const void* q, int32_t batch, int32_t num_q_heads,
                              const milo_factors* f, const void* K_suffix, const void* V_suffix,
