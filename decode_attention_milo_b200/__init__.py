@@ -62,6 +62,8 @@ def load_library(path: str | None = None):
     L.milo_compress.argtypes = [vp, vp, i32, i32, i64, i32, i32, f64, i32, i32, u32, vp, ctypes.POINTER(vp)]
     L.milo_decode_attn.restype = i32
     L.milo_decode_attn.argtypes = [vp, i32, i32, vp, vp, vp, i32, f32, vp, vp]
+    L.milo_decode_attn_profiled.restype = i32
+    L.milo_decode_attn_profiled.argtypes = [vp, i32, i32, vp, vp, vp, i32, f32, vp, vp, vp, vp]
     L.milo_decode_launches.restype = i32
     L.milo_decode_launches.argtypes = [vp, i32, i32, i32]
     L.milo_factors_ranks.restype = i32
@@ -191,6 +193,19 @@ def decode_attn(q, factors: Factors, K_suf=None, V_suf=None, scale: float = 0.0,
                                            _dev_ptr(K_suf, "K_suf") if S else None,
                                            _dev_ptr(V_suf, "V_suf") if S else None, S, float(scale),
                                            _dev_ptr(out, "out"), _stream_ptr(stream)), "milo_decode_attn")
+    return out
+
+
+def decode_attn_profiled(q, factors: Factors, K_suf, V_suf, out, event_before, event_after, scale: float = 0.0,
+                         stream=None):
+    """decode_attn that records two torch.cuda.Event objects around the main decode kernel."""
+    B, Hq, _ = q.shape
+    S = 0 if K_suf is None else K_suf.shape[2]
+    _check(load_library().milo_decode_attn_profiled(
+        _dev_ptr(q, "q"), B, Hq, factors.handle, _dev_ptr(K_suf, "K_suf") if S else None,
+        _dev_ptr(V_suf, "V_suf") if S else None, S, float(scale), _dev_ptr(out, "out"), _stream_ptr(stream),
+        ctypes.c_void_p(event_before.cuda_event), ctypes.c_void_p(event_after.cuda_event)),
+        "milo_decode_attn_profiled")
     return out
 
 

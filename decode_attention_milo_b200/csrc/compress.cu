@@ -11,7 +11,7 @@
 //   alloc    H_b = −Σ p ln p (p = λ/Σλ, fp64), w_b = e^{H_b}, quotas
 //            clamp(lam·w_b, r_min, d) with Σ = R, largest-remainder ranks,
 //            row offsets                                  (one CTA per pool)
-//   project  U_b = X_b · B_b[:, :r_b], stored transposed, and B_bᵀ rows
+//   project  U_b = X_b · B_b[:, :r_b], stored transposed in 128-token slabs, and B_bᵀ rows
 //                                                         (one CTA per block)
 #include <math.h>
 
@@ -349,7 +349,8 @@ __global__ void __launch_bounds__(kThreads) project_kernel(const T* __restrict__
       float acc = 0.f;
 #pragma unroll 8
       for (int c = 0; c < D; ++c) acc = fmaf(xt[c * CH + tt], Bs[j * D + c], acc);
-      tok[(row0 + j) * n + t0 + tt] = from_f32<T>(acc);
+      const int t = t0 + tt;  // chunk-major: [t / 128][j][t % 128] inside the block's slab
+      tok[row0 * n + (int64_t)(t >> 7) * (r * 128) + j * 128 + (t & 127)] = from_f32<T>(acc);
     }
   }
 }

@@ -78,7 +78,8 @@ __global__ void __launch_bounds__(kThreads) prefix_kernel(const T* __restrict__ 
   float mloc = -INFINITY;
   for (int t = threadIdx.x; t < n; t += kThreads) {
     float a = 0.f;
-    for (int j = 0; j < rk; ++j) a = fmaf(qt[j], to_f32(tok[(ok + j) * n + t]), a);
+    const T* col = tok + ok * n + (int64_t)(t >> 7) * (rk * 128) + (t & 127);  // chunk-major slab
+    for (int j = 0; j < rk; ++j) a = fmaf(qt[j], to_f32(col[j * 128]), a);
     a *= scale;
     s[t] = a;
     mloc = fmaxf(mloc, a);
@@ -93,9 +94,9 @@ __global__ void __launch_bounds__(kThreads) prefix_kernel(const T* __restrict__ 
   const float l = block_sum(lloc, red);  // contains __syncthreads: s[] complete below
   // ã = p · P_b
   for (int j = warp; j < rv; j += kThreads / 32) {
-    const T* prow = tok + (ov + j) * n;
+    const T* slab = tok + ov * n + j * 128;
     float a = 0.f;
-    for (int t = lane; t < n; t += 32) a = fmaf(s[t], to_f32(prow[t]), a);
+    for (int t = lane; t < n; t += 32) a = fmaf(s[t], to_f32(slab[(int64_t)(t >> 7) * (rv * 128) + (t & 127)]), a);
     a = warp_sum(a);
     if (lane == 0) qt[j] = a;
   }
@@ -182,7 +183,7 @@ __global__ void __launch_bounds__(D) combine_kernel(const float* __restrict__ pa
 }
 
 template <typename T, int D>
-cudaError_t run(const DecodeShape& s, const DecodeBuffers& b, cudaStream_t st) {
+cudaError_t run(const DecodeShape& s, const DecodeBuffers& b, cudaStream_t st, cudaEvent_t ev0, cudaEvent_t ev1) {
   const int G = s.Hq / s.H, rows = s.Bq * G;
   const T* q = static_cast<const T*>(b.q);
   const size_t psm = (size_t)s.n * sizeof(float);
@@ -191,9 +192,11 @@ cudaError_t run(const DecodeShape& s, const DecodeBuffers& b, cudaStream_t st) {
                                          (int)psm);
     if (e != cudaSuccess) return e;
   }
+  if (ev0) cudaEventRecord(ev0, st);
   prefix_kernel<T, D><<<dim3(rows, s.nb, s.H), kThreads, psm, st>>>(
       q, static_cast<const T*>(b.tok), static_cast<const T*>(b.dim), b.ranks, b.row_offsets, s.H, s.nb, s.n,
       s.Hq, G, s.scale, b.partials, b.status);
+  if (ev1) cudaEventRecord(ev1, st);
   if (s.S > 0) {
     const size_t ssm = (size_t)s.S * sizeof(float);
     if (ssm > 48 * 1024) {
@@ -217,13 +220,14 @@ size_t simt_decode_partials_floats(const DecodeShape& s) {
   return ((size_t)s.H * s.nb * s.Bq * G + (size_t)s.Bq * s.H * G) * (s.d + 2);
 }
 
-cudaError_t launch_decode_simt(const DecodeShape& s, const DecodeBuffers& b, cudaStream_t st) {
+cudaError_t launch_decode_simt(const DecodeShape& s, const DecodeBuffers& b, cudaStream_t st, cudaEvent_t ev0,
+                               cudaEvent_t ev1) {
   if (s.bf16) {
-    if (s.d == 64) return run<__nv_bfloat16, 64>(s, b, st);
-    return run<__nv_bfloat16, 128>(s, b, st);
+    if (s.d == 64) return run<__nv_bfloat16, 64>(s, b, st, ev0, ev1);
+    return run<__nv_bfloat16, 128>(s, b, st, ev0, ev1);
   }
-  if (s.d == 64) return run<float, 64>(s, b, st);
-  return run<float, 128>(s, b, st);
+  if (s.d == 64) return run<float, 64>(s, b, st, ev0, ev1);
+  return run<float, 128>(s, b, st, ev0, ev1);
 }
 
 }  // namespace milo

@@ -240,15 +240,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(bar(B_QFULL), 1);
     ptx::mbar_init(bar(B_QEMPTY), 1);
     ptx::mbar_init(bar(B_QTFULL), 1);
-    ptx::mbar_init(bar(B_QTREADY), 128);
+    ptx::mbar_init(bar(B_QTREADY), 4);
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(bar(B_SFULL + i), 1);
-      ptx::mbar_init(bar(B_SEMPTY + i), 128);
-      ptx::mbar_init(bar(B_PFULL + i), 128);
+      ptx::mbar_init(bar(B_SEMPTY + i), 4);
+      ptx::mbar_init(bar(B_PFULL + i), 4);
       ptx::mbar_init(bar(B_PEMPTY + i), 1);
     }
     ptx::mbar_init(bar(B_ATFULL), 1);
-    ptx::mbar_init(bar(B_ATREADY), 128);
+    ptx::mbar_init(bar(B_ATREADY), 4);
     ptx::mbar_init(bar(B_ACCFULL), 1);
     ptx::mbar_init(bar(B_FINAL), 1);
     sh->abort_flag = 0;
@@ -298,9 +298,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int rkp = pad16(bi.rk), rvp = pad16(bi.rv);
           // consumption order: B_K, U(0), [U(1), P(0)], ..., [U(n-1), P(n-2)], P(n-1), Q_V
           ok = pr.item(&map_dim, 0, bi.rowk, rkp, NCB);
+          // token factor slabs: chunk cc of the block is rows [row0·cpb + cc·r, +r) of the 128-wide view
           for (int cc = c; cc <= cend && ok; ++cc) {
-            if (cc < cend) ok = pr.item(&map_tok, (cc - b * p.cpb) * kChunk, bi.rowk, rkp, 2);
-            if (ok && cc > c) ok = pr.item(&map_tok, (cc - 1 - b * p.cpb) * kChunk, bi.rowv, rvp, 2);
+            if (cc < cend) ok = pr.item(&map_tok, 0, bi.rowk * p.cpb + (int64_t)(cc - b * p.cpb) * bi.rk, rkp, 2);
+            if (ok && cc > c)
+              ok = pr.item(&map_tok, 0, bi.rowv * p.cpb + (int64_t)(cc - 1 - b * p.cpb) * bi.rv, rvp, 2);
           }
           if (ok) ok = pr.item(&map_dim, 0, bi.rowv, rvp, NCB);
           c = cend;
@@ -507,8 +509,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem + ((uint32_t)(32 * quarter) << 16);
     uint32_t chunk_ix = 0, qt_uses = 0, at_uses = 0, acc_uses = 0;
     bool ok = true;
+    // one arrival per warp on the barriers the warpgroup signals (init count 4)
+    auto arrive = [&](int b) {
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(b));
+    };
     for (int si = s_begin; si < s_end && ok; ++si) {
       const Seg sg = p.segs[si];
+      // a warp whose 32 rows are all padding only keeps the barrier protocol
+      const bool active = 32 * quarter < sg.rows;
       float m_used = -INFINITY, l = 0.f;
       bool first_chunk = true;
       const bool prefix = sg.type == 0;
@@ -531,28 +540,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = wait_bar(bar(B_QTFULL), qt_uses & 1, sh, p.status))) break;
           ++qt_uses;
           ptx::tc_fence_after();
-          for (int c16 = 0; c16 < rkp; c16 += 16) {
-            float v[16];
-            ptx::tmem_ld16(tl + kTmR + c16, v);
-            ptx::tmem_wait_ld();
-            uint32_t hi[8], lo[8];
+          if (active) {
+            for (int half = 0; half < rkp; half += 64) {
+              float v[64];
 #pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              const float a = (c16 + e < rk) ? v[e] : 0.f;
-              const float b2 = (c16 + e + 1 < rk) ? v[e + 1] : 0.f;
-              const uint32_t h2 = ptx::pack_bf16(a, b2);
-              const float ah = __uint_as_float(h2 << 16), bh = __uint_as_float(h2 & 0xFFFF0000u);
-              hi[e / 2] = h2;
-              lo[e / 2] = ptx::pack_bf16(a - ah, b2 - bh);
+              for (int q = 0; q < 4; ++q) ptx::tmem_ld16(tl + kTmR + half + 16 * q, v + 16 * q);
+              ptx::tmem_wait_ld();
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int col = half + 16 * q;
+                if (col < rkp) {
+                  uint32_t hi[8], lo[8];
+#pragma unroll
+                  for (int e = 0; e < 16; e += 2) {
+                    const float a = (col + e < rk) ? v[16 * q + e] : 0.f;
+                    const float b2 = (col + e + 1 < rk) ? v[16 * q + e + 1] : 0.f;
+                    const uint32_t h2 = ptx::pack_bf16(a, b2);
+                    hi[e / 2] = h2;
+                    lo[e / 2] =
+                        ptx::pack_bf16(a - __uint_as_float(h2 << 16), b2 - __uint_as_float(h2 & 0xFFFF0000u));
+                  }
+                  st_tile8(base + kOffQtHi, row, col, hi[0], hi[1], hi[2], hi[3]);
+                  st_tile8(base + kOffQtHi, row, col + 8, hi[4], hi[5], hi[6], hi[7]);
+                  st_tile8(base + kOffQtLo, row, col, lo[0], lo[1], lo[2], lo[3]);
+                  st_tile8(base + kOffQtLo, row, col + 8, lo[4], lo[5], lo[6], lo[7]);
+                }
+              }
             }
-            st_tile8(base + kOffQtHi, row, c16, hi[0], hi[1], hi[2], hi[3]);
-            st_tile8(base + kOffQtHi, row, c16 + 8, hi[4], hi[5], hi[6], hi[7]);
-            st_tile8(base + kOffQtLo, row, c16, lo[0], lo[1], lo[2], lo[3]);
-            st_tile8(base + kOffQtLo, row, c16 + 8, lo[4], lo[5], lo[6], lo[7]);
+            ptx::fence_async_smem();
           }
-          ptx::fence_async_smem();
           ptx::tc_fence_before();
-          ptx::mbar_arrive(bar(B_QTREADY));
+          arrive(B_QTREADY);
         } else {
           cend = sg.c1;
         }
@@ -562,30 +580,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = wait_bar(bar(B_SFULL + slot), (k >> 1) & 1, sh, p.status))) break;
           ptx::tc_fence_after();
           float s[kChunk];
+          if (active) {
 #pragma unroll
-          for (int q = 0; q < kChunk / 16; ++q) ptx::tmem_ld16(tl + kTmS0 + 128 * slot + 16 * q, s + 16 * q);
-          ptx::tmem_wait_ld();
+            for (int q = 0; q < kChunk / 16; ++q) ptx::tmem_ld16(tl + kTmS0 + 128 * slot + 16 * q, s + 16 * q);
+            ptx::tmem_wait_ld();
+          }
           ptx::tc_fence_before();
-          ptx::mbar_arrive(bar(B_SEMPTY + slot));
-          if (!prefix) {
-            const int valid = p.S - cc * kChunk;
-#pragma unroll
-            for (int j = 0; j < kChunk; ++j)
-              if (j >= valid) s[j] = -INFINITY;
-          }
-          float mx = -INFINITY;
-#pragma unroll
-          for (int j = 0; j < kChunk; ++j) mx = fmaxf(mx, s[j]);
-          mx *= p.c;
-          // running max: keep the one in use unless the chunk exceeds it by more than 2^8 (then rescale)
-          const bool grow = !first_chunk && mx > m_used + 8.f;
+          arrive(B_SEMPTY + slot);
           float alpha = 1.f;
-          if (grow) {
-            alpha = ptx::ex2(m_used - mx);
-            m_used = mx;
-            l *= alpha;
+          bool grow = false;
+          if (active) {
+            if (!prefix) {
+              const int valid = p.S - cc * kChunk;
+#pragma unroll
+              for (int j = 0; j < kChunk; ++j)
+                if (j >= valid) s[j] = -INFINITY;
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < kChunk; ++j) mx = fmaxf(mx, s[j]);
+            mx *= p.c;
+            // keep the running max in use unless the chunk exceeds it by more than 2^8 (then rescale)
+            grow = !first_chunk && mx > m_used + 8.f;
+            if (grow) {
+              alpha = ptx::ex2(m_used - mx);
+              m_used = mx;
+              l *= alpha;
+            }
+            if (first_chunk) m_used = mx;
           }
-          if (first_chunk) m_used = mx;
           if (__any_sync(0xffffffffu, grow)) {
             // rare: rescale what this warp's rows accumulated so far (alpha = 1 for rows that did not grow)
             const bool have_at = prefix && cc > c;  // ã holds earlier chunks of this block
@@ -620,24 +643,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           first_chunk = false;
           // p = exp2(S·c − m), row sum, bf16 tile
           if (!(ok = wait_bar(bar(B_PEMPTY + slot), ((k >> 1) & 1) ^ 1, sh, p.status))) break;
-          const uint32_t pt = base + kOffP + 32768 * slot;
-          float lsum = 0.f;
+          if (active) {
+            const uint32_t pt = base + kOffP + 32768 * slot;
+            float lsum = 0.f;
 #pragma unroll
-          for (int g8 = 0; g8 < kChunk / 8; ++g8) {
-            uint32_t w[4];
+            for (int g8 = 0; g8 < kChunk / 8; ++g8) {
+              uint32_t w[4];
 #pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-              const float a = ptx::ex2(fmaf(s[8 * g8 + e], p.c, -m_used));
-              const float b2 = ptx::ex2(fmaf(s[8 * g8 + e + 1], p.c, -m_used));
-              lsum += a + b2;
-              w[e / 2] = ptx::pack_bf16(a, b2);
+              for (int e = 0; e < 8; e += 2) {
+                const float a = ptx::ex2(fmaf(s[8 * g8 + e], p.c, -m_used));
+                const float b2 = ptx::ex2(fmaf(s[8 * g8 + e + 1], p.c, -m_used));
+                lsum += a + b2;
+                w[e / 2] = ptx::pack_bf16(a, b2);
+              }
+              st_tile8(pt, row, 8 * g8, w[0], w[1], w[2], w[3]);
             }
-            st_tile8(pt, row, 8 * g8, w[0], w[1], w[2], w[3]);
+            l += lsum;
+            ptx::fence_async_smem();
           }
-          l += lsum;
-          ptx::fence_async_smem();
           ptx::tc_fence_before();
-          ptx::mbar_arrive(bar(B_PFULL + slot));
+          arrive(B_PFULL + slot);
           ++chunk_ix;
         }
         if (!ok) break;
@@ -646,20 +671,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = wait_bar(bar(B_ATFULL), at_uses & 1, sh, p.status))) break;
           ++at_uses;
           ptx::tc_fence_after();
-          for (int c16 = 0; c16 < rvp; c16 += 16) {
-            float v[16];
-            ptx::tmem_ld16(tl + kTmR + c16, v);
-            ptx::tmem_wait_ld();
-            uint32_t w[8];
+          if (active) {
+            for (int half = 0; half < rvp; half += 64) {
+              float v[64];
 #pragma unroll
-            for (int e = 0; e < 16; e += 2)
-              w[e / 2] = ptx::pack_bf16(c16 + e < rv ? v[e] : 0.f, c16 + e + 1 < rv ? v[e + 1] : 0.f);
-            st_tile8(base + kOffQtHi, row, c16, w[0], w[1], w[2], w[3]);
-            st_tile8(base + kOffQtHi, row, c16 + 8, w[4], w[5], w[6], w[7]);
+              for (int q = 0; q < 4; ++q) ptx::tmem_ld16(tl + kTmR + half + 16 * q, v + 16 * q);
+              ptx::tmem_wait_ld();
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int col = half + 16 * q;
+                if (col < rvp) {
+                  uint32_t w[8];
+#pragma unroll
+                  for (int e = 0; e < 16; e += 2)
+                    w[e / 2] = ptx::pack_bf16(col + e < rv ? v[16 * q + e] : 0.f,
+                                              col + e + 1 < rv ? v[16 * q + e + 1] : 0.f);
+                  st_tile8(base + kOffQtHi, row, col, w[0], w[1], w[2], w[3]);
+                  st_tile8(base + kOffQtHi, row, col + 8, w[4], w[5], w[6], w[7]);
+                }
+              }
+            }
+            ptx::fence_async_smem();
           }
-          ptx::fence_async_smem();
           ptx::tc_fence_before();
-          ptx::mbar_arrive(bar(B_ATREADY));
+          arrive(B_ATREADY);
         }
         c = cend;
         first_block = false;
@@ -669,19 +704,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = wait_bar(bar(B_ACCFULL), acc_uses & 1, sh, p.status))) break;
       ++acc_uses;
       ptx::tc_fence_after();
-      float* dst = p.part_acc + ((int64_t)sg.pid * 128 + row) * D;
-#pragma unroll 1
-      for (int c16 = 0; c16 < D; c16 += 16) {
-        float v[16];
-        ptx::tmem_ld16(tl + kTmAcc + c16, v);
-        ptx::tmem_wait_ld();
-        if (row < sg.rows) {
+      if (active) {
+        float* dst = p.part_acc + ((int64_t)sg.pid * 128 + row) * D;
+        for (int half = 0; half < D; half += 64) {
+          float v[64];
 #pragma unroll
-          for (int e = 0; e < 16; e += 4)
-            *reinterpret_cast<float4*>(dst + c16 + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+          for (int q = 0; q < 4; ++q) ptx::tmem_ld16(tl + kTmAcc + half + 16 * q, v + 16 * q);
+          ptx::tmem_wait_ld();
+          if (row < sg.rows) {
+#pragma unroll
+            for (int e = 0; e < 64; e += 4)
+              *reinterpret_cast<float4*>(dst + half + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+          }
         }
+        if (row < sg.rows) p.part_ml[(int64_t)sg.pid * 128 + row] = make_float2(m_used, l);
       }
-      if (row < sg.rows) p.part_ml[(int64_t)sg.pid * 128 + row] = make_float2(m_used, l);
       ptx::tc_fence_before();
     }
   }
@@ -693,35 +730,70 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) ptx::tmem_dealloc(tmem, 512);
 }
 
-// Merges the partials of one output row (i, hq).
+// Merges the partials of one output row (i, hq): m = max m_k, l = Σ l_k 2^{m_k−m},
+// out = Σ acc_k 2^{m_k−m} / l.  The (m, l) pairs are read in parallel first, so the
+// acc loads of the second phase are independent of each other.
+constexpr int kMaxParts = 1024;
 template <int D>
 __global__ void __launch_bounds__(D) combine_tc_kernel(const float* __restrict__ part_acc,
                                                       const float2* __restrict__ part_ml,
                                                       const int* __restrict__ pre_range,
                                                       const int* __restrict__ suf_range, int H, int Hq, int ipt,
                                                       int nrt, __nv_bfloat16* __restrict__ out) {
+  __shared__ float wgt[kMaxParts];
+  __shared__ int src[kMaxParts];
+  __shared__ float red[D / 32];
+  __shared__ float s_m, s_l;
   const int hq = blockIdx.x, i = blockIdx.y, c = threadIdx.x;
   const int G = Hq / H, h = hq / G, g = hq % G;
   const int rt = i / ipt, prow = (i % ipt) * G + g;
   const int p0 = pre_range[2 * (h * nrt + rt)], p1 = pre_range[2 * (h * nrt + rt) + 1];
   const int s0 = suf_range[2 * (i * H + h)], s1 = suf_range[2 * (i * H + h) + 1];
-  float m = -INFINITY;
-  for (int q = p0; q < p1; ++q) m = fmaxf(m, part_ml[(int64_t)q * 128 + prow].x);
-  for (int q = s0; q < s1; ++q) m = fmaxf(m, part_ml[(int64_t)q * 128 + g].x);
-  float l = 0.f, acc = 0.f;
-  for (int q = p0; q < p1; ++q) {
-    const float2 ml = part_ml[(int64_t)q * 128 + prow];
-    const float w = exp2f(ml.x - m);
-    l = fmaf(ml.y, w, l);
-    acc = fmaf(part_acc[((int64_t)q * 128 + prow) * D + c], w, acc);
+  const int npre = p1 - p0, nall = npre + (s1 - s0);
+  float mloc = -INFINITY;
+  for (int t = c; t < nall; t += D) {
+    const int idx = t < npre ? (p0 + t) * 128 + prow : (s0 + t - npre) * 128 + g;
+    src[t] = idx;
+    const float2 ml = part_ml[idx];
+    wgt[t] = ml.x;
+    mloc = fmaxf(mloc, ml.x);
   }
-  for (int q = s0; q < s1; ++q) {
-    const float2 ml = part_ml[(int64_t)q * 128 + g];
-    const float w = exp2f(ml.x - m);
-    l = fmaf(ml.y, w, l);
-    acc = fmaf(part_acc[((int64_t)q * 128 + g) * D + c], w, acc);
+  mloc = warp_max(mloc);
+  if ((c & 31) == 0) red[c / 32] = mloc;
+  __syncthreads();
+  if (c == 0) {
+    float m = red[0];
+    for (int w = 1; w < D / 32; ++w) m = fmaxf(m, red[w]);
+    s_m = m;
   }
-  out[((int64_t)i * Hq + hq) * D + c] = __float2bfloat16_rn(acc / l);
+  __syncthreads();
+  const float m = s_m;
+  float lloc = 0.f;
+  for (int t = c; t < nall; t += D) {
+    const float w = exp2f(wgt[t] - m);
+    wgt[t] = w;
+    lloc = fmaf(part_ml[src[t]].y, w, lloc);
+  }
+  lloc = warp_sum(lloc);
+  __syncthreads();
+  if ((c & 31) == 0) red[c / 32] = lloc;
+  __syncthreads();
+  if (c == 0) {
+    float l = 0.f;
+    for (int w = 0; w < D / 32; ++w) l += red[w];
+    s_l = l;
+  }
+  __syncthreads();
+  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+  int t = 0;
+  for (; t + 4 <= nall; t += 4) {
+    acc0 = fmaf(part_acc[(int64_t)src[t] * D + c], wgt[t], acc0);
+    acc1 = fmaf(part_acc[(int64_t)src[t + 1] * D + c], wgt[t + 1], acc1);
+    acc2 = fmaf(part_acc[(int64_t)src[t + 2] * D + c], wgt[t + 2], acc2);
+    acc3 = fmaf(part_acc[(int64_t)src[t + 3] * D + c], wgt[t + 3], acc3);
+  }
+  for (; t < nall; ++t) acc0 = fmaf(part_acc[(int64_t)src[t] * D + c], wgt[t], acc0);
+  out[((int64_t)i * Hq + hq) * D + c] = __float2bfloat16_rn(((acc0 + acc1) + (acc2 + acc3)) / s_l);
 }
 
 // ------------------------------------------------------------------------------------------------ host
@@ -855,6 +927,13 @@ static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& 
   }
   for (int i = 0; i < 2 * H * nrt; ++i)
     if (pre_range[i] < 0) pre_range[i] = 0;
+  for (int h = 0; h < H; ++h)
+    for (int i = 0; i < Bq; ++i) {
+      const int rt = i / ipt;
+      const int parts = pre_range[2 * (h * nrt + rt) + 1] - pre_range[2 * (h * nrt + rt)] +
+                        suf_range[2 * (i * H + h) + 1] - suf_range[2 * (i * H + h)];
+      if (parts > kMaxParts) return cudaErrorInvalidValue;
+    }
   pl->off_segs = grid + 1;
   pl->off_pre = pl->off_segs + (int)segs.size() * (int)(sizeof(Seg) / sizeof(int));
   pl->off_suf = pl->off_pre + 2 * H * nrt;
@@ -881,7 +960,8 @@ static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& 
   // factor maps
   const uint64_t rows = (uint64_t)2 * H * in.pool_rows;
   {
-    const uint64_t dims[2] = {(uint64_t)s.n, rows}, st[1] = {(uint64_t)s.n * 2};
+    // the token factor as a [rows · n/128][128] array of 128-token slab rows
+    const uint64_t dims[2] = {(uint64_t)kChunk, rows * cpb}, st[1] = {(uint64_t)kChunk * 2};
     const uint32_t box[2] = {64, 16};
     if (!make_map(&pl->map_tok, in.tok, 2, dims, st, box)) return cudaErrorInvalidValue;
   }
@@ -896,7 +976,8 @@ static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& 
   return cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
 }
 
-cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, void* out, cudaStream_t st) {
+cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, void* out, cudaStream_t st,
+                      cudaEvent_t ev0, cudaEvent_t ev1) {
   TcPlan* pl = *plan;
   if (!pl || pl->Bq != s.Bq || pl->Hq != s.Hq || pl->S != s.S || pl->tok != in.tok) {
     tc_plan_destroy(pl);
@@ -943,13 +1024,16 @@ cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, v
   p.ipt = pl->ipt;
   p.S = s.S;
   p.c = s.scale * 1.4426950408889634f;
+  cudaError_t e;
+  if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
   if (D == 64)
     decode_tc_kernel<64><<<pl->grid, kThreads, kSmemBytes, st>>>(pl->map_tok, pl->map_dim, mq_pre, mq_suf, mk, mv, p);
   else
     decode_tc_kernel<128><<<pl->grid, kThreads, kSmemBytes, st>>>(pl->map_tok, pl->map_dim, mq_pre, mq_suf, mk, mv,
                                                                    p);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (ev1 && (e = cudaEventRecord(ev1, st)) != cudaSuccess) return e;
   const int* pre = pl->d_work + pl->off_pre;
   const int* suf = pl->d_work + pl->off_suf;
   if (D == 64)

@@ -25,7 +25,9 @@ struct TcInputs {
 
 bool tc_supported(const DecodeShape& s);
 int tc_launches(const DecodeShape& s);
-cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, void* out, cudaStream_t st);
+// ev0 / ev1 (optional) are recorded on `st` right before and right after the main decode kernel.
+cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, void* out, cudaStream_t st,
+                      cudaEvent_t ev0 = nullptr, cudaEvent_t ev1 = nullptr);
 void tc_plan_destroy(TcPlan* plan);
 
 }  // namespace milo

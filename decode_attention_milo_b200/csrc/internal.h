@@ -55,6 +55,8 @@ struct DecodeBuffers {
   uint32_t* status;
 };
 size_t simt_decode_partials_floats(const DecodeShape& s);
-cudaError_t launch_decode_simt(const DecodeShape& s, const DecodeBuffers& b, cudaStream_t st);
+// ev0 / ev1 (optional) are recorded on `st` right before and right after the per-block kernel.
+cudaError_t launch_decode_simt(const DecodeShape& s, const DecodeBuffers& b, cudaStream_t st,
+                               cudaEvent_t ev0 = nullptr, cudaEvent_t ev1 = nullptr);
 
 }  // namespace milo

@@ -75,7 +75,7 @@ bool valid_dtype(int32_t dt) { return dt == MILO_F32 || dt == MILO_BF16; }
 milo_status check_layer_shape(int32_t dtype, int32_t H, int64_t T, int32_t d, int32_t n, int32_t r_min) {
   if (!valid_dtype(dtype) || H <= 0 || T <= 0 || n <= 0 || r_min < 1) return MILO_ERR_INVALID_ARGUMENT;
   if (d != 64 && d != 128) return d > 0 ? MILO_ERR_UNSUPPORTED : MILO_ERR_INVALID_ARGUMENT;
-  if (T % n != 0 || n < d || n % 64 != 0 || r_min > d) return MILO_ERR_INVALID_ARGUMENT;
+  if (T % n != 0 || n < d || n % 128 != 0 || r_min > d) return MILO_ERR_INVALID_ARGUMENT;
   if (T / n > (1 << 20) || H > 1024) return MILO_ERR_INVALID_ARGUMENT;
   return MILO_OK;
 }
@@ -312,9 +312,9 @@ int32_t milo_decode_launches(const milo_factors* f, int32_t batch, int32_t num_q
   return suffix_len > 0 ? 3 : 2;
 }
 
-milo_status milo_decode_attn(const void* q, int32_t batch, int32_t num_q_heads, const milo_factors* fc,
-                             const void* K_suffix, const void* V_suffix, int32_t suffix_len, float scale,
-                             void* out, void* stream) {
+static milo_status decode_impl(const void* q, int32_t batch, int32_t num_q_heads, const milo_factors* fc,
+                               const void* K_suffix, const void* V_suffix, int32_t suffix_len, float scale,
+                               void* out, void* stream, cudaEvent_t ev0, cudaEvent_t ev1) {
   if (!fc || !q || !out || batch <= 0 || num_q_heads <= 0 || suffix_len < 0) return MILO_ERR_INVALID_ARGUMENT;
   milo_factors* f = const_cast<milo_factors*>(fc);
   if (num_q_heads % f->H != 0) return MILO_ERR_INVALID_ARGUMENT;
@@ -340,7 +340,7 @@ milo_status milo_decode_attn(const void* q, int32_t batch, int32_t num_q_heads, 
     }
     milo::TcInputs in{q,        K_suffix, V_suffix,     f->tok,       f->dim,
                       f->ranks, f->row_offsets, f->status, f->pool_rows, f->host_ranks.data()};
-    return cuda_status(milo::tc_decode(&f->tc_plan, ds, in, out, s));
+    return cuda_status(milo::tc_decode(&f->tc_plan, ds, in, out, s, ev0, ev1));
   }
   const size_t need = milo::simt_decode_partials_floats(ds);
   if (need > f->partials_floats) {
@@ -352,7 +352,21 @@ milo_status milo_decode_attn(const void* q, int32_t batch, int32_t num_q_heads, 
     f->partials_floats = need;
   }
   db.partials = f->partials;
-  return cuda_status(milo::launch_decode_simt(ds, db, s));
+  return cuda_status(milo::launch_decode_simt(ds, db, s, ev0, ev1));
+}
+
+milo_status milo_decode_attn(const void* q, int32_t batch, int32_t num_q_heads, const milo_factors* f,
+                             const void* K_suffix, const void* V_suffix, int32_t suffix_len, float scale,
+                             void* out, void* stream) {
+  return decode_impl(q, batch, num_q_heads, f, K_suffix, V_suffix, suffix_len, scale, out, stream, nullptr,
+                     nullptr);
+}
+
+milo_status milo_decode_attn_profiled(const void* q, int32_t batch, int32_t num_q_heads, const milo_factors* f,
+                                      const void* K_suffix, const void* V_suffix, int32_t suffix_len, float scale,
+                                      void* out, void* stream, void* event_before, void* event_after) {
+  return decode_impl(q, batch, num_q_heads, f, K_suffix, V_suffix, suffix_len, scale, out, stream,
+                     static_cast<cudaEvent_t>(event_before), static_cast<cudaEvent_t>(event_after));
 }
 
 }  // extern "C"

@@ -29,15 +29,16 @@
  *
  * Layout of a factor object (one layer):
  *   pool p = 2*h + t for KV head h and tensor t (0 = keys, 1 = values);
- *   block b of pool p holds ranks[p*nb + b] = r rows in two row arrays that
- *   share one row index space:
- *     tok [rows][n]  token-side factor, transposed: row j of block b is
- *                    column j of U_b = X_b · B_b  (X_b the n×d block)
- *     dim [rows][d]  dimension-side factor: row j is column j of B_b
- *   so that X_b ≈ U_b · B_bᵀ = Σ_j tok[row0+j]ᵀ · dim[row0+j].  The rows of
- *   block b start at row_offsets[p*(nb+1) + b]; the blocks of a pool are
- *   consecutive and pool p starts at row p * pool_rows.  Factor elements have
- *   the dtype of the compressed cache.
+ *   block b of pool p has rank r = ranks[p*nb + b] and owns rows
+ *   [row0, row0 + r), row0 = row_offsets[p*(nb+1) + b], of two arrays:
+ *     dim  [rows][d]  dimension-side factor: row row0+j is column j of B_b
+ *     tok  r·n elements from element row0·n: the token-side factor
+ *          U_b = X_b·B_b (X_b the n×d block) transposed and cut into
+ *          128-token slabs, element (j, t) at
+ *          row0·n + (t / 128)·(r·128) + j·128 + (t % 128)
+ *   so that X_b ≈ U_b · B_bᵀ.  The blocks of a pool are consecutive and pool p
+ *   starts at row p * pool_rows.  Factor elements have the dtype of the
+ *   compressed cache.
  */
 #ifndef MILO_H_
 #define MILO_H_
@@ -80,7 +81,7 @@ typedef struct {
   int32_t reserved;
   const int32_t* ranks;       /* device [2H][nb]                         */
   const int64_t* row_offsets; /* device [2H][nb+1]                       */
-  const void* tok;            /* device [2H*pool_rows][n]                */
+  const void* tok;            /* device, 2H*pool_rows*n elements (slabs)  */
   const void* dim;            /* device [2H*pool_rows][d]                */
   /* present only with MILO_KEEP_INTERMEDIATES, else NULL: */
   const float* eigvals;       /* device [2H][nb][d], descending (λ_i = σ_i²)           */
@@ -100,7 +101,7 @@ typedef struct {
  * pool (clamped to [r_min, d], largest-remainder rounding), and the
  * projection U_b = X_b·B_b[:, :r_b].
  *   K, V        device [H][T][d] in `dtype`; read only.
- *   block_size  n: T % n == 0, n >= d.
+ *   block_size  n: T % n == 0, n % 128 == 0, n >= d.
  *   head_dim    d ∈ {64, 128}.
  *   budget      storage budget > 0 (fraction of the raw cache; > 1 allowed).
  *   r_min       1 <= r_min <= d; MILO_ERR_BUDGET if R < nb*r_min.
@@ -142,6 +143,19 @@ milo_status milo_decode_attn(const void* q, int32_t batch, int32_t num_q_heads,
                              int32_t suffix_len, float scale, void* out, void* stream);
 
 /*
+ * milo_decode_attn_profiled — milo_decode_attn that also records two caller-created
+ * CUDA events (cudaEvent_t passed as void*, NULL = skip) on `stream`: event_before
+ * right before the main per-block decode kernel and event_after right after it,
+ * before the combine kernel, so cudaEventElapsedTime gives that kernel's duration.
+ * Same arguments, results and errors as milo_decode_attn otherwise.
+ */
+milo_status milo_decode_attn_profiled(const void* q, int32_t batch, int32_t num_q_heads,
+                                      const milo_factors* f, const void* K_suffix,
+                                      const void* V_suffix, int32_t suffix_len, float scale,
+                                      void* out, void* stream, void* event_before,
+                                      void* event_after);
+
+/*
  * Number of kernels one milo_decode_attn call with these arguments launches
  * (>= 1), or a negative milo_status for invalid arguments.  Host-only, no GPU work.
  */
@@ -165,7 +179,8 @@ milo_status milo_factors_status(const milo_factors* f, uint32_t* host_bits);
  * Builds a factor object from host arrays in the layout above (a copy), e.g.
  * factors computed elsewhere or saved earlier.  host_ranks [2H][nb];
  * host_tok [2H*pool_rows][n] and host_dim [2H*pool_rows][d] in `dtype`, with
- * pool_rows = Σ of each pool's ranks (all pools must have the same sum).
+ * pool_rows = Σ of each pool's ranks (all pools must have the same sum);
+ * host_tok holds each block's 128-token slabs as described above.
  * Synchronises `stream`.
  */
 milo_status milo_factors_import(int32_t dtype, int32_t num_kv_heads, int64_t context,

@@ -26,14 +26,28 @@ def stored_layer(layer: dict, dtype: str) -> dict:
                 V=[oracle.stored_factors(p, c) for p in layer["V"]])
 
 
+SLAB = 128  # tokens per slab of the token-side factor
+
+
+def tok_slabs(u: np.ndarray) -> np.ndarray:
+    """U_b (n × r) → the library's slab order: [n/128][r][128] flattened to (n/128·r, 128)."""
+    n, r = u.shape
+    return u.T.reshape(r, n // SLAB, SLAB).transpose(1, 0, 2).reshape(-1, SLAB)
+
+
+def untok_slabs(flat: np.ndarray, n: int, r: int) -> np.ndarray:
+    """Inverse of tok_slabs: r·n elements → U_b (n × r)."""
+    return flat.reshape(n // SLAB, r, SLAB).transpose(1, 0, 2).reshape(r, n).T
+
+
 def pack_factors(layer: dict, dtype: str):
-    """Oracle layer → (ranks [2H][nb] int32, tok [rows][n], dim [rows][d]) in storage dtype."""
+    """Oracle layer → (ranks [2H][nb] int32, tok (Σr·n/128, 128), dim [rows][d]) in storage dtype."""
     H = len(layer["K"])
     pools = []
     for h in range(H):
         pools += [layer["K"][h], layer["V"][h]]
     ranks = np.array([p["ranks"] for p in pools], dtype=np.int32)
-    tok = np.concatenate([u.T for p in pools for u in p["U"]], axis=0)
+    tok = np.concatenate([tok_slabs(u) for p in pools for u in p["U"]], axis=0)
     dim = np.concatenate([b.T for p in pools for b in p["B"]], axis=0)
     return ranks, to_storage(tok, dtype), to_storage(dim, dtype)
 
@@ -75,11 +89,11 @@ def factor_arrays(f) -> dict:
     out["ranks"] = device_view(d["ranks"], (H2, nb), "<i4").cpu().numpy()
     out["row_offsets"] = device_view(d["row_offsets"], (H2, nb + 1), "<i8").cpu().numpy()
     if bf:
-        tok = device_view(d["tok"], (H2 * rows, n), "<i2").cpu().numpy().view(np.uint16)
+        tok = device_view(d["tok"], (H2 * rows * n,), "<i2").cpu().numpy().view(np.uint16)
         dim = device_view(d["dim"], (H2 * rows, dd), "<i2").cpu().numpy().view(np.uint16)
         out["tok"], out["dim"] = from_storage(tok, "bf16"), from_storage(dim, "bf16")
     else:
-        out["tok"] = device_view(d["tok"], (H2 * rows, n), "<f4").cpu().numpy().astype(np.float64)
+        out["tok"] = device_view(d["tok"], (H2 * rows * n,), "<f4").cpu().numpy().astype(np.float64)
         out["dim"] = device_view(d["dim"], (H2 * rows, dd), "<f4").cpu().numpy().astype(np.float64)
     if d["eigvals"]:
         out["eigvals"] = device_view(d["eigvals"], (H2, nb, dd), "<f4").cpu().numpy().astype(np.float64)

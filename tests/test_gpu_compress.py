@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 
 import oracle
-from milo_testutil import factor_arrays, from_torch, rel_l2, to_torch
+from milo_testutil import factor_arrays, from_torch, rel_l2, to_torch, untok_slabs
 from synth import WORKLOADS, from_storage, gen_layer
 
 pytestmark = pytest.mark.gpu
@@ -82,7 +82,8 @@ def test_stored_factors_reconstruct_near_optimum_7b():
         X = (K if p % 2 == 0 else V)[p // 2]
         for b in range(wl.num_blocks):
             r0, r1 = got["row_offsets"][p, b], got["row_offsets"][p, b + 1]
-            rec = got["tok"][r0:r1].T @ got["dim"][r0:r1]
+            u = untok_slabs(got["tok"][r0 * n:r1 * n], n, r1 - r0)
+            rec = u @ got["dim"][r0:r1]
             xb = X[b * n:(b + 1) * n]
             opt = math.sqrt(float(np.sum(pools[p]["sigma"][b][r1 - r0:] ** 2)))
             err = np.linalg.norm(xb - rec)

@@ -58,3 +58,17 @@ def test_tiny_layer_shapes():
     assert L["K_suf"].shape == (1, 1, 0, 64)
     q = gen_queries(wl, 0)
     assert abs(q.std() - 1.0) < 0.3
+
+
+def test_token_slab_packing_roundtrip():
+    import sys, os
+    sys.path.insert(0, os.path.dirname(__file__))
+    from milo_testutil import tok_slabs, untok_slabs
+    rng = np.random.default_rng(2)
+    u = rng.standard_normal((512, 37))
+    flat = tok_slabs(u)
+    assert flat.shape == (4 * 37, 128)
+    # element (j, t) sits at (t // 128) * (r * 128) + j * 128 + t % 128
+    j, t = 11, 300
+    assert flat.reshape(-1)[(t // 128) * 37 * 128 + j * 128 + t % 128] == u[t, j]
+    assert np.array_equal(untok_slabs(flat.reshape(-1), 512, 37), u)
