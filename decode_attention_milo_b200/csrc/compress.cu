@@ -93,58 +93,66 @@ __global__ void __launch_bounds__(kThreads) jacobi_kernel(const float* __restric
   float* A = smem;          // column-major: column j at A[j*D]
   float* W = smem + D * D;  // accumulated rotations, column-major
   float* lam = W + D * D;   // D
-  __shared__ int rotated;
   const int blk = blockIdx.x + blockIdx.y * nb;
   const float* G = gram + (int64_t)blk * D * D;
   for (int e = threadIdx.x; e < D * D; e += kThreads) {
     A[e] = G[e];  // G symmetric: row-major == column-major
     W[e] = (e / D == e % D) ? 1.f : 0.f;
   }
-  if (threadIdx.x == 0) rotated = 0;
   __syncthreads();
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  constexpr int NW = kThreads / 32;
+  constexpr int PP = (D / 2) / NW;  // column pairs per warp per round
   bool converged = false;
   for (int sweep = 0; sweep < max_sweeps; ++sweep) {
+    int rotated = 0;
     for (int s = 0; s < D - 1; ++s) {
-      for (int k = warp; k < D / 2; k += kThreads / 32) {
-        int p, q;
-        rr_pair(D, s, k, p, q);
-        float ap[E], aq[E];
-        float al = 0.f, be = 0.f, ga = 0.f;
+      // the warp's PP pairs are handled together so that their loads and reductions overlap
+      float ap[PP][E], aq[PP][E], al[PP], be[PP], ga[PP];
+      int pj[PP], qj[PP];
+#pragma unroll
+      for (int t = 0; t < PP; ++t) {
+        rr_pair(D, s, warp + t * NW, pj[t], qj[t]);
+        al[t] = be[t] = ga[t] = 0.f;
 #pragma unroll
         for (int e = 0; e < E; ++e) {
-          ap[e] = A[p * D + lane + 32 * e];
-          aq[e] = A[q * D + lane + 32 * e];
-          al = fmaf(ap[e], ap[e], al);
-          be = fmaf(aq[e], aq[e], be);
-          ga = fmaf(ap[e], aq[e], ga);
+          ap[t][e] = A[pj[t] * D + lane + 32 * e];
+          aq[t][e] = A[qj[t] * D + lane + 32 * e];
+          al[t] = fmaf(ap[t][e], ap[t][e], al[t]);
+          be[t] = fmaf(aq[t][e], aq[t][e], be[t]);
+          ga[t] = fmaf(ap[t][e], aq[t][e], ga[t]);
         }
-        al = warp_sum(al);
-        be = warp_sum(be);
-        ga = warp_sum(ga);
-        if (ga != 0.f && fabsf(ga) > kJacobiTol * sqrtf(al) * sqrtf(be)) {
-          const float zeta = (be - al) / (2.f * ga);
-          const float t = (zeta >= 0.f ? 1.f : -1.f) / (fabsf(zeta) + sqrtf(1.f + zeta * zeta));
-          const float c = 1.f / sqrtf(1.f + t * t);
-          const float sn = c * t;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int t = 0; t < PP; ++t) {
+          al[t] += __shfl_xor_sync(0xffffffffu, al[t], o);
+          be[t] += __shfl_xor_sync(0xffffffffu, be[t], o);
+          ga[t] += __shfl_xor_sync(0xffffffffu, ga[t], o);
+        }
+#pragma unroll
+      for (int t = 0; t < PP; ++t) {
+        if (ga[t] != 0.f && fabsf(ga[t]) > kJacobiTol * sqrtf(al[t]) * sqrtf(be[t])) {
+          const float zeta = (be[t] - al[t]) / (2.f * ga[t]);
+          const float tn = (zeta >= 0.f ? 1.f : -1.f) / (fabsf(zeta) + sqrtf(1.f + zeta * zeta));
+          const float c = 1.f / sqrtf(1.f + tn * tn);
+          const float sn = c * tn;
+          const int p = pj[t], q = qj[t];
 #pragma unroll
           for (int e = 0; e < E; ++e) {
-            A[p * D + lane + 32 * e] = c * ap[e] - sn * aq[e];
-            A[q * D + lane + 32 * e] = sn * ap[e] + c * aq[e];
+            A[p * D + lane + 32 * e] = c * ap[t][e] - sn * aq[t][e];
+            A[q * D + lane + 32 * e] = sn * ap[t][e] + c * aq[t][e];
             const float wp = W[p * D + lane + 32 * e], wq = W[q * D + lane + 32 * e];
             W[p * D + lane + 32 * e] = c * wp - sn * wq;
             W[q * D + lane + 32 * e] = sn * wp + c * wq;
           }
-          if (lane == 0) rotated = 1;
+          rotated = 1;
         }
       }
       __syncthreads();
     }
-    const bool any = rotated != 0;
-    __syncthreads();
-    if (threadIdx.x == 0) rotated = 0;
-    __syncthreads();
-    if (!any) {
+    if (!__syncthreads_or(rotated)) {
       converged = true;
       break;
     }

@@ -596,9 +596,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int j = 0; j < kChunk; ++j)
                 if (j >= valid) s[j] = -INFINITY;
             }
-            float mx = -INFINITY;
+            // tree max (8 independent lanes of reduction, then fold)
+            float m8[8];
 #pragma unroll
-            for (int j = 0; j < kChunk; ++j) mx = fmaxf(mx, s[j]);
+            for (int e = 0; e < 8; ++e) m8[e] = s[e];
+#pragma unroll
+            for (int j = 8; j < kChunk; j += 8)
+#pragma unroll
+              for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], s[j + e]);
+            float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
             mx *= p.c;
             // keep the running max in use unless the chunk exceeds it by more than 2^8 (then rescale)
             grow = !first_chunk && mx > m_used + 8.f;
@@ -645,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = wait_bar(bar(B_PEMPTY + slot), ((k >> 1) & 1) ^ 1, sh, p.status))) break;
           if (active) {
             const uint32_t pt = base + kOffP + 32768 * slot;
-            float lsum = 0.f;
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial row sums
 #pragma unroll
             for (int g8 = 0; g8 < kChunk / 8; ++g8) {
               uint32_t w[4];
@@ -653,12 +660,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int e = 0; e < 8; e += 2) {
                 const float a = ptx::ex2(fmaf(s[8 * g8 + e], p.c, -m_used));
                 const float b2 = ptx::ex2(fmaf(s[8 * g8 + e + 1], p.c, -m_used));
-                lsum += a + b2;
+                ls[e / 2] += a + b2;
                 w[e / 2] = ptx::pack_bf16(a, b2);
               }
               st_tile8(pt, row, 8 * g8, w[0], w[1], w[2], w[3]);
             }
-            l += lsum;
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             ptx::fence_async_smem();
           }
           ptx::tc_fence_before();
@@ -855,6 +862,9 @@ void tc_plan_destroy(TcPlan* plan) {
   delete plan;
 }
 
+// fixed per-chunk, per-block and per-suffix-unit times used to balance the work list (measured orders)
+constexpr double kChunkNs = 700.0, kBlockNs = 1500.0, kUnitNs = 1500.0;
+
 static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& in) {
   const int H = s.H, nb = s.nb, D = s.d, G = s.Hq / s.H, Bq = s.Bq, S = s.S;
   const int cpb = s.n / kChunk;
@@ -874,13 +884,17 @@ static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& 
     for (int rt = 0; rt < nrt; ++rt)
       for (int b = 0; b < nb; ++b) {
         const int rk = in.host_ranks[(size_t)(2 * h) * nb + b], rv = in.host_ranks[(size_t)(2 * h + 1) * nb + b];
+        // cost in nanoseconds: bytes at ~44 GB/s per SM, plus the fixed time of a chunk (softmax of
+        // 128 × 128 scores) and of a block (q̃ and ã round trips through TMEM and smem)
         for (int cc = 0; cc < cpb; ++cc)
           atoms.push_back({0, h, rt, b * cpb + cc,
-                           2.0 * (rk + rv) * kChunk + (cc == 0 ? 2.0 * (rk + rv) * D : 0.0)});
+                           (2.0 * (rk + rv) * kChunk + (cc == 0 ? 2.0 * (rk + rv) * D : 0.0)) / 44.0 + kChunkNs +
+                               (cc == 0 ? kBlockNs : 0.0)});
       }
   for (int i = 0; i < Bq; ++i)
     for (int h = 0; h < H; ++h)
-      for (int c = 0; c < nsc; ++c) atoms.push_back({1, h, i, c, 2.0 * 2.0 * kChunk * D});
+      for (int c = 0; c < nsc; ++c)
+        atoms.push_back({1, h, i, c, 2.0 * 2.0 * kChunk * D / 44.0 + kChunkNs + (c == 0 ? kUnitNs : 0.0)});
   double total = 0;
   for (auto& a : atoms) total += a.cost;
   const int grid = std::max(1, std::min(sms, (int)atoms.size()));
