@@ -64,6 +64,8 @@ def load_library(path: str | None = None):
     L.milo_decode_attn.argtypes = [vp, i32, i32, vp, vp, vp, i32, f32, vp, vp]
     L.milo_decode_attn_profiled.restype = i32
     L.milo_decode_attn_profiled.argtypes = [vp, i32, i32, vp, vp, vp, i32, f32, vp, vp, vp, vp]
+    L.milo_decode_attn_noalloc.restype = i32
+    L.milo_decode_attn_noalloc.argtypes = [vp, i32, i32, vp, vp, vp, i32, f32, vp, vp]
     L.milo_decode_launches.restype = i32
     L.milo_decode_launches.argtypes = [vp, i32, i32, i32]
     L.milo_factors_ranks.restype = i32
@@ -206,6 +208,20 @@ def decode_attn_profiled(q, factors: Factors, K_suf, V_suf, out, event_before, e
         _dev_ptr(V_suf, "V_suf") if S else None, S, float(scale), _dev_ptr(out, "out"), _stream_ptr(stream),
         ctypes.c_void_p(event_before.cuda_event), ctypes.c_void_p(event_after.cuda_event)),
         "milo_decode_attn_profiled")
+    return out
+
+
+def decode_attn_noalloc(q, factors: Factors, K_suf=None, V_suf=None, scale: float = 0.0, out=None, stream=None):
+    """decode_attn through milo_decode_attn_noalloc: the library allocates nothing (bf16 factors only)."""
+    import torch
+    B, Hq, _ = q.shape
+    S = 0 if K_suf is None else K_suf.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    _check(load_library().milo_decode_attn_noalloc(
+        _dev_ptr(q, "q"), B, Hq, factors.handle, _dev_ptr(K_suf, "K_suf") if S else None,
+        _dev_ptr(V_suf, "V_suf") if S else None, S, float(scale), _dev_ptr(out, "out"), _stream_ptr(stream)),
+        "milo_decode_attn_noalloc")
     return out
 
 

@@ -27,6 +27,7 @@
 
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "common.cuh"
@@ -1056,6 +1057,223 @@ cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, v
   else
     combine_tc_kernel<128><<<dim3(s.Hq, s.Bq), 128, 0, st>>>(pl->part_acc, pl->part_ml, pre, suf, s.H, s.Hq,
                                                             pl->ipt, pl->nrt, static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError();
+}
+
+
+// ================================================================================================
+// Decode without allocation: the same kernels, with their scratch (work list and partials) in a
+// fixed device array.  See milo_decode_attn_noalloc in milo.h.
+// ================================================================================================
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB, held by every device that loads us
+constexpr int kNoAllocMaxWords = 1 << 18;                  // host-side work-list staging (1 MiB)
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_dev_ptr[kNoAllocMaxDevices];  // device address of g_noalloc_scratch, per device
+int g_noalloc_host_words[kNoAllocMaxWords];   // work list staging, guarded by g_noalloc_mu
+
+// Byte-balanced work list as in build_plan, written into `w` without heap allocation.
+// Returns the number of words used, or -1 if `cap` words are not enough.
+int build_worklist_fixed(const DecodeShape& s, const int32_t* host_ranks, int grid, int* w, int cap, int& nsegs,
+                         int& off_segs, int& off_pre, int& off_suf, int& ipt_out, int& nrt_out) {
+  const int H = s.H, nb = s.nb, D = s.d, G = s.Hq / s.H, Bq = s.Bq, S = s.S;
+  const int cpb = s.n / kChunk;
+  const int ipt = std::min(Bq, 128 / G);
+  const int nrt = (Bq + ipt - 1) / ipt;
+  const int nsc = (S + kChunk - 1) / kChunk;
+  const int seg_words = (int)(sizeof(Seg) / sizeof(int));
+  auto for_each_atom = [&](auto&& fn) {
+    for (int h = 0; h < H; ++h)
+      for (int rt = 0; rt < nrt; ++rt)
+        for (int b = 0; b < nb; ++b) {
+          const int rk = host_ranks[(size_t)(2 * h) * nb + b], rv = host_ranks[(size_t)(2 * h + 1) * nb + b];
+          for (int cc = 0; cc < cpb; ++cc)
+            fn(0, h, rt, b * cpb + cc,
+               (2.0 * (rk + rv) * kChunk + (cc == 0 ? 2.0 * (rk + rv) * D : 0.0)) / 44.0 + kChunkNs +
+                   (cc == 0 ? kBlockNs : 0.0));
+        }
+    for (int i = 0; i < Bq; ++i)
+      for (int h = 0; h < H; ++h)
+        for (int c = 0; c < nsc; ++c)
+          fn(1, h, i, c, 2.0 * 2.0 * kChunk * D / 44.0 + kChunkNs + (c == 0 ? kUnitNs : 0.0));
+  };
+  double total = 0;
+  for_each_atom([&](int, int, int, int, double cost) { total += cost; });
+  off_segs = grid + 1;
+  if (off_segs > cap) return -1;
+  int* seg_first = w;
+  Seg* segs = reinterpret_cast<Seg*>(w + off_segs);
+  const int max_segs = (cap - off_segs) / seg_words;
+  for (int k = 0; k <= grid; ++k) seg_first[k] = 0;
+  int n = 0, cta = 0;
+  bool overflow = false;
+  double cum = 0;
+  for_each_atom([&](int type, int h, int tile, int c, double cost) {
+    if (overflow) return;
+    const double mid = cum + 0.5 * cost;
+    cum += cost;
+    while (cta + 1 < grid && mid >= total * (cta + 1) / grid) {
+      ++cta;
+      seg_first[cta] = n;
+    }
+    if (n > 0 && seg_first[cta] < n && segs[n - 1].type == type && segs[n - 1].h == h && segs[n - 1].tile == tile &&
+        segs[n - 1].c1 == c) {
+      segs[n - 1].c1 = c + 1;
+      return;
+    }
+    if (n >= max_segs) {
+      overflow = true;
+      return;
+    }
+    Seg sg{};
+    sg.type = type;
+    sg.h = h;
+    sg.tile = tile;
+    sg.c0 = c;
+    sg.c1 = c + 1;
+    sg.pid = n;
+    sg.rows = type == 0 ? std::min(ipt, Bq - tile * ipt) * G : G;
+    segs[n++] = sg;
+  });
+  if (overflow) return -1;
+  for (int k = cta + 1; k <= grid; ++k) seg_first[k] = n;
+  off_pre = off_segs + n * seg_words;
+  off_suf = off_pre + 2 * H * nrt;
+  const int nwords = off_suf + 2 * Bq * H;
+  if (nwords > cap) return -1;
+  int* pre = w + off_pre;
+  int* suf = w + off_suf;
+  for (int i = 0; i < 2 * H * nrt; ++i) pre[i] = -1;
+  for (int i = 0; i < 2 * Bq * H; ++i) suf[i] = 0;
+  for (int q = 0; q < n; ++q) {
+    const Seg& sg = segs[q];
+    int* r = sg.type == 0 ? &pre[2 * (sg.h * nrt + sg.tile)] : &suf[2 * (sg.tile * H + sg.h)];
+    if (sg.type == 0 && r[0] < 0) r[0] = sg.pid;
+    if (sg.type == 1 && r[1] == 0 && r[0] == 0) r[0] = sg.pid;
+    r[1] = sg.pid + 1;
+  }
+  for (int i = 0; i < 2 * H * nrt; ++i)
+    if (pre[i] < 0) pre[i] = 0;
+  for (int h = 0; h < H; ++h)
+    for (int i = 0; i < Bq; ++i) {
+      const int rt = i / ipt;
+      const int parts = pre[2 * (h * nrt + rt) + 1] - pre[2 * (h * nrt + rt)] + suf[2 * (i * H + h) + 1] -
+                        suf[2 * (i * H + h)];
+      if (parts > kMaxParts) return -1;
+    }
+  nsegs = n;
+  ipt_out = ipt;
+  nrt_out = nrt;
+  return nwords;
+}
+
+}  // namespace
+
+size_t tc_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* out, cudaStream_t st,
+                              bool* too_large) {
+  *too_large = false;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+  if (!g_noalloc_dev_ptr[dev]) {
+    // once per device, with that device current: host code cannot use the array's name as a device address
+    void* ptr = nullptr;
+    if ((e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch)) != cudaSuccess) return e;
+    g_noalloc_dev_ptr[dev] = ptr;
+    auto kfn = s.d == 64 ? (const void*)decode_tc_kernel<64> : (const void*)decode_tc_kernel<128>;
+    if ((e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes)) != cudaSuccess)
+      return e;
+  }
+  unsigned char* scratch = static_cast<unsigned char*>(g_noalloc_dev_ptr[dev]);
+  int sms = 148;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int cpb = s.n / kChunk, nsc = (s.S + kChunk - 1) / kChunk;
+  const int64_t natoms = (int64_t)s.H * ((s.Bq + std::min(s.Bq, 128 / (s.Hq / s.H)) - 1) /
+                                         std::min(s.Bq, 128 / (s.Hq / s.H))) * s.nb * cpb +
+                         (int64_t)s.Bq * s.H * nsc;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sms, natoms));
+  int nsegs = 0, off_segs = 0, off_pre = 0, off_suf = 0, ipt = 0, nrt = 0;
+  const int nwords = build_worklist_fixed(s, in.host_ranks, grid, g_noalloc_host_words, kNoAllocMaxWords, nsegs,
+                                          off_segs, off_pre, off_suf, ipt, nrt);
+  const size_t words_bytes = ((size_t)std::max(nwords, 0) * sizeof(int) + 255) & ~(size_t)255;
+  const size_t ml_bytes = ((size_t)nsegs * 128 * sizeof(float2) + 255) & ~(size_t)255;
+  const size_t acc_bytes = (size_t)nsegs * 128 * s.d * sizeof(float);
+  if (nwords < 0 || words_bytes + ml_bytes + acc_bytes > kNoAllocScratchBytes) {
+    *too_large = true;
+    return cudaErrorInvalidValue;
+  }
+  int* d_work = reinterpret_cast<int*>(scratch);
+  float2* part_ml = reinterpret_cast<float2*>(scratch + words_bytes);
+  float* part_acc = reinterpret_cast<float*>(scratch + words_bytes + ml_bytes);
+  // pageable source: the call returns once the words are staged, so the host buffer can be reused
+  if ((e = cudaMemcpyAsync(d_work, g_noalloc_host_words, (size_t)nwords * sizeof(int), cudaMemcpyHostToDevice, st)) !=
+      cudaSuccess)
+    return e;
+  const int D = s.d, G = s.Hq / s.H;
+  CUtensorMap map_tok, map_dim, mq_pre, mq_suf, mk, mv;
+  const uint64_t rows = (uint64_t)2 * s.H * in.pool_rows;
+  {
+    const uint64_t dims[2] = {(uint64_t)kChunk, rows * cpb}, strd[1] = {(uint64_t)kChunk * 2};
+    const uint32_t box[2] = {64, 16};
+    if (!make_map(&map_tok, in.tok, 2, dims, strd, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)D, rows}, strd[1] = {(uint64_t)D * 2};
+    const uint32_t box[2] = {64, 16};
+    if (!make_map(&map_dim, in.dim, 2, dims, strd, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)s.Hq, (uint64_t)s.Bq};
+    const uint64_t strd[2] = {(uint64_t)D * 2, (uint64_t)s.Hq * D * 2};
+    const uint32_t box_pre[3] = {64, (uint32_t)G, (uint32_t)ipt};
+    const uint32_t box_suf[3] = {64, (uint32_t)G, 1};
+    if (!make_map(&mq_pre, in.q, 3, dims, strd, box_pre)) return cudaErrorInvalidValue;
+    if (!make_map(&mq_suf, in.q, 3, dims, strd, box_suf)) return cudaErrorInvalidValue;
+  }
+  if (s.S > 0) {
+    const uint64_t dims[2] = {(uint64_t)D, (uint64_t)s.Bq * s.H * s.S}, strd[1] = {(uint64_t)D * 2};
+    const uint32_t box[2] = {64, 16};
+    if (!make_map(&mk, in.K_suf, 2, dims, strd, box)) return cudaErrorInvalidValue;
+    if (!make_map(&mv, in.V_suf, 2, dims, strd, box)) return cudaErrorInvalidValue;
+  } else {
+    mk = map_dim;
+    mv = map_dim;
+  }
+  Params p;
+  p.seg_first = d_work;
+  p.segs = reinterpret_cast<const Seg*>(d_work + off_segs);
+  p.ranks = in.ranks;
+  p.row_offsets = in.row_offsets;
+  p.part_acc = part_acc;
+  p.part_ml = part_ml;
+  p.status = in.status;
+  p.nb = s.nb;
+  p.cpb = cpb;
+  p.H = s.H;
+  p.G = G;
+  p.ipt = ipt;
+  p.S = s.S;
+  p.c = s.scale * 1.4426950408889634f;
+  if (D == 64)
+    decode_tc_kernel<64><<<grid, kThreads, kSmemBytes, st>>>(map_tok, map_dim, mq_pre, mq_suf, mk, mv, p);
+  else
+    decode_tc_kernel<128><<<grid, kThreads, kSmemBytes, st>>>(map_tok, map_dim, mq_pre, mq_suf, mk, mv, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (D == 64)
+    combine_tc_kernel<64><<<dim3(s.Hq, s.Bq), 64, 0, st>>>(part_acc, part_ml, d_work + off_pre, d_work + off_suf,
+                                                          s.H, s.Hq, ipt, nrt, static_cast<__nv_bfloat16*>(out));
+  else
+    combine_tc_kernel<128><<<dim3(s.Hq, s.Bq), 128, 0, st>>>(part_acc, part_ml, d_work + off_pre, d_work + off_suf,
+                                                            s.H, s.Hq, ipt, nrt, static_cast<__nv_bfloat16*>(out));
   return cudaGetLastError();
 }
 

@@ -30,4 +30,10 @@ cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, v
                       cudaEvent_t ev0 = nullptr, cudaEvent_t ev1 = nullptr);
 void tc_plan_destroy(TcPlan* plan);
 
+// The same decode with its scratch in a fixed device array (no allocation).  *too_large is set when
+// the work list or the partials of this shape do not fit the array.
+cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* out, cudaStream_t st,
+                              bool* too_large);
+size_t tc_noalloc_scratch_bytes();
+
 }  // namespace milo

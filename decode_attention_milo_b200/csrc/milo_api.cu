@@ -362,6 +362,44 @@ milo_status milo_decode_attn(const void* q, int32_t batch, int32_t num_q_heads, 
                      nullptr);
 }
 
+// Host staging of the ranks for milo_decode_attn_noalloc when the factor object has no host copy yet.
+static int32_t g_noalloc_ranks[1 << 16];
+static std::mutex g_noalloc_ranks_mu;
+
+milo_status milo_decode_attn_noalloc(const void* q, int32_t batch, int32_t num_q_heads, const milo_factors* fc,
+                                     const void* K_suffix, const void* V_suffix, int32_t suffix_len, float scale,
+                                     void* out, void* stream) {
+  if (!fc || !q || !out || batch <= 0 || num_q_heads <= 0 || suffix_len < 0) return MILO_ERR_INVALID_ARGUMENT;
+  milo_factors* f = const_cast<milo_factors*>(fc);
+  if (num_q_heads % f->H != 0) return MILO_ERR_INVALID_ARGUMENT;
+  if (suffix_len > 0 && (!K_suffix || !V_suffix)) return MILO_ERR_INVALID_ARGUMENT;
+  if (!(scale == scale) || isinf(scale)) return MILO_ERR_INVALID_ARGUMENT;
+  if (batch > 65535 || num_q_heads > 4096 || suffix_len > (1 << 20)) return MILO_ERR_INVALID_ARGUMENT;
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)f->d);
+  milo::DecodeShape ds{f->H, f->nb, f->n, f->d, batch, num_q_heads, suffix_len, f->dtype == MILO_BF16, sc};
+  if (f->dtype != MILO_BF16 || !milo::tc_supported(ds)) return MILO_ERR_UNSUPPORTED;
+  const size_t nranks = (size_t)2 * f->H * f->nb;
+  if (nranks > sizeof(g_noalloc_ranks) / sizeof(int32_t)) return MILO_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(f->mu);
+  std::lock_guard<std::mutex> lock_r(g_noalloc_ranks_mu);
+  const int32_t* host_ranks = f->host_ranks.empty() ? nullptr : f->host_ranks.data();
+  if (!host_ranks) {
+    MILO_CUDA(cudaEventSynchronize(f->ready));
+    MILO_CUDA(cudaMemcpy(g_noalloc_ranks, f->ranks, nranks * sizeof(int32_t), cudaMemcpyDeviceToHost));
+    host_ranks = g_noalloc_ranks;
+  }
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  MILO_CUDA(cudaStreamIsCapturing(s, &cap));
+  if (cap == cudaStreamCaptureStatusNone) MILO_CUDA(cudaStreamWaitEvent(s, f->ready, 0));
+  milo::TcInputs in{q,        K_suffix, V_suffix,     f->tok,       f->dim,
+                    f->ranks, f->row_offsets, f->status, f->pool_rows, host_ranks};
+  bool too_large = false;
+  const cudaError_t e = milo::tc_decode_noalloc(ds, in, out, s, &too_large);
+  if (too_large) return MILO_ERR_UNSUPPORTED;
+  return cuda_status(e);
+}
+
 milo_status milo_decode_attn_profiled(const void* q, int32_t batch, int32_t num_q_heads, const milo_factors* f,
                                       const void* K_suffix, const void* V_suffix, int32_t suffix_len, float scale,
                                       void* out, void* stream, void* event_before, void* event_after) {

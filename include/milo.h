@@ -156,6 +156,38 @@ milo_status milo_decode_attn_profiled(const void* q, int32_t batch, int32_t num_
                                       void* event_after);
 
 /*
+ * milo_decode_attn_noalloc — milo_decode_attn for callers that cannot allocate
+ * device memory.  The pages have no counterpart: it is a deployment variant.
+ * Who needs it: code that runs where cudaMalloc is not allowed or not wanted —
+ * while a stream is being captured in global mode (cudaMalloc is illegal there),
+ * inside an engine whose allocator owns all device memory and forbids side
+ * allocations, or on a latency-critical path that cannot afford the device-wide
+ * synchronisation cudaMalloc implies.  milo_decode_attn allocates its work list
+ * and partials on the first call for a shape; this entry point allocates nothing
+ * (no cudaMalloc, cudaFree, or allocating library routine) and keeps both in one
+ * fixed array in device memory of MILO_NOALLOC_SCRATCH_BYTES (32 MiB) that every
+ * GPU loading the library holds until the process exits.
+ *   Arguments, layout and results: as milo_decode_attn, for bf16 factors only
+ *   (MILO_ERR_UNSUPPORTED for fp32).
+ *   Size limit: a shape whose work list plus partials (about 66 KB per work
+ *   segment at d = 128; the Qwen2.5-7B layer at batch 16 needs about 15 MB)
+ *   exceed the array returns MILO_ERR_UNSUPPORTED before anything is launched.
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.  If the factor object has never been decoded,
+ *   the call synchronises once on the factors to read their ranks.
+ *   Sharing: every call on a device uses the same array and leaves its contents
+ *   behind; each call writes every scratch word it reads, so nothing has to
+ *   start at zero, but calls that overlap on the GPU (different streams, or
+ *   different factor objects at once) race on it and must be serialised.
+ */
+#define MILO_NOALLOC_SCRATCH_BYTES (32u << 20)
+milo_status milo_decode_attn_noalloc(const void* q, int32_t batch, int32_t num_q_heads,
+                                     const milo_factors* f, const void* K_suffix,
+                                     const void* V_suffix, int32_t suffix_len, float scale,
+                                     void* out, void* stream);
+
+/*
  * Number of kernels one milo_decode_attn call with these arguments launches
  * (>= 1), or a negative milo_status for invalid arguments.  Host-only, no GPU work.
  */
