@@ -37,39 +37,37 @@
 namespace milo {
 namespace {
 
-constexpr int kThreads = 192;        // 6 warps
-constexpr int kStages = 4;           // TMA ring stages
-constexpr int kStageBytes = 16384;   // one piece: 64 rows × 128 columns of bf16
+constexpr int kThreads = 192;        // warp 0: TMA producer; warp 1: MMA issuer; warps 2..5: softmax
+constexpr int kSigQt = 1, kSigP = 2, kSigAt = 3;  // named barriers: softmax warps → MMA warp
+constexpr int kRingBytes = 94208;   // TMA ring: variable-size items, each one contiguous tile
+constexpr int kItemSlots = 16;       // items in flight at most (one FULL/EMPTY barrier pair each)
 constexpr int kChunk = 128;          // tokens per score chunk
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 // shared-memory map (bytes from a 1024-aligned base)
 constexpr int kOffQ = 0;          // [cb][128 rows][128 B]  query rows, K-major over d
-constexpr int kOffQtHi = 32768;   // [cb][128][128 B]  q̃ high part, K-major over rank; later ã
+constexpr int kOffQtHi = 32768;   // [cb][128][128 B]  q̃ high part, K-major over rank
 constexpr int kOffQtLo = 65536;   // [cb][128][128 B]  q̃ low part
-constexpr int kOffP = 98304;      // 2 × [cb][128][128 B]  probabilities, K-major over tokens
-constexpr int kOffRing = 163840;  // kStages × [cb][64 rows][128 B]
-constexpr int kOffBar = kOffRing + kStages * kStageBytes;  // 229376
-constexpr int kSmemBytes = kOffBar + 1024 + 1024;          // barriers + alignment slack
+constexpr int kOffP = 98304;      // [cb][128][128 B]  probabilities (K-major over tokens); then ã for G4
+constexpr int kOffRing = 131072;  // kRingBytes of items laid out [64-column block][rows][128 B]
+constexpr int kOffBar = kOffRing + kRingBytes;             // 225280: barriers, then the Shared block
+constexpr int kBarRegion = 4096;
+constexpr int kSmemBytes = kOffBar + kBarRegion + 1024;     // + alignment slack (230400)
 constexpr uint32_t kTileCb = 16384;  // column-block stride of a 128-row tile
-constexpr uint32_t kPieceCb = 8192;  // column-block stride of a 64-row piece
+constexpr int kMaxSegsSmem = 16, kMaxBlocksSmem = 64;  // per-CTA work tables staged in smem
 
-// TMEM columns: acc [0,128), S slots [128,256) and [256,384), q̃ / ã [384,512)
-constexpr uint32_t kTmAcc = 0, kTmS0 = 128, kTmR = 384;
+// TMEM columns: acc [0,128), two S slots [128,256) and [256,384) (q̃ of a block also passes through
+// an S slot), ã [384,512)
+constexpr uint32_t kTmAcc = 0, kTmS0 = 128, kTmA = 384;
 
 enum Bar {
   B_FULL = 0,
-  B_EMPTY = B_FULL + kStages,
-  B_QFULL = B_EMPTY + kStages,
+  B_EMPTY = B_FULL + kItemSlots,
+  B_QFULL = B_EMPTY + kItemSlots,
   B_QEMPTY,
-  B_QTFULL,
-  B_QTREADY,
   B_SFULL,
-  B_SEMPTY = B_SFULL + 2,
-  B_PFULL = B_SEMPTY + 2,
-  B_PEMPTY = B_PFULL + 2,
-  B_ATFULL = B_PEMPTY + 2,
-  B_ATREADY,
+  B_PEMPTY = B_SFULL + 2,
+  B_ATFULL,
   B_ACCFULL,
   B_FINAL,
   B_COUNT
@@ -97,18 +95,31 @@ struct Params {
   float c;  // scale · log2(e)
 };
 
+struct BlockInfo {
+  int rk, rv;
+  int64_t rowk, rowv;
+};
+
+// Per-CTA state in shared memory: the CTA's segments and the rank / row offset of every block they
+// touch, staged once at start so that no role reads them from global memory inside the pipeline.
 struct Shared {
   uint32_t tmem_base;
   int abort_flag;
+  int nseg;        // segments of this CTA staged (0 when they did not fit: roles read global memory)
+  int nblk;        // blocks staged
+  int blk0[kMaxSegsSmem + 1];  // first table entry of each segment
+  Seg segs[kMaxSegsSmem];
+  BlockInfo blocks[kMaxBlocksSmem];
+  uint32_t pos_log[kItemSlots], len_log[kItemSlots];  // producer's record of the items in flight
 };
+static_assert(8 * B_COUNT + 64 + sizeof(Shared) <= kBarRegion, "barrier region too small");
 
 // Warp-collective bounded wait on an mbarrier phase (all 32 lanes call it together; the result is uniform).
 // Gives up after kWaitNs, records kStatusDecodeTimeout and raises the CTA's abort flag, or returns false at
 // once when another role already aborted.  `drain` waits ignore the abort flag (used to let the CTA's own
 // copies and MMAs land before it exits) but keep the time limit.
-__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, Shared* sh, uint32_t* status,
-                                      bool drain = false) {
-  if (__all_sync(0xffffffffu, ptx::mbar_try_wait(bar, parity))) return true;
+__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, Shared* sh, uint32_t* status,
+                                           bool drain) {
   uint64_t t0 = 0;
   if ((threadIdx.x & 31) == 0) t0 = ptx::globaltimer();
   for (uint32_t i = 1;; ++i) {
@@ -129,12 +140,14 @@ __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, Shared* sh,
   }
 }
 
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Shared* sh, uint32_t* status,
+                                         bool drain = false) {
+  if (__all_sync(0xffffffffu, ptx::mbar_try_wait(bar, parity))) return true;
+  return wait_bar_slow(bar, parity, sh, status, drain);
+}
+
 __device__ __forceinline__ int pad16(int r) { return (r + 15) & ~15; }
 
-struct BlockInfo {
-  int rk, rv;
-  int64_t rowk, rowv;
-};
 __device__ __forceinline__ bool block_info(const Params& p, int h, int b, int D, BlockInfo& bi) {
   bi.rk = p.ranks[(int64_t)(2 * h) * p.nb + b];
   bi.rv = p.ranks[(int64_t)(2 * h + 1) * p.nb + b];
@@ -143,15 +156,41 @@ __device__ __forceinline__ bool block_info(const Params& p, int h, int b, int D,
   return bi.rk >= 1 && bi.rk <= D && bi.rv >= 1 && bi.rv <= D;
 }
 
-// Ring position shared by producer and consumer: both walk the same item sequence.
-struct Ring {
-  uint32_t stage = 0, phase = 0;
-  __device__ void advance() {
-    if (++stage == kStages) {
-      stage = 0;
-      phase ^= 1;
-    }
+// Block `k` (0-based, in walk order) of segment `si` of this CTA: from the smem table when staged.
+__device__ __forceinline__ bool seg_block(const Params& p, const Shared* sh, int si_local, int k, int h, int b, int D,
+                                          BlockInfo& bi) {
+  if (sh->nseg > 0) {
+    bi = sh->blocks[sh->blk0[si_local] + k];
+    return bi.rk >= 1 && bi.rk <= D && bi.rv >= 1 && bi.rv <= D;
   }
+  return block_info(p, h, b, D, bi);
+}
+__device__ __forceinline__ Seg get_seg(const Params& p, const Shared* sh, int s_begin, int si) {
+  return sh->nseg > 0 ? sh->segs[si - s_begin] : p.segs[si];
+}
+
+// Placement of items in the TMA ring.  Producer and consumer call place() with the same sizes in the same
+// order, so they agree on every item's offset without exchanging it; an item that does not fit before the
+// end of the ring starts at offset 0.
+struct RingPlace {
+  uint32_t head = 0;  // next free byte offset
+  uint32_t n = 0;     // items placed so far
+  __device__ uint32_t place(uint32_t bytes) {
+    const uint32_t pos = head + bytes <= (uint32_t)kRingBytes ? head : 0u;
+    head = pos + bytes;
+    ++n;
+    return pos;
+  }
+};
+
+// Block range of a prefix segment: chunks [c0, c1) cover blocks c0/cpb .. (c1-1)/cpb.
+struct BlockWalk {
+  int c, c1, cpb;
+  __device__ int block() const { return c / cpb; }
+  __device__ int chunks() const { return min(c1, (c / cpb + 1) * cpb) - c; }  // chunks of this block here
+  __device__ int first_cc() const { return c - (c / cpb) * cpb; }            // chunk index inside the block
+  __device__ bool has_next() const { return c + chunks() < c1; }
+  __device__ void next() { c += chunks(); }
 };
 
 // -------------------------------------------------------------------------------------------- producer
@@ -159,34 +198,52 @@ template <int D>
 struct Producer {
   static constexpr int NCB = D / 64;
   uint32_t base;
-  Ring ring;
+  RingPlace ring;
+  uint32_t oldest = 0;  // first item not yet known to be released
   uint32_t q_uses = 0;
-  bool issued[kStages];
-  uint32_t issued_parity[kStages];
   Shared* sh;
   uint32_t* status;
+  uint32_t* pos_log;  // [kItemSlots] offsets of the items in flight (smem, producer only)
+  uint32_t* len_log;  // [kItemSlots] their sizes
 
   __device__ uint32_t bar(int i) const { return base + kOffBar + 8 * i; }
 
-  // `rows` (multiple of 16, <= 64) rows × `ncb` 64-column blocks of a 2D map at (x0, y0) → one ring stage.
-  __device__ bool piece(const CUtensorMap* m, int x0, int64_t y0, int rows, int ncb) {
-    if (!wait_bar(bar(B_EMPTY + ring.stage), ring.phase ^ 1, sh, status)) return false;
-    const uint32_t dst = base + kOffRing + ring.stage * kStageBytes;
-    const uint32_t fb = bar(B_FULL + ring.stage);
-    if ((threadIdx.x & 31) == 0) {
-      ptx::mbar_arrive_expect_tx(fb, rows * 128 * ncb);
-      for (int cb = 0; cb < ncb; ++cb)
-        for (int k = 0; k < rows; k += 16)
-          ptx::tma_load_2d(dst + cb * kPieceCb + k * 128, m, fb, x0 + 64 * cb, (int)(y0 + k));
-    }
-    issued[ring.stage] = true;
-    issued_parity[ring.stage] = ring.phase;
-    ring.advance();
+  // Waits until the oldest item in flight has been consumed and forgets it.
+  __device__ bool retire_oldest() {
+    const uint32_t j = oldest;
+    if (!wait_bar(bar(B_EMPTY + j % kItemSlots), (j / kItemSlots) & 1, sh, status)) return false;
+    ++oldest;
     return true;
   }
+
+  // `rows` (multiple of 16, <= 128) rows × `ncb` 64-column blocks of a 2D map at (x0, y0) → one item,
+  // laid out [cb][rows][128 B].
   __device__ bool item(const CUtensorMap* m, int x0, int64_t y0, int rows, int ncb) {
-    for (int r = 0; r < rows; r += 64)
-      if (!piece(m, x0, y0 + r, min(64, rows - r), ncb)) return false;
+    const uint32_t bytes = (uint32_t)rows * 128u * ncb;
+    const uint32_t i = ring.n;
+    const uint32_t pos = ring.place(bytes);
+    // free the space: retire the oldest items while any item in flight overlaps it (after a wrap a newer
+    // item can overlap while the oldest does not), and keep at most kItemSlots in flight
+    while (oldest < i) {
+      bool busy = i - oldest >= (uint32_t)kItemSlots;
+      for (uint32_t j = oldest; j < i && !busy; ++j) {
+        const uint32_t k = j % kItemSlots;
+        busy = pos < pos_log[k] + len_log[k] && pos_log[k] < pos + bytes;
+      }
+      if (!busy) break;
+      if (!retire_oldest()) return false;
+    }
+    pos_log[i % kItemSlots] = pos;
+    len_log[i % kItemSlots] = bytes;
+    const uint32_t dst = base + kOffRing + pos;
+    const uint32_t fb = bar(B_FULL + i % kItemSlots);
+    if ((threadIdx.x & 31) == 0) {
+      ptx::mbar_arrive_expect_tx(fb, bytes);
+      for (int cb = 0; cb < ncb; ++cb)
+        for (int k = 0; k < rows; k += 16)
+          ptx::tma_load_2d(dst + cb * rows * 128 + k * 128, m, fb, x0 + 64 * cb, (int)(y0 + k));
+    }
+    __syncwarp();
     return true;
   }
   __device__ bool q_tile(const CUtensorMap* m, int y, int z, int box_rows) {
@@ -204,9 +261,13 @@ struct Producer {
 __device__ __forceinline__ uint64_t kdesc(uint32_t tile, int k, uint32_t cbs) {
   return ptx::sw128_desc(tile + (uint32_t)(k >> 2) * cbs + (uint32_t)(k & 3) * 32, 16, 1024);
 }
-// MN-major SW128 descriptor of k-step k (16 rows) of a 64-row piece (MN column blocks kPieceCb apart).
-__device__ __forceinline__ uint64_t mndesc(uint32_t piece, int k) {
-  return ptx::sw128_desc(piece + (uint32_t)k * 2048, kPieceCb, 1024);
+// Offset, in descriptor units (16 B), of k-step k of a K-major operand whose column blocks are `cbs` apart.
+__device__ __forceinline__ uint64_t kstep(int k, uint32_t cbs) {
+  return (uint64_t)(((uint32_t)(k >> 2) * cbs + (uint32_t)(k & 3) * 32) >> 4);
+}
+// MN-major SW128 descriptor of an item [cb][rows][128 B]: k-step k (16 rows) starts 2048 B further.
+__device__ __forceinline__ uint64_t mndesc(uint32_t item, int k, uint32_t cbs) {
+  return ptx::sw128_desc(item + (uint32_t)k * 2048, cbs, 1024);
 }
 
 // Writes 8 consecutive bf16 (4 packed words) at (row, col) of a K-major SW128 tile (128-row, 16 KB col blocks).
@@ -234,22 +295,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- setup: zero the query tile (rows no TMA box writes stay finite), barriers, TMEM
   for (int i = threadIdx.x; i < 32768 / 16; i += kThreads) ptx::st_shared_v4(base + kOffQ + 16 * i, 0, 0, 0, 0);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kItemSlots; ++i) {
       ptx::mbar_init(bar(B_FULL + i), 1);
       ptx::mbar_init(bar(B_EMPTY + i), 1);
     }
     ptx::mbar_init(bar(B_QFULL), 1);
     ptx::mbar_init(bar(B_QEMPTY), 1);
-    ptx::mbar_init(bar(B_QTFULL), 1);
-    ptx::mbar_init(bar(B_QTREADY), 4);
-    for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(bar(B_SFULL + i), 1);
-      ptx::mbar_init(bar(B_SEMPTY + i), 4);
-      ptx::mbar_init(bar(B_PFULL + i), 4);
-      ptx::mbar_init(bar(B_PEMPTY + i), 1);
-    }
+    ptx::mbar_init(bar(B_SFULL), 1);
+    ptx::mbar_init(bar(B_SFULL + 1), 1);
+    ptx::mbar_init(bar(B_PEMPTY), 1);
     ptx::mbar_init(bar(B_ATFULL), 1);
-    ptx::mbar_init(bar(B_ATREADY), 4);
     ptx::mbar_init(bar(B_ACCFULL), 1);
     ptx::mbar_init(bar(B_FINAL), 1);
     sh->abort_flag = 0;
@@ -267,467 +322,606 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tmem_alloc(ptx::smem_u32(&sh->tmem_base), 512);
     ptx::tmem_relinquish();
   }
+  const int s_begin = p.seg_first[blockIdx.x], s_end = p.seg_first[blockIdx.x + 1];
+  // stage this CTA's segments and the rank / row offsets of their blocks in shared memory
+  const int nseg_here = s_end - s_begin;
+  const bool stage_tables = nseg_here <= kMaxSegsSmem;
+  if (stage_tables && (int)threadIdx.x < nseg_here) sh->segs[threadIdx.x] = p.segs[s_begin + threadIdx.x];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int nblk = 0;
+    for (int i = 0; i < (stage_tables ? nseg_here : 0); ++i) {
+      sh->blk0[i] = nblk;
+      const Seg& sg = sh->segs[i];
+      if (sg.type == 0) nblk += (sg.c1 - 1) / p.cpb - sg.c0 / p.cpb + 1;
+    }
+    sh->blk0[stage_tables ? nseg_here : 0] = nblk;
+    const bool fits = stage_tables && nblk <= kMaxBlocksSmem;
+    sh->nblk = fits ? nblk : 0;
+    sh->nseg = fits ? nseg_here : 0;
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < sh->nblk; t += kThreads) {
+    int i = 0;
+    while (sh->blk0[i + 1] <= t) ++i;
+    const Seg& sg = sh->segs[i];
+    BlockInfo bi;
+    block_info(p, sg.h, sg.c0 / p.cpb + (t - sh->blk0[i]), D, bi);
+    sh->blocks[t] = bi;
+  }
   ptx::fence_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
-  const int s_begin = p.seg_first[blockIdx.x], s_end = p.seg_first[blockIdx.x + 1];
 
   if (warp == 0) {
     // ==================================================================== TMA producer
+    // Loads items in exactly the order the issuing warp consumes them (see the softmax section).
     Producer<D> pr;
     pr.base = base;
     pr.sh = sh;
     pr.status = p.status;
-    for (int i = 0; i < kStages; ++i) pr.issued[i] = false;
+    pr.pos_log = sh->pos_log;
+    pr.len_log = sh->len_log;
     bool ok = true;
+    auto bad_block = [&]() {
+      atomicOr(p.status, kStatusDecodeBounds);
+      sh->abort_flag = 1;
+      return false;
+    };
+    // token-factor slab of chunk cc (index inside the block) of a block: rows [row0·cpb + cc·r, +r)
+    auto tok_item = [&](int64_t row0, int r, int cc) {
+      return pr.item(&map_tok, 0, row0 * p.cpb + (int64_t)cc * r, pad16(r), 2);
+    };
+    auto dim_item = [&](int64_t row0, int r) { return pr.item(&map_dim, 0, row0, pad16(r), NCB); };
     for (int si = s_begin; si < s_end && ok; ++si) {
-      const Seg sg = p.segs[si];
+      const Seg sg = get_seg(p, sh, s_begin, si);
       if (sg.type == 0) {
         ok = pr.q_tile(&map_qpre, sg.h * p.G, sg.tile * p.ipt, p.G * p.ipt);
-        for (int c = sg.c0; c < sg.c1 && ok;) {
-          const int b = c / p.cpb;
-          const int cend = min(sg.c1, (b + 1) * p.cpb);
-          BlockInfo bi;
-          if (!block_info(p, sg.h, b, D, bi)) {
-            atomicOr(p.status, kStatusDecodeBounds);
-            sh->abort_flag = 1;
-            ok = false;
-            break;
+        BlockWalk w{sg.c0, sg.c1, p.cpb};
+        BlockInfo bi, bn, prev;
+        bool have_prev = false;
+        int kb = 0;
+        if (ok && !seg_block(p, sh, si - s_begin, kb, sg.h, w.block(), D, bi)) ok = bad_block();
+        if (ok) ok = dim_item(bi.rowk, bi.rk);  // B_K of the first block
+        while (ok) {
+          const int n = w.chunks(), cc0 = w.first_cc();
+          const bool next = w.has_next();
+          if (next && !seg_block(p, sh, si - s_begin, kb + 1, sg.h, w.block() + 1, D, bn)) ok = bad_block();
+          if (ok) ok = tok_item(bi.rowk, bi.rk, cc0);                       // U(0)
+          if (ok && n >= 2) ok = tok_item(bi.rowk, bi.rk, cc0 + 1);         // U(1)
+          else if (ok && next) ok = dim_item(bn.rowk, bn.rk);               // B_K(next)
+          if (ok && have_prev) ok = dim_item(prev.rowv, prev.rv);           // Q_V(previous block)
+          for (int j = 0; j < n && ok; ++j) {
+            ok = tok_item(bi.rowv, bi.rv, cc0 + j);                         // P(j)
+            if (ok && j + 2 < n) ok = tok_item(bi.rowk, bi.rk, cc0 + j + 2);  // U(j+2)
+            else if (ok && j + 2 == n && next) ok = dim_item(bn.rowk, bn.rk);  // B_K(next)
           }
-          const int rkp = pad16(bi.rk), rvp = pad16(bi.rv);
-          // consumption order: B_K, U(0), [U(1), P(0)], ..., [U(n-1), P(n-2)], P(n-1), Q_V
-          ok = pr.item(&map_dim, 0, bi.rowk, rkp, NCB);
-          // token factor slabs: chunk cc of the block is rows [row0·cpb + cc·r, +r) of the 128-wide view
-          for (int cc = c; cc <= cend && ok; ++cc) {
-            if (cc < cend) ok = pr.item(&map_tok, 0, bi.rowk * p.cpb + (int64_t)(cc - b * p.cpb) * bi.rk, rkp, 2);
-            if (ok && cc > c)
-              ok = pr.item(&map_tok, 0, bi.rowv * p.cpb + (int64_t)(cc - 1 - b * p.cpb) * bi.rv, rvp, 2);
-          }
-          if (ok) ok = pr.item(&map_dim, 0, bi.rowv, rvp, NCB);
-          c = cend;
+          if (!ok || !next) break;
+          prev = bi;
+          have_prev = true;
+          w.next();
+          bi = bn;
+          ++kb;
         }
+        if (ok) ok = dim_item(bi.rowv, bi.rv);  // Q_V of the last block
       } else {
         ok = pr.q_tile(&map_qsuf, sg.h * p.G, sg.tile, p.G);
         const int64_t row0 = ((int64_t)sg.tile * p.H + sg.h) * p.S;
-        // consumption order: K(0), [K(1), V(0)], ..., V(n-1)
-        for (int c = sg.c0; c <= sg.c1 && ok; ++c) {
-          if (c < sg.c1) ok = pr.item(&map_ksuf, 0, row0 + (int64_t)c * kChunk, kChunk, NCB);
-          if (ok && c > sg.c0) ok = pr.item(&map_vsuf, 0, row0 + (int64_t)(c - 1) * kChunk, kChunk, NCB);
+        const int n = sg.c1 - sg.c0;
+        auto kv = [&](const CUtensorMap* m, int j) {
+          return pr.item(m, 0, row0 + (int64_t)(sg.c0 + j) * kChunk, kChunk, NCB);
+        };
+        if (ok) ok = kv(&map_ksuf, 0);
+        if (ok && n >= 2) ok = kv(&map_ksuf, 1);
+        for (int j = 0; j < n && ok; ++j) {
+          ok = kv(&map_vsuf, j);
+          if (ok && j + 2 < n) ok = kv(&map_ksuf, j + 2);
         }
       }
     }
     // drain: every copy this warp issued must have landed before the CTA exits
-    for (int i = 0; i < kStages; ++i)
-      if (pr.issued[i]) wait_bar(bar(B_FULL + i), pr.issued_parity[i], sh, p.status, true);
+    for (uint32_t j = pr.oldest; j < pr.ring.n; ++j)
+      wait_bar(bar(B_FULL + j % kItemSlots), (j / kItemSlots) & 1, sh, p.status, true);
     if (pr.q_uses) wait_bar(bar(B_QFULL), (pr.q_uses - 1) & 1, sh, p.status, true);
   } else if (warp == 1) {
-    // ==================================================================== MMA issuer
-    Ring ring;
-    uint32_t q_uses = 0, qt_uses = 0, at_uses = 0;
-    uint32_t chunk_ix = 0;  // chunks processed by this CTA: S and P slot = chunk_ix & 1
+    // ==================================================================== MMA issuer (warp 1)
+    // Issues the tensor-core MMAs when the softmax warps signal (named barriers: q̃ ready, P ready, ã ready)
+    // that the smem operands they produce are complete, so issuing overlaps the next softmax step.
     const bool leader = lane == 0;
     bool ok = true;
-    auto take = [&](uint32_t& addr) -> bool {
-      if (!wait_bar(bar(B_FULL + ring.stage), ring.phase, sh, p.status)) return false;
+    auto sync_wg = [&](int id) {  // wait for the softmax warps' signal `id`
+      asm volatile("bar.sync %0, 160;" ::"r"(id) : "memory");
       ptx::tc_fence_after();
-      addr = base + kOffRing + ring.stage * kStageBytes;
+    };
+    // ---------------- MMA issue (warp 1 only)
+    RingPlace ring;          // consumer view of the TMA ring
+    uint32_t cur = 0;        // item being consumed
+    uint32_t sidx_i = 0;     // S-slot uses issued
+    uint32_t q_uses = 0;
+    auto take = [&](int rows, int ncb, uint32_t& addr) -> bool {
+      cur = ring.n;
+      const uint32_t pos = ring.place((uint32_t)rows * 128u * ncb);
+      if (!wait_bar(bar(B_FULL + cur % kItemSlots), (cur / kItemSlots) & 1, sh, p.status)) return false;
+      ptx::tc_fence_after();
+      addr = base + kOffRing + pos;
       return true;
     };
-    auto release = [&]() {
-      if (leader) ptx::umma_commit(bar(B_EMPTY + ring.stage));
-      ring.advance();
+    auto release = [&]() {  // the item's space is free once the MMAs issued so far have read it
+      if (leader) ptx::umma_commit(bar(B_EMPTY + cur % kItemSlots));
     };
-    auto wait_s_empty = [&](uint32_t k) {
-      const bool r = wait_bar(bar(B_SEMPTY + (k & 1)), ((k >> 1) & 1) ^ 1, sh, p.status);
-      ptx::tc_fence_after();
-      return r;
+    constexpr uint32_t idS = ptx::idesc_bf16(128, 128, false, true);
+    constexpr uint32_t idD = ptx::idesc_bf16(128, D, false, true);
+    auto s_commit = [&]() {
+      if (leader) ptx::umma_commit(bar(B_SFULL + (sidx_i & 1)));
+      ++sidx_i;
     };
-    auto wait_p_full = [&](uint32_t k) {
-      const bool r = wait_bar(bar(B_PFULL + (k & 1)), (k >> 1) & 1, sh, p.status);
-      ptx::tc_fence_after();
-      return r;
+    // G1: q̃ = Q · B_b into the next S slot, N = padded rank
+    auto g1 = [&](int rk) -> bool {
+      const int rp = pad16(rk);
+      uint32_t it;
+      if (!take(rp, NCB, it)) return false;
+      if (leader) {
+        const uint64_t db = kdesc(it, 0, 0);
+        const uint32_t cbs = (uint32_t)rp * 128u, id = ptx::idesc_bf16(128, rp, false, false);
+        const uint32_t d = tmem + kTmS0 + 128 * (sidx_i & 1);
+#pragma unroll 1
+        for (int k = 0; k < D / 16; ++k) ptx::umma_bf16(d, kdesc(base + kOffQ, 0, kTileCb) + kstep(k, kTileCb), db + kstep(k, cbs), id, k > 0);
+      }
+      release();
+      s_commit();
+      return true;
     };
-    const uint32_t idS = ptx::idesc_bf16(128, 128, false, true);
-    for (int si = s_begin; si < s_end && ok; ++si) {
-      const Seg sg = p.segs[si];
-      if (!(ok = wait_bar(bar(B_QFULL), q_uses & 1, sh, p.status))) break;
+    // G2: S = q̃_hi·U + q̃_lo·U into the next S slot (B MN-major, N = 128 tokens)
+    auto g2 = [&](int rk) -> bool {
+      const int rp = pad16(rk);
+      uint32_t it;
+      if (!take(rp, 2, it)) return false;
+      if (leader) {
+        const uint32_t d = tmem + kTmS0 + 128 * (sidx_i & 1);
+        const uint64_t db = mndesc(it, 0, (uint32_t)rp * 128u);
+        for (int t = 0; t < rp / 16; ++t) {
+          const uint64_t bd = db + (uint64_t)(t * 128);
+          ptx::umma_bf16(d, kdesc(base + kOffQtHi, 0, kTileCb) + kstep(t, kTileCb), bd, idS, t > 0);
+          ptx::umma_bf16(d, kdesc(base + kOffQtLo, 0, kTileCb) + kstep(t, kTileCb), bd, idS, 1);
+        }
+      }
+      release();
+      s_commit();
+      return true;
+    };
+    // G3: ã (+)= p · P_b, N = padded rank; `fresh` overwrites ã
+    auto g3 = [&](int rv, bool fresh) -> bool {
+      const int rp = pad16(rv);
+      uint32_t it;
+      if (!take(rp, 2, it)) return false;
+      if (leader) {
+        const uint64_t db = kdesc(it, 0, 0);
+        const uint32_t cbs = (uint32_t)rp * 128u, id = ptx::idesc_bf16(128, rp, false, false);
+#pragma unroll 1
+        for (int t = 0; t < kChunk / 16; ++t)
+          ptx::umma_bf16(tmem + kTmA, kdesc(base + kOffP, 0, kTileCb) + kstep(t, kTileCb), db + kstep(t, cbs), id, (t > 0 || !fresh) ? 1u : 0u);
+      }
+      release();
+      return true;
+    };
+    // G4: acc (+)= ã · Q_bᵀ, ã in the P buffer, B MN-major, N = d
+    auto g4 = [&](int rv, bool fresh) -> bool {
+      const int rp = pad16(rv);
+      uint32_t it;
+      if (!take(rp, NCB, it)) return false;
+      if (leader) {
+        const uint64_t db = mndesc(it, 0, (uint32_t)rp * 128u);
+        for (int t = 0; t < rp / 16; ++t)
+          ptx::umma_bf16(tmem + kTmAcc, kdesc(base + kOffP, 0, kTileCb) + kstep(t, kTileCb), db + (uint64_t)(t * 128), idD,
+                         (t > 0 || !fresh) ? 1u : 0u);
+      }
+      release();
+      return true;
+    };
+    // G2' (suffix): S = q · K_sufᵀ, B K-major over d, N = 128 tokens
+    auto g2s = [&]() -> bool {
+      uint32_t it;
+      if (!take(kChunk, NCB, it)) return false;
+      if (leader) {
+        const uint64_t db = kdesc(it, 0, 0);
+        const uint32_t d = tmem + kTmS0 + 128 * (sidx_i & 1), id = ptx::idesc_bf16(128, kChunk, false, false);
+#pragma unroll
+        for (int t = 0; t < D / 16; ++t) ptx::umma_bf16(d, kdesc(base + kOffQ, 0, kTileCb) + kstep(t, kTileCb), db + kstep(t, kChunk * 128u), id, t > 0);
+      }
+      release();
+      s_commit();
+      return true;
+    };
+    // G3' (suffix): acc (+)= p · V_suf, B MN-major, K = 128 tokens, N = d
+    auto g3s = [&](bool fresh) -> bool {
+      uint32_t it;
+      if (!take(kChunk, NCB, it)) return false;
+      if (leader) {
+        const uint64_t db = mndesc(it, 0, kChunk * 128u);
+#pragma unroll
+        for (int t = 0; t < kChunk / 16; ++t)
+          ptx::umma_bf16(tmem + kTmAcc, kdesc(base + kOffP, 0, kTileCb) + kstep(t, kTileCb), db + (uint64_t)(t * 128), idD,
+                         (t > 0 || !fresh) ? 1u : 0u);
+      }
+      release();
+      return true;
+    };
+    auto commit = [&](int b) {
+      if (leader) ptx::umma_commit(bar(b));
+    };
+    auto wait_q = [&]() -> bool {
+      const bool r = wait_bar(bar(B_QFULL), q_uses & 1, sh, p.status);
       ++q_uses;
       ptx::tc_fence_after();
+      return r;
+    };
+    bool bounds_ok = true;
+    for (int si = s_begin; si < s_end && bounds_ok; ++si) {
+      const Seg sg = get_seg(p, sh, s_begin, si);
       if (sg.type == 0) {
-        bool first_block = true;
-        for (int c = sg.c0; c < sg.c1 && ok;) {
-          const int b = c / p.cpb;
-          const int cend = min(sg.c1, (b + 1) * p.cpb);
-          const int nch = cend - c;
-          BlockInfo bi;
-          if (!block_info(p, sg.h, b, D, bi)) {
-            atomicOr(p.status, kStatusDecodeBounds);
-            sh->abort_flag = 1;
-            ok = false;
-            break;
-          }
-          const int rkp = pad16(bi.rk), rvp = pad16(bi.rv);
-          // G1: q̃ = Q · B_b → TMEM R (free: ã of the previous block was converted before its G4)
-          for (int r0 = 0; r0 < rkp && ok; r0 += 64) {
-            uint32_t pc;
-            if (!(ok = take(pc))) break;
-            const int np = min(64, rkp - r0);
-            if (leader)
-              for (int k = 0; k < D / 16; ++k)
-                ptx::umma_bf16(tmem + kTmR + r0, kdesc(base + kOffQ, k, kTileCb), kdesc(pc, k, kPieceCb),
-                               ptx::idesc_bf16(128, np, false, false), k > 0);
-            release();
-          }
-          if (!ok) break;
-          if (leader) {
-            ptx::umma_commit(bar(B_QTFULL));
-            if (cend == sg.c1) ptx::umma_commit(bar(B_QEMPTY));  // last read of Q in this segment
-          }
-          if (!(ok = wait_bar(bar(B_QTREADY), qt_uses & 1, sh, p.status))) break;
-          ++qt_uses;
-          ptx::tc_fence_after();
-          for (int j = 0; j <= nch && ok; ++j) {
-            if (j < nch) {
-              // G2(j): S = q̃_hi·U + q̃_lo·U
-              const uint32_t k = chunk_ix + j;
-              if (!(ok = wait_s_empty(k))) break;
-              const uint32_t dS = tmem + kTmS0 + 128 * (k & 1);
-              for (int r0 = 0; r0 < rkp && ok; r0 += 64) {
-                uint32_t pc;
-                if (!(ok = take(pc))) break;
-                const int kk = min(64, rkp - r0) / 16;
-                if (leader)
-                  for (int t = 0; t < kk; ++t) {
-                    const uint64_t bd = mndesc(pc, t);
-                    const int ka = r0 / 16 + t;
-                    ptx::umma_bf16(dS, kdesc(base + kOffQtHi, ka, kTileCb), bd, idS, ka > 0);
-                    ptx::umma_bf16(dS, kdesc(base + kOffQtLo, ka, kTileCb), bd, idS, 1);
-                  }
-                release();
-              }
-              if (!ok) break;
-              if (leader) ptx::umma_commit(bar(B_SFULL + (k & 1)));
-            }
-            if (j > 0) {
-              // G3(j-1): ã += p · P_b
-              const uint32_t k = chunk_ix + j - 1;
-              if (!(ok = wait_p_full(k))) break;
-              const uint32_t pt = base + kOffP + 32768 * (k & 1);
-              for (int r0 = 0; r0 < rvp && ok; r0 += 64) {
-                uint32_t pc;
-                if (!(ok = take(pc))) break;
-                const int np = min(64, rvp - r0);
-                if (leader)
-                  for (int t = 0; t < kChunk / 16; ++t)
-                    ptx::umma_bf16(tmem + kTmR + r0, kdesc(pt, t, kTileCb), kdesc(pc, t, kPieceCb),
-                                   ptx::idesc_bf16(128, np, false, false), (t > 0 || j > 1) ? 1u : 0u);
-                release();
-              }
-              if (!ok) break;
-              if (leader) ptx::umma_commit(bar(B_PEMPTY + (k & 1)));
-            }
-          }
-          if (!ok) break;
-          chunk_ix += nch;
-          if (leader) ptx::umma_commit(bar(B_ATFULL));
-          // G4: acc += ã · Q_bᵀ once the softmax warps have moved ã to smem
-          if (!(ok = wait_bar(bar(B_ATREADY), at_uses & 1, sh, p.status))) break;
-          ++at_uses;
-          ptx::tc_fence_after();
-          for (int r0 = 0; r0 < rvp && ok; r0 += 64) {
-            uint32_t pc;
-            if (!(ok = take(pc))) break;
-            const int kk = min(64, rvp - r0) / 16;
-            if (leader)
-              for (int t = 0; t < kk; ++t) {
-                const int ka = r0 / 16 + t;
-                ptx::umma_bf16(tmem + kTmAcc, kdesc(base + kOffQtHi, ka, kTileCb), mndesc(pc, t),
-                               ptx::idesc_bf16(128, D, false, true), (ka > 0 || !first_block) ? 1u : 0u);
-              }
-            release();
-          }
-          if (!ok) break;
-          c = cend;
-          first_block = false;
+        BlockWalk w{sg.c0, sg.c1, p.cpb};
+        BlockInfo bi, bn, prev;
+        int kb = 0;
+        bool have_prev = false;
+        if (!seg_block(p, sh, si - s_begin, kb, sg.h, w.block(), D, bi)) {
+          bounds_ok = false;
+          break;
         }
-        if (ok && leader) ptx::umma_commit(bar(B_ACCFULL));
+        if (ok) {
+          ok = wait_q() && g1(bi.rk);
+          if (ok && !w.has_next()) commit(B_QEMPTY);  // last read of Q in this segment
+        }
+        while (true) {
+          const int n = w.chunks();
+          const bool next = w.has_next();
+          bool next_is_last = false;
+          if (next) {
+            if (!seg_block(p, sh, si - s_begin, kb + 1, sg.h, w.block() + 1, D, bn)) {
+              bounds_ok = false;
+              break;
+            }
+            BlockWalk w2 = w;
+            w2.next();
+            next_is_last = !w2.has_next();
+          }
+          auto g1_next = [&]() -> bool {
+            if (!g1(bn.rk)) return false;
+            if (next_is_last) commit(B_QEMPTY);
+            return true;
+          };
+          sync_wg(kSigQt);
+          if (ok) {
+            ok = g2(bi.rk);
+            if (ok && n >= 2) ok = g2(bi.rk);
+            else if (ok && next) ok = g1_next();
+          }
+          if (have_prev) {
+            sync_wg(kSigAt);
+            if (ok) {
+              ok = g4(prev.rv, kb == 1);
+              commit(B_PEMPTY);
+            }
+          }
+          for (int j = 0; j < n; ++j) {
+            sync_wg(kSigP);
+            if (ok) {
+              ok = g3(bi.rv, j == 0);
+              commit(j + 1 < n ? B_PEMPTY : B_ATFULL);
+              if (ok && j + 2 < n) ok = g2(bi.rk);
+              else if (ok && j + 2 == n && next) ok = g1_next();
+            }
+          }
+          if (!next) break;
+          prev = bi;
+          have_prev = true;
+          w.next();
+          bi = bn;
+          ++kb;
+        }
+        if (!bounds_ok) break;
+        sync_wg(kSigAt);
+        if (ok) {
+          ok = g4(bi.rv, kb == 0);
+          commit(B_PEMPTY);
+          commit(B_ACCFULL);
+        }
       } else {
-        const int nch = sg.c1 - sg.c0;
-        for (int j = 0; j <= nch && ok; ++j) {
-          if (j < nch) {
-            // G2'(j): S = q · K_sufᵀ, two 64-token pieces
-            const uint32_t k = chunk_ix + j;
-            if (!(ok = wait_s_empty(k))) break;
-            const uint32_t dS = tmem + kTmS0 + 128 * (k & 1);
-            for (int pi = 0; pi < 2 && ok; ++pi) {
-              uint32_t pc;
-              if (!(ok = take(pc))) break;
-              if (leader)
-                for (int t = 0; t < D / 16; ++t)
-                  ptx::umma_bf16(dS + 64 * pi, kdesc(base + kOffQ, t, kTileCb), kdesc(pc, t, kPieceCb),
-                                 ptx::idesc_bf16(128, 64, false, false), t > 0);
-              release();
+        const int n = sg.c1 - sg.c0;
+        if (ok) {
+          ok = wait_q() && g2s();
+          if (ok && n >= 2) ok = g2s();
+          if (ok && n <= 2) commit(B_QEMPTY);
+        }
+        for (int j = 0; j < n; ++j) {
+          sync_wg(kSigP);
+          if (ok) {
+            ok = g3s(j == 0);
+            commit(B_PEMPTY);
+            if (ok && j + 2 < n) {
+              ok = g2s();
+              if (ok && j + 2 == n - 1) commit(B_QEMPTY);
             }
-            if (!ok) break;
-            if (leader) {
-              ptx::umma_commit(bar(B_SFULL + (k & 1)));
-              if (j == nch - 1) ptx::umma_commit(bar(B_QEMPTY));
-            }
-          }
-          if (j > 0) {
-            // G3'(j-1): acc += p · V_suf
-            const uint32_t k = chunk_ix + j - 1;
-            if (!(ok = wait_p_full(k))) break;
-            const uint32_t pt = base + kOffP + 32768 * (k & 1);
-            for (int pi = 0; pi < 2 && ok; ++pi) {
-              uint32_t pc;
-              if (!(ok = take(pc))) break;
-              if (leader)
-                for (int t = 0; t < 4; ++t)
-                  ptx::umma_bf16(tmem + kTmAcc, kdesc(pt, 4 * pi + t, kTileCb), mndesc(pc, t),
-                                 ptx::idesc_bf16(128, D, false, true), (j > 1 || pi > 0 || t > 0) ? 1u : 0u);
-              release();
-            }
-            if (!ok) break;
-            if (leader) ptx::umma_commit(bar(B_PEMPTY + (k & 1)));
           }
         }
-        if (!ok) break;
-        chunk_ix += nch;
-        if (leader) ptx::umma_commit(bar(B_ACCFULL));
+        if (ok) commit(B_ACCFULL);
       }
     }
     // drain: every MMA issued must complete before TMEM is freed
-    if (leader) ptx::umma_commit(bar(B_FINAL));
+    commit(B_FINAL);
     __syncwarp();
     wait_bar(bar(B_FINAL), 0, sh, p.status, true);
   } else {
-    // ==================================================================== softmax warpgroup
+    // ==================================================================== softmax warpgroup (warps 2..5)
+    // One thread per row and TMEM lane; signals the MMA warp through named barriers when its smem output
+    // (q̃, P or ã) is complete.
     const int quarter = warp & 3;
     const int row = 32 * quarter + lane;
     const uint32_t tl = tmem + ((uint32_t)(32 * quarter) << 16);
-    uint32_t chunk_ix = 0, qt_uses = 0, at_uses = 0, acc_uses = 0;
+    uint32_t sidx = 0, pk = 0, at_uses = 0, acc_uses = 0;  // consumption counters
     bool ok = true;
-    // one arrival per warp on the barriers the warpgroup signals (init count 4)
-    auto arrive = [&](int b) {
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(b));
+    auto signal = [&](int id) {  // arrive on the MMA warp's named barrier `id` (does not wait)
+      ptx::tc_fence_before();
+      asm volatile("bar.arrive %0, 160;" ::"r"(id) : "memory");
     };
-    for (int si = s_begin; si < s_end && ok; ++si) {
-      const Seg sg = p.segs[si];
-      // a warp whose 32 rows are all padding only keeps the barrier protocol
-      const bool active = 32 * quarter < sg.rows;
-      float m_used = -INFINITY, l = 0.f;
-      bool first_chunk = true;
-      const bool prefix = sg.type == 0;
-      int c = sg.c0;
-      bool first_block = true;
-      while (c < sg.c1 && ok) {
-        int cend, rv = 0, rvp = 0;
-        if (prefix) {
-          const int b = c / p.cpb;
-          cend = min(sg.c1, (b + 1) * p.cpb);
-          BlockInfo bi;
-          if (!block_info(p, sg.h, b, D, bi)) {
-            ok = false;
-            break;
-          }
-          rv = bi.rv;
-          rvp = pad16(bi.rv);
-          const int rk = bi.rk, rkp = pad16(bi.rk);
-          // q̃ (fp32, TMEM) → bf16 hi + lo in smem, columns >= r zeroed
-          if (!(ok = wait_bar(bar(B_QTFULL), qt_uses & 1, sh, p.status))) break;
-          ++qt_uses;
-          ptx::tc_fence_after();
-          if (active) {
-            for (int half = 0; half < rkp; half += 64) {
-              float v[64];
-#pragma unroll
-              for (int q = 0; q < 4; ++q) ptx::tmem_ld16(tl + kTmR + half + 16 * q, v + 16 * q);
-              ptx::tmem_wait_ld();
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int col = half + 16 * q;
-                if (col < rkp) {
-                  uint32_t hi[8], lo[8];
-#pragma unroll
-                  for (int e = 0; e < 16; e += 2) {
-                    const float a = (col + e < rk) ? v[16 * q + e] : 0.f;
-                    const float b2 = (col + e + 1 < rk) ? v[16 * q + e + 1] : 0.f;
-                    const uint32_t h2 = ptx::pack_bf16(a, b2);
-                    hi[e / 2] = h2;
-                    lo[e / 2] =
-                        ptx::pack_bf16(a - __uint_as_float(h2 << 16), b2 - __uint_as_float(h2 & 0xFFFF0000u));
-                  }
-                  st_tile8(base + kOffQtHi, row, col, hi[0], hi[1], hi[2], hi[3]);
-                  st_tile8(base + kOffQtHi, row, col + 8, hi[4], hi[5], hi[6], hi[7]);
-                  st_tile8(base + kOffQtLo, row, col, lo[0], lo[1], lo[2], lo[3]);
-                  st_tile8(base + kOffQtLo, row, col + 8, lo[4], lo[5], lo[6], lo[7]);
-                }
-              }
-            }
-            ptx::fence_async_smem();
-          }
-          ptx::tc_fence_before();
-          arrive(B_QTREADY);
-        } else {
-          cend = sg.c1;
-        }
-        for (int cc = c; cc < cend && ok; ++cc) {
-          const uint32_t k = chunk_ix;
-          const uint32_t slot = k & 1;
-          if (!(ok = wait_bar(bar(B_SFULL + slot), (k >> 1) & 1, sh, p.status))) break;
-          ptx::tc_fence_after();
-          float s[kChunk];
-          if (active) {
-#pragma unroll
-            for (int q = 0; q < kChunk / 16; ++q) ptx::tmem_ld16(tl + kTmS0 + 128 * slot + 16 * q, s + 16 * q);
-            ptx::tmem_wait_ld();
-          }
-          ptx::tc_fence_before();
-          arrive(B_SEMPTY + slot);
-          float alpha = 1.f;
-          bool grow = false;
-          if (active) {
-            if (!prefix) {
-              const int valid = p.S - cc * kChunk;
-#pragma unroll
-              for (int j = 0; j < kChunk; ++j)
-                if (j >= valid) s[j] = -INFINITY;
-            }
-            // tree max (8 independent lanes of reduction, then fold)
-            float m8[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) m8[e] = s[e];
-#pragma unroll
-            for (int j = 8; j < kChunk; j += 8)
-#pragma unroll
-              for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], s[j + e]);
-            float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-            mx *= p.c;
-            // keep the running max in use unless the chunk exceeds it by more than 2^8 (then rescale)
-            grow = !first_chunk && mx > m_used + 8.f;
-            if (grow) {
-              alpha = ptx::ex2(m_used - mx);
-              m_used = mx;
-              l *= alpha;
-            }
-            if (first_chunk) m_used = mx;
-          }
-          if (__any_sync(0xffffffffu, grow)) {
-            // rare: rescale what this warp's rows accumulated so far (alpha = 1 for rows that did not grow)
-            const bool have_at = prefix && cc > c;  // ã holds earlier chunks of this block
-            const bool have_acc = prefix ? !first_block : true;
-            if (have_at || !prefix) {
-              // the previous G3 must have landed before ã (or the suffix acc) is touched
-              if (!(ok = wait_bar(bar(B_PEMPTY + ((k - 1) & 1)), ((k - 1) >> 1) & 1, sh, p.status))) break;
-              ptx::tc_fence_after();
-            }
-            if (have_at) {
-              for (int c16 = 0; c16 < rvp; c16 += 16) {
-                float v[16];
-                ptx::tmem_ld16(tl + kTmR + c16, v);
-                ptx::tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] *= alpha;
-                ptx::tmem_st16(tl + kTmR + c16, v);
-              }
-            }
-            if (have_acc) {
-              for (int c16 = 0; c16 < D; c16 += 16) {
-                float v[16];
-                ptx::tmem_ld16(tl + kTmAcc + c16, v);
-                ptx::tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] *= alpha;
-                ptx::tmem_st16(tl + kTmAcc + c16, v);
-              }
-            }
-            ptx::tmem_wait_st();
-          }
-          first_chunk = false;
-          // p = exp2(S·c − m), row sum, bf16 tile
-          if (!(ok = wait_bar(bar(B_PEMPTY + slot), ((k >> 1) & 1) ^ 1, sh, p.status))) break;
-          if (active) {
-            const uint32_t pt = base + kOffP + 32768 * slot;
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial row sums
-#pragma unroll
-            for (int g8 = 0; g8 < kChunk / 8; ++g8) {
-              uint32_t w[4];
-#pragma unroll
-              for (int e = 0; e < 8; e += 2) {
-                const float a = ptx::ex2(fmaf(s[8 * g8 + e], p.c, -m_used));
-                const float b2 = ptx::ex2(fmaf(s[8 * g8 + e + 1], p.c, -m_used));
-                ls[e / 2] += a + b2;
-                w[e / 2] = ptx::pack_bf16(a, b2);
-              }
-              st_tile8(pt, row, 8 * g8, w[0], w[1], w[2], w[3]);
-            }
-            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-            ptx::fence_async_smem();
-          }
-          ptx::tc_fence_before();
-          arrive(B_PFULL + slot);
-          ++chunk_ix;
-        }
-        if (!ok) break;
-        if (prefix) {
-          // ã (fp32, TMEM) → bf16 in smem (over q̃_hi, whose readers are done), columns >= r zeroed
-          if (!(ok = wait_bar(bar(B_ATFULL), at_uses & 1, sh, p.status))) break;
-          ++at_uses;
-          ptx::tc_fence_after();
-          if (active) {
-            for (int half = 0; half < rvp; half += 64) {
-              float v[64];
-#pragma unroll
-              for (int q = 0; q < 4; ++q) ptx::tmem_ld16(tl + kTmR + half + 16 * q, v + 16 * q);
-              ptx::tmem_wait_ld();
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int col = half + 16 * q;
-                if (col < rvp) {
-                  uint32_t w[8];
-#pragma unroll
-                  for (int e = 0; e < 16; e += 2)
-                    w[e / 2] = ptx::pack_bf16(col + e < rv ? v[16 * q + e] : 0.f,
-                                              col + e + 1 < rv ? v[16 * q + e + 1] : 0.f);
-                  st_tile8(base + kOffQtHi, row, col, w[0], w[1], w[2], w[3]);
-                  st_tile8(base + kOffQtHi, row, col + 8, w[4], w[5], w[6], w[7]);
-                }
-              }
-            }
-            ptx::fence_async_smem();
-          }
-          ptx::tc_fence_before();
-          arrive(B_ATREADY);
-        }
-        c = cend;
-        first_block = false;
+    // ---------------- softmax helpers (all four warps)
+    // q̃ of a block (fp32, in the next S slot) → bf16 hi + lo in smem, columns >= r zeroed
+    // Every helper below ends with the warpgroup barrier, also after a failed wait, so that the four warps
+    // always execute the same sequence of named barriers (which have no time limit).
+    auto convert_qt = [&](bool active, int rk) -> bool {
+      if (!wait_bar(bar(B_SFULL + (sidx & 1)), (sidx >> 1) & 1, sh, p.status)) {
+        ++sidx;
+        signal(kSigQt);
+        return false;
       }
-      if (!ok) break;
-      // segment result: (m, l, acc) of this row
-      if (!(ok = wait_bar(bar(B_ACCFULL), acc_uses & 1, sh, p.status))) break;
+      ptx::tc_fence_after();
+      const uint32_t src = tl + kTmS0 + 128 * (sidx & 1);
+      if (active) {
+        for (int c16 = 0; c16 < pad16(rk); c16 += 16) {
+          float v[16];
+          ptx::tmem_ld16(src + c16, v);
+          ptx::tmem_wait_ld();
+          uint32_t hi[8], lo[8];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            const float a = (c16 + e < rk) ? v[e] : 0.f;
+            const float b2 = (c16 + e + 1 < rk) ? v[e + 1] : 0.f;
+            const uint32_t h2 = ptx::pack_bf16(a, b2);
+            hi[e / 2] = h2;
+            lo[e / 2] = ptx::pack_bf16(a - __uint_as_float(h2 << 16), b2 - __uint_as_float(h2 & 0xFFFF0000u));
+          }
+          st_tile8(base + kOffQtHi, row, c16, hi[0], hi[1], hi[2], hi[3]);
+          st_tile8(base + kOffQtHi, row, c16 + 8, hi[4], hi[5], hi[6], hi[7]);
+          st_tile8(base + kOffQtLo, row, c16, lo[0], lo[1], lo[2], lo[3]);
+          st_tile8(base + kOffQtLo, row, c16 + 8, lo[4], lo[5], lo[6], lo[7]);
+        }
+        ptx::fence_async_smem();
+      }
+      ++sidx;
+      signal(kSigQt);
+      return true;
+    };
+    // ã (fp32, TMEM) → bf16 in the P buffer (its last reader, G3, has completed), columns >= r zeroed
+    auto convert_at = [&](bool active, int rv) -> bool {
+      if (!wait_bar(bar(B_ATFULL), at_uses & 1, sh, p.status)) {
+        ++at_uses;
+        signal(kSigAt);
+        return false;
+      }
+      ++at_uses;
+      ptx::tc_fence_after();
+      if (active) {
+        for (int c16 = 0; c16 < pad16(rv); c16 += 16) {
+          float v[16];
+          ptx::tmem_ld16(tl + kTmA + c16, v);
+          ptx::tmem_wait_ld();
+          uint32_t wv[8];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2)
+            wv[e / 2] = ptx::pack_bf16(c16 + e < rv ? v[e] : 0.f, c16 + e + 1 < rv ? v[e + 1] : 0.f);
+          st_tile8(base + kOffP, row, c16, wv[0], wv[1], wv[2], wv[3]);
+          st_tile8(base + kOffP, row, c16 + 8, wv[4], wv[5], wv[6], wv[7]);
+        }
+        ptx::fence_async_smem();
+      }
+      signal(kSigAt);
+      return true;
+    };
+    // one chunk of scores: online softmax, probabilities into the P buffer.  `rescale_at` / `rescale_acc`
+    // say whether ã / acc hold earlier chunks that a grown running max must rescale.
+    auto chunk = [&](bool active, int valid, bool& first_chunk, float& m_used, float& l, bool rescale_at,
+                     int rvp, bool rescale_acc) -> bool {
+      const uint32_t slot = sidx & 1;
+      if (!wait_bar(bar(B_SFULL + slot), (sidx >> 1) & 1, sh, p.status)) {
+        ++sidx;
+        ++pk;
+        signal(kSigP);
+        return false;
+      }
+      ptx::tc_fence_after();
+      ++sidx;
+      const uint32_t src = tl + kTmS0 + 128 * slot;
+      float alpha = 1.f;
+      bool grow = false;
+      if (active) {
+        // pass 1 over the scores (32 columns at a time, compact loop): the chunk's row max
+        float m8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
+#pragma unroll 1
+        for (int c32 = 0; c32 < kChunk; c32 += 32) {
+          float s[32];
+          ptx::tmem_ld32(src + c32, s);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 32; t += 8)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], c32 + t + e < valid ? s[t + e] : -INFINITY);
+        }
+        float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        mx *= p.c;
+        // keep the running max in use unless the chunk exceeds it by more than 2^8 (then rescale)
+        grow = !first_chunk && mx > m_used + 8.f;
+        if (grow) {
+          alpha = ptx::ex2(m_used - mx);
+          m_used = mx;
+          l *= alpha;
+        }
+        if (first_chunk) m_used = mx;
+      }
+      if (pk > 0) {
+        // the previous chunk's G3 (or the previous block's G4, which read ã from the P buffer) has landed
+        if (!wait_bar(bar(B_PEMPTY), (pk - 1) & 1, sh, p.status)) {
+          ++pk;
+          signal(kSigP);
+          return false;
+        }
+        ptx::tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, grow)) {
+        // rare: rescale what this warp's rows accumulated so far (alpha = 1 for rows that did not grow)
+        if (rescale_at) {
+          for (int c16 = 0; c16 < rvp; c16 += 16) {
+            float v[16];
+            ptx::tmem_ld16(tl + kTmA + c16, v);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] *= alpha;
+            ptx::tmem_st16(tl + kTmA + c16, v);
+          }
+        }
+        if (rescale_acc) {
+          for (int c16 = 0; c16 < D; c16 += 16) {
+            float v[16];
+            ptx::tmem_ld16(tl + kTmAcc + c16, v);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] *= alpha;
+            ptx::tmem_st16(tl + kTmAcc + c16, v);
+          }
+        }
+        ptx::tmem_wait_st();
+      }
+      first_chunk = false;
+      if (active) {
+        // pass 2: p = exp2(S·c − m) as bf16 into the P buffer, row sum in fp32 (32 columns at a time)
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial row sums
+#pragma unroll 1
+        for (int c32 = 0; c32 < kChunk; c32 += 32) {
+          float s[32];
+          ptx::tmem_ld32(src + c32, s);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int g8 = 0; g8 < 4; ++g8) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              const int t = c32 + 8 * g8 + e;
+              const float a = t < valid ? ptx::ex2(fmaf(s[8 * g8 + e], p.c, -m_used)) : 0.f;
+              const float b2 = t + 1 < valid ? ptx::ex2(fmaf(s[8 * g8 + e + 1], p.c, -m_used)) : 0.f;
+              ls[e / 2] += a + b2;
+              wv[e / 2] = ptx::pack_bf16(a, b2);
+            }
+            st_tile8(base + kOffP, row, c32 + 8 * g8, wv[0], wv[1], wv[2], wv[3]);
+          }
+        }
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        ptx::fence_async_smem();
+      }
+      ++pk;
+      signal(kSigP);
+      return true;
+    };
+    auto write_partial = [&](const Seg& sg, bool active, float m_used, float l) -> bool {
+      if (!wait_bar(bar(B_ACCFULL), acc_uses & 1, sh, p.status)) {
+        ++acc_uses;
+        return false;
+      }
       ++acc_uses;
       ptx::tc_fence_after();
       if (active) {
         float* dst = p.part_acc + ((int64_t)sg.pid * 128 + row) * D;
-        for (int half = 0; half < D; half += 64) {
-          float v[64];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) ptx::tmem_ld16(tl + kTmAcc + half + 16 * q, v + 16 * q);
+        for (int c16 = 0; c16 < D; c16 += 16) {
+          float v[16];
+          ptx::tmem_ld16(tl + kTmAcc + c16, v);
           ptx::tmem_wait_ld();
           if (row < sg.rows) {
 #pragma unroll
-            for (int e = 0; e < 64; e += 4)
-              *reinterpret_cast<float4*>(dst + half + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+            for (int e = 0; e < 16; e += 4)
+              *reinterpret_cast<float4*>(dst + c16 + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
           }
         }
         if (row < sg.rows) p.part_ml[(int64_t)sg.pid * 128 + row] = make_float2(m_used, l);
       }
-      ptx::tc_fence_before();
+      // acc is read before any MMA of the next segment writes it: those follow a later signal
+      return true;
+    };
+    auto fail_bounds = [&]() {
+      if (warp == 2 && lane == 0) atomicOr(p.status, kStatusDecodeBounds);
+      sh->abort_flag = 1;
+      return false;
+    };
+
+    // The loops below depend only on the work list, never on `ok`: after a failure (an expired wait, which
+    // also raises the CTA's abort flag so that later waits return at once) the warps still walk the same
+    // steps and barriers, skipping the work, and then leave together.
+    bool bounds_ok = true;
+    for (int si = s_begin; si < s_end && bounds_ok; ++si) {
+      const Seg sg = get_seg(p, sh, s_begin, si);
+      const bool active = 32 * quarter < sg.rows;  // a warp whose rows are all padding keeps the protocol only
+      float m_used = -INFINITY, l = 0.f;
+      bool first_chunk = true;
+      if (sg.type == 0) {
+        BlockWalk w{sg.c0, sg.c1, p.cpb};
+        BlockInfo bi, bn, prev;
+        int kb = 0;
+        bool have_prev = false;
+        if (!seg_block(p, sh, si - s_begin, kb, sg.h, w.block(), D, bi)) {
+          bounds_ok = fail_bounds();
+          break;
+        }
+        while (true) {
+          const int n = w.chunks();
+          const bool next = w.has_next();
+          bool next_is_last = false;
+          if (next) {
+            if (!seg_block(p, sh, si - s_begin, kb + 1, sg.h, w.block() + 1, D, bn)) {
+              bounds_ok = fail_bounds();
+              break;
+            }
+            BlockWalk w2 = w;
+            w2.next();
+            next_is_last = !w2.has_next();
+          }
+          // q̃ of this block to smem, then the first two S-slot uses
+          ok = convert_qt(active, bi.rk) && ok;
+          // the previous block's ã to smem and its expansion G4
+          if (have_prev) {
+            ok = convert_at(active, prev.rv) && ok;
+          }
+          for (int j = 0; j < n; ++j) {
+            ok = chunk(active, kChunk, first_chunk, m_used, l, j > 0, pad16(bi.rv), have_prev) && ok;
+          }
+          if (!next) break;
+          prev = bi;
+          have_prev = true;
+          w.next();
+          bi = bn;
+          ++kb;
+        }
+        if (!bounds_ok) break;
+        // the last block's ã and G4, then the segment's result
+        ok = convert_at(active, bi.rv) && ok;
+        ok = write_partial(sg, active, m_used, l) && ok;
+      } else {
+        const int n = sg.c1 - sg.c0;
+        for (int j = 0; j < n; ++j) {
+          const int valid = min(kChunk, p.S - (sg.c0 + j) * kChunk);
+          ok = chunk(active, valid, first_chunk, m_used, l, false, 0, j > 0) && ok;
+        }
+        ok = write_partial(sg, active, m_used, l) && ok;
+      }
     }
   }
 
