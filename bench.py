@@ -37,7 +37,7 @@ METRIC = "compressed-KV decode tokens/s at Qwen2.5-7B shape; achieved HBM GB/s v
 def _args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--steps", type=int, default=20000)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", default="milo", choices=["milo", "reference"])
     p.add_argument("--workload", default="qwen2.5-7b-layer")
@@ -56,28 +56,52 @@ def _peaks():
 
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+    """Samples SM clocks and throttle reasons every 20 ms while the timed region runs (NVML; nvidia-smi
+    when NVML cannot be loaded)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clocks-event reason bits
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap"}
 
     def __init__(self, index: int):
         self.index = index
-        self.rows = []
+        self.rows = []  # (sm_mhz, sm_max_mhz, reason bits)
         self._stop = threading.Event()
         self._t = None
 
+    def _sample_nvml(self, nv, h):
+        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        try:
+            bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+        except Exception:
+            bits = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+        return float(sm), float(mx), int(bits)
+
+    def _sample_smi(self):
+        fields = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_power_cap")
+        r = subprocess.run(["nvidia-smi", f"--id={self.index}", f"--query-gpu={fields}",
+                            "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
+        v = [x.strip() for x in r.stdout.strip().split(",")]
+        bits = sum(b for b, x in zip((0x8, 0x40, 0x20, 0x4), v[2:]) if x == "Active")
+        return float(v[0]), float(v[1]), bits
+
     def _run(self):
-        while not self._stop.is_set():
+        nv = h = None
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByIndex(self.index)
+        except Exception:
+            nv = None
+        while True:
             try:
-                r = subprocess.run(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                                    "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
-                if r.returncode == 0 and r.stdout.strip():
-                    self.rows.append([x.strip() for x in r.stdout.strip().split(",")])
+                self.rows.append(self._sample_nvml(nv, h) if nv else self._sample_smi())
             except Exception:
                 pass
-            self._stop.wait(0.2)
+            if self._stop.wait(0.02 if nv else 0.2):
+                break
 
     def __enter__(self):
         self._t = threading.Thread(target=self._run, daemon=True)
@@ -91,11 +115,8 @@ class ClockSampler:
     def summary(self):
         if not self.rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in self.rows for i in range(4) if len(r) > 5 + i and r[5 + i] == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+        reasons = sorted({name for _, _, bits in self.rows for b, name in self.REASONS.items() if bits & b})
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": max(r[1] for r in self.rows),
                 "reasons": reasons, "samples": len(self.rows)}
 
 

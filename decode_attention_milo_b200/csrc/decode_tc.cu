@@ -5,19 +5,21 @@
 // With K_b ≈ U_b·B_bᵀ and V_b ≈ P_b·Q_bᵀ (tok rows = U_bᵀ / P_bᵀ, dim rows =
 // B_bᵀ / Q_bᵀ), for the query rows of one KV head (batch × GQA group, M = 128):
 //   G1  q̃  = Q · B_b                  TMEM fp32, then split into bf16 hi + lo in smem
-//   G2  S   = q̃ · U_bᵀ                per 128-token chunk, two MMAs (hi, lo)
-//       p   = exp2(S·scale·log2e − m)  online softmax on the CUDA cores
-//   G3  ã  += p · P_b                 TMEM fp32
-//   G4  acc += ã · Q_bᵀ               once per block, TMEM fp32
+//   G2  S   = q̃ · U_bᵀ                per 128-token chunk, two MMAs (hi, lo) per k-step
+//       p   = exp2(S·scale·log2e − m)  online softmax on the CUDA cores, packed bf16 back into TMEM
+//   G3  ã  += p · P_b                 A operand p read from TMEM, fp32 in TMEM
+//   G4  acc += ã · Q_bᵀ               once per block, ã packed bf16 in TMEM as the A operand
 // and for each query's uncompressed suffix S = q·K_sufᵀ, acc += p·V_suf.
 // A block's factors are read from HBM once and shared by every row.
 //
 // One persistent CTA per SM walks a host-built list of segments (a KV head's
 // row tile over a contiguous range of 128-token chunks, or one query's suffix
-// chunks), balanced by bytes.  Warp 0 issues TMA loads into a 4-stage ring in
-// exactly the order warp 1 consumes them; warp 1 issues tcgen05.mma; warps
-// 2..5 (one per TMEM lane quarter, one thread per row) run the softmax and the
-// TMEM↔smem conversions.  Each segment leaves a partial (m, l, acc) that the
+// chunks), balanced by estimated time.  Warp 0 issues TMA loads into a byte
+// ring in exactly the order warp 1 consumes them; warp 1 issues tcgen05.mma;
+// warps 4..11 (two warpgroups splitting each tile by columns, one thread per
+// row and TMEM lane) run the softmax and the TMEM conversions.  Scores use two
+// TMEM slots, so the softmax of one chunk overlaps G3 of the previous chunk
+// and G2 of the next.  Each segment leaves a partial (m, l, acc) that the
 // combine kernel merges per output row.
 //
 // Every wait is bounded (1 s): on expiry the kernel records
@@ -37,9 +39,22 @@
 namespace milo {
 namespace {
 
-constexpr int kThreads = 192;        // warp 0: TMA producer; warp 1: MMA issuer; warps 2..5: softmax
-constexpr int kSigQt = 1, kSigP = 2, kSigAt = 3;  // named barriers: softmax warps → MMA warp
-constexpr int kRingBytes = 94208;   // TMA ring: variable-size items, each one contiguous tile
+// warp 0: TMA producer; warp 1: MMA issuer; warps kSoftWarp0 .. kSoftWarp0 + 7: softmax (with kSoftWarp0 = 4,
+// warps 2 and 3 are idle and warpgroup 0 holds only the producer and the issuer).
+constexpr int kSoftWarp0 = 2;
+constexpr int kThreads = 32 * (kSoftWarp0 + 8);
+// Register split (setmaxnreg, needs kSoftWarp0 = 4): warpgroup 0 gives registers to the two softmax
+// warpgroups.  The split must fit in what the launch allocates (kThreads × kLaunchRegs), or the increase
+// would wait forever: the host refuses a build whose kernel was allocated fewer registers.
+constexpr bool kRegSplit = false;
+constexpr int kRegsLow = 120, kRegsHigh = 192, kLaunchRegs = 168;
+static_assert(!kRegSplit || (kSoftWarp0 == 4 && 128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs),
+              "register split exceeds the launch");
+constexpr int kSigThreads = 288;  // softmax warps + MMA warp on a signal barrier
+// named barriers (0 is __syncthreads): softmax warps → MMA warp (P alternates by S slot), one per TMEM
+// lane quarter for its two softmax warps, and one for all softmax warps
+constexpr int kSigQt = 1, kSigAt = 2, kSigP0 = 3, kPairBar0 = 5, kSoftBar = 9;
+constexpr int kRingBytes = 122880;  // TMA ring: variable-size items, each one contiguous tile
 constexpr int kItemSlots = 16;       // items in flight at most (one FULL/EMPTY barrier pair each)
 constexpr int kChunk = 128;          // tokens per score chunk
 constexpr uint64_t kWaitNs = 1000000000ull;
@@ -48,27 +63,30 @@ constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr int kOffQ = 0;          // [cb][128 rows][128 B]  query rows, K-major over d
 constexpr int kOffQtHi = 32768;   // [cb][128][128 B]  q̃ high part, K-major over rank
 constexpr int kOffQtLo = 65536;   // [cb][128][128 B]  q̃ low part
-constexpr int kOffP = 98304;      // [cb][128][128 B]  probabilities (K-major over tokens); then ã for G4
-constexpr int kOffRing = 131072;  // kRingBytes of items laid out [64-column block][rows][128 B]
-constexpr int kOffBar = kOffRing + kRingBytes;             // 225280: barriers, then the Shared block
-constexpr int kBarRegion = 4096;
+constexpr int kOffRing = 98304;   // kRingBytes of items laid out [64-column block][rows][128 B]
+constexpr int kOffBar = kOffRing + kRingBytes;             // 221184: barriers, then the Shared block
+constexpr int kBarRegion = 8192;
 constexpr int kSmemBytes = kOffBar + kBarRegion + 1024;     // + alignment slack (230400)
 constexpr uint32_t kTileCb = 16384;  // column-block stride of a 128-row tile
 constexpr int kMaxSegsSmem = 16, kMaxBlocksSmem = 64;  // per-CTA work tables staged in smem
 
 // TMEM columns: acc [0,128), two S slots [128,256) and [256,384) (q̃ of a block also passes through
-// an S slot), ã [384,512)
+// an S slot; p is packed over the scores it came from), ã [384,512) (packed in place for G4)
 constexpr uint32_t kTmAcc = 0, kTmS0 = 128, kTmA = 384;
+
+// TMEM column, relative to its region, of k-step t (16 bf16) of an A operand that the two softmax
+// warpgroups packed in place: warpgroup w holds K indices [64w, 64w + 64) in columns [64w, 64w + 32).
+__device__ __forceinline__ uint32_t ta_col(int t) { return (uint32_t)(64 * (t >> 2) + 8 * (t & 3)); }
 
 enum Bar {
   B_FULL = 0,
   B_EMPTY = B_FULL + kItemSlots,
   B_QFULL = B_EMPTY + kItemSlots,
   B_QEMPTY,
-  B_SFULL,
-  B_PEMPTY = B_SFULL + 2,
-  B_ATFULL,
-  B_ACCFULL,
+  B_SFULL,                // [2] S slot written (G1 / G2 / G2')
+  B_SFREE = B_SFULL + 2,  // [2] p in the S slot read (G3 / G3')
+  B_ATFULL = B_SFREE + 2, // ã of a block complete
+  B_ACCDONE,              // acc written (G4, or a suffix segment's last G3')
   B_FINAL,
   B_COUNT
 };
@@ -100,6 +118,26 @@ struct BlockInfo {
   int64_t rowk, rowv;
 };
 
+// Tensor maps of one row-major bf16 operand array (rows of 64 or 128 columns): 2D maps with boxes of
+// 16, 32, 64 and 128 rows × 64 columns, and for 128-column arrays 3D maps (x: 64 columns, y: rows,
+// z: the two 64-column blocks) whose box of h rows × both column blocks lands in shared memory as
+// [column block][h][128 B], one instruction for a whole item.
+struct RowMaps {
+  CUtensorMap m2[4];
+  CUtensorMap m3[4];
+};
+struct Maps {
+  RowMaps tok, dim, ksuf, vsuf;  // the suffix maps use the 128-row boxes only
+  CUtensorMap qpre, qsuf;
+  CUtensorMap pacc;  // partial accumulators [segments · 128][d] fp32, boxes of 128 rows × 32 columns
+};
+
+__device__ __forceinline__ const CUtensorMap* map_of(const RowMaps& m, bool three_d, int hi) {
+  // constant indices: the result stays an address in the kernel-parameter space
+  if (three_d) return hi == 0 ? &m.m3[0] : hi == 1 ? &m.m3[1] : hi == 2 ? &m.m3[2] : &m.m3[3];
+  return hi == 0 ? &m.m2[0] : hi == 1 ? &m.m2[1] : hi == 2 ? &m.m2[2] : &m.m2[3];
+}
+
 // Per-CTA state in shared memory: the CTA's segments and the rank / row offset of every block they
 // touch, staged once at start so that no role reads them from global memory inside the pipeline.
 struct Shared {
@@ -111,6 +149,8 @@ struct Shared {
   Seg segs[kMaxSegsSmem];
   BlockInfo blocks[kMaxBlocksSmem];
   uint32_t pos_log[kItemSlots], len_log[kItemSlots];  // producer's record of the items in flight
+  float mx_x[2][2][128];  // row maxima exchanged by the two softmax warpgroups (double-buffered)
+  float l_x[128];         // warpgroup 1's row sums at a segment's end
 };
 static_assert(8 * B_COUNT + 64 + sizeof(Shared) <= kBarRegion, "barrier region too small");
 
@@ -144,6 +184,19 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Shared* 
                                          bool drain = false) {
   if (__all_sync(0xffffffffu, ptx::mbar_try_wait(bar, parity))) return true;
   return wait_bar_slow(bar, parity, sh, status, drain);
+}
+
+// Multiplies `ncols` (a multiple of 16) fp32 TMEM columns of this warp's lanes by `alpha` (warp-collective).
+__device__ __forceinline__ void rescale_tmem(uint32_t taddr, int ncols, float alpha) {
+  for (int c16 = 0; c16 < ncols; c16 += 16) {
+    float t16[16];
+    ptx::tmem_ld16(taddr + c16, t16);
+    ptx::tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 16; ++e) t16[e] *= alpha;
+    ptx::tmem_st16(taddr + c16, t16);
+  }
+  ptx::tmem_wait_st();
 }
 
 __device__ __forceinline__ int pad16(int r) { return (r + 15) & ~15; }
@@ -216,21 +269,21 @@ struct Producer {
     return true;
   }
 
-  // `rows` (multiple of 16, <= 128) rows × `ncb` 64-column blocks of a 2D map at (x0, y0) → one item,
-  // laid out [cb][rows][128 B].
-  __device__ bool item(const CUtensorMap* m, int x0, int64_t y0, int rows, int ncb) {
+  // `rows` (multiple of 16, <= 128) rows × `ncb` 64-column blocks at row y0 → one item, laid out
+  // [cb][rows][128 B].  A power-of-two height over two column blocks is one 3D load; other heights are
+  // 2D loads of 128/64/32/16 rows per column block.
+  __device__ bool item(const RowMaps& m, int64_t y0, int rows, int ncb) {
     const uint32_t bytes = (uint32_t)rows * 128u * ncb;
     const uint32_t i = ring.n;
+    const uint32_t head = ring.head;  // end of the newest item in flight
     const uint32_t pos = ring.place(bytes);
-    // free the space: retire the oldest items while any item in flight overlaps it (after a wrap a newer
-    // item can overlap while the oldest does not), and keep at most kItemSlots in flight
+    // Free the space: the items in flight occupy the cyclic byte range [start of the oldest, head) (with any
+    // gap skipped at a wrap counted as occupied); retire the oldest until [pos, pos + bytes) lies outside it
+    // and fewer than kItemSlots items are in flight.
     while (oldest < i) {
-      bool busy = i - oldest >= (uint32_t)kItemSlots;
-      for (uint32_t j = oldest; j < i && !busy; ++j) {
-        const uint32_t k = j % kItemSlots;
-        busy = pos < pos_log[k] + len_log[k] && pos_log[k] < pos + bytes;
-      }
-      if (!busy) break;
+      const uint32_t tail = pos_log[oldest % kItemSlots];
+      const bool room = tail < head ? (pos + bytes <= tail || pos >= head) : (pos + bytes <= tail && pos >= head);
+      if (room && i - oldest < (uint32_t)kItemSlots) break;
       if (!retire_oldest()) return false;
     }
     pos_log[i % kItemSlots] = pos;
@@ -239,9 +292,20 @@ struct Producer {
     const uint32_t fb = bar(B_FULL + i % kItemSlots);
     if ((threadIdx.x & 31) == 0) {
       ptx::mbar_arrive_expect_tx(fb, bytes);
-      for (int cb = 0; cb < ncb; ++cb)
-        for (int k = 0; k < rows; k += 16)
-          ptx::tma_load_2d(dst + cb * rows * 128 + k * 128, m, fb, x0 + 64 * cb, (int)(y0 + k));
+      const int k16 = rows >> 4;
+      if (ncb == 2 && (k16 & (k16 - 1)) == 0) {
+        const int hi = k16 == 1 ? 0 : k16 == 2 ? 1 : k16 == 4 ? 2 : 3;
+        ptx::tma_load_3d(dst, map_of(m, true, hi), fb, 0, (int)y0, 0);
+      } else {
+        int r0 = 0;
+        for (int hi = 3; hi >= 0; --hi) {
+          const int h = 16 << hi;
+          if (rows - r0 < h) continue;
+          for (int cb = 0; cb < ncb; ++cb)
+            ptx::tma_load_2d(dst + cb * rows * 128 + r0 * 128, map_of(m, false, hi), fb, 64 * cb, (int)(y0 + r0));
+          r0 += h;
+        }
+      }
     }
     __syncwarp();
     return true;
@@ -280,9 +344,7 @@ __device__ __forceinline__ void st_tile8(uint32_t tile, int row, int col, uint32
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    decode_tc_kernel(const __grid_constant__ CUtensorMap map_tok, const __grid_constant__ CUtensorMap map_dim,
-                     const __grid_constant__ CUtensorMap map_qpre, const __grid_constant__ CUtensorMap map_qsuf,
-                     const __grid_constant__ CUtensorMap map_ksuf, const __grid_constant__ CUtensorMap map_vsuf,
+    decode_tc_kernel(const __grid_constant__ Maps maps,
                      const Params p) {
   constexpr int NCB = D / 64;
   extern __shared__ uint8_t smem_raw[];
@@ -301,22 +363,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::mbar_init(bar(B_QFULL), 1);
     ptx::mbar_init(bar(B_QEMPTY), 1);
-    ptx::mbar_init(bar(B_SFULL), 1);
-    ptx::mbar_init(bar(B_SFULL + 1), 1);
-    ptx::mbar_init(bar(B_PEMPTY), 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(bar(B_SFULL + i), 1);
+      ptx::mbar_init(bar(B_SFREE + i), 1);
+    }
     ptx::mbar_init(bar(B_ATFULL), 1);
-    ptx::mbar_init(bar(B_ACCFULL), 1);
+    ptx::mbar_init(bar(B_ACCDONE), 1);
     ptx::mbar_init(bar(B_FINAL), 1);
     sh->abort_flag = 0;
     ptx::fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    ptx::tma_prefetch_desc(&map_tok);
-    ptx::tma_prefetch_desc(&map_dim);
-    ptx::tma_prefetch_desc(&map_qpre);
-    ptx::tma_prefetch_desc(&map_qsuf);
-    ptx::tma_prefetch_desc(&map_ksuf);
-    ptx::tma_prefetch_desc(&map_vsuf);
+    ptx::tma_prefetch_desc(&maps.qpre);
+    ptx::tma_prefetch_desc(&maps.qsuf);
   }
   if (warp == 1) {
     ptx::tmem_alloc(ptx::smem_u32(&sh->tmem_base), 512);
@@ -355,6 +414,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
 
+  if (warp < kSoftWarp0) {
+  // the register decrease dominates the producer's and the MMA issuer's code
+  if (kRegSplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
   if (warp == 0) {
     // ==================================================================== TMA producer
     // Loads items in exactly the order the issuing warp consumes them (see the softmax section).
@@ -372,13 +434,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // token-factor slab of chunk cc (index inside the block) of a block: rows [row0·cpb + cc·r, +r)
     auto tok_item = [&](int64_t row0, int r, int cc) {
-      return pr.item(&map_tok, 0, row0 * p.cpb + (int64_t)cc * r, pad16(r), 2);
+      return pr.item(maps.tok, row0 * p.cpb + (int64_t)cc * r, pad16(r), 2);
     };
-    auto dim_item = [&](int64_t row0, int r) { return pr.item(&map_dim, 0, row0, pad16(r), NCB); };
+    auto dim_item = [&](int64_t row0, int r) { return pr.item(maps.dim, row0, pad16(r), NCB); };
     for (int si = s_begin; si < s_end && ok; ++si) {
       const Seg sg = get_seg(p, sh, s_begin, si);
       if (sg.type == 0) {
-        ok = pr.q_tile(&map_qpre, sg.h * p.G, sg.tile * p.ipt, p.G * p.ipt);
+        ok = pr.q_tile(&maps.qpre, sg.h * p.G, sg.tile * p.ipt, p.G * p.ipt);
         BlockWalk w{sg.c0, sg.c1, p.cpb};
         BlockInfo bi, bn, prev;
         bool have_prev = false;
@@ -407,17 +469,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok) ok = dim_item(bi.rowv, bi.rv);  // Q_V of the last block
       } else {
-        ok = pr.q_tile(&map_qsuf, sg.h * p.G, sg.tile, p.G);
+        ok = pr.q_tile(&maps.qsuf, sg.h * p.G, sg.tile, p.G);
         const int64_t row0 = ((int64_t)sg.tile * p.H + sg.h) * p.S;
         const int n = sg.c1 - sg.c0;
-        auto kv = [&](const CUtensorMap* m, int j) {
-          return pr.item(m, 0, row0 + (int64_t)(sg.c0 + j) * kChunk, kChunk, NCB);
+        auto kv = [&](const RowMaps& m, int j) {
+          return pr.item(m, row0 + (int64_t)(sg.c0 + j) * kChunk, kChunk, NCB);
         };
-        if (ok) ok = kv(&map_ksuf, 0);
-        if (ok && n >= 2) ok = kv(&map_ksuf, 1);
+        if (ok) ok = kv(maps.ksuf, 0);
+        if (ok && n >= 2) ok = kv(maps.ksuf, 1);
         for (int j = 0; j < n && ok; ++j) {
-          ok = kv(&map_vsuf, j);
-          if (ok && j + 2 < n) ok = kv(&map_ksuf, j + 2);
+          ok = kv(maps.vsuf, j);
+          if (ok && j + 2 < n) ok = kv(maps.ksuf, j + 2);
         }
       }
     }
@@ -427,19 +489,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (pr.q_uses) wait_bar(bar(B_QFULL), (pr.q_uses - 1) & 1, sh, p.status, true);
   } else if (warp == 1) {
     // ==================================================================== MMA issuer (warp 1)
-    // Issues the tensor-core MMAs when the softmax warps signal (named barriers: q̃ ready, P ready, ã ready)
-    // that the smem operands they produce are complete, so issuing overlaps the next softmax step.
+    // Issues the tensor-core MMAs when the softmax warps signal (named barriers) that what they produce is
+    // complete: q̃ in smem, P in an S slot of TMEM, or ã packed in TMEM.  The probabilities and ã are the A
+    // operands of G3 / G4 straight from TMEM.
     const bool leader = lane == 0;
     bool ok = true;
     auto sync_wg = [&](int id) {  // wait for the softmax warps' signal `id`
-      asm volatile("bar.sync %0, 160;" ::"r"(id) : "memory");
+      asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kSigThreads) : "memory");
       ptx::tc_fence_after();
     };
-    // ---------------- MMA issue (warp 1 only)
-    RingPlace ring;          // consumer view of the TMA ring
-    uint32_t cur = 0;        // item being consumed
-    uint32_t sidx_i = 0;     // S-slot uses issued
+    RingPlace ring;                      // consumer view of the TMA ring
+    uint32_t cur = 0;                    // item being consumed
+    uint32_t use_i = 0, use_c = 0;       // S-slot uses issued / consumed (signalled)
     uint32_t q_uses = 0;
+    uint32_t sfree_odd = 0;              // bit s: B_SFREE[s] committed an odd number of times
     auto take = [&](int rows, int ncb, uint32_t& addr) -> bool {
       cur = ring.n;
       const uint32_t pos = ring.place((uint32_t)rows * 128u * ncb);
@@ -451,23 +514,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto release = [&]() {  // the item's space is free once the MMAs issued so far have read it
       if (leader) ptx::umma_commit(bar(B_EMPTY + cur % kItemSlots));
     };
+    auto commit = [&](int b) {
+      if (leader) ptx::umma_commit(bar(b));
+    };
+    // An MMA that overwrites a TMEM region which an earlier MMA of this thread reads as its A operand (p in
+    // an S slot, ã) needs no wait: the tensor pipe executes one thread's MMAs in issue order, and each reads
+    // its operands before any later one writes its accumulator.
+    auto slot_free = [&](uint32_t) -> bool { return true; };
+    auto s_commit = [&]() {
+      commit(B_SFULL + (use_i & 1));
+      ++use_i;
+    };
+    auto p_commit = [&](uint32_t s) {  // P in slot s has been read once the MMAs issued so far complete
+      commit(B_SFREE + s);
+      sfree_odd ^= 1u << s;
+    };
     constexpr uint32_t idS = ptx::idesc_bf16(128, 128, false, true);
     constexpr uint32_t idD = ptx::idesc_bf16(128, D, false, true);
-    auto s_commit = [&]() {
-      if (leader) ptx::umma_commit(bar(B_SFULL + (sidx_i & 1)));
-      ++sidx_i;
-    };
     // G1: q̃ = Q · B_b into the next S slot, N = padded rank
     auto g1 = [&](int rk) -> bool {
       const int rp = pad16(rk);
       uint32_t it;
-      if (!take(rp, NCB, it)) return false;
+      if (!slot_free(use_i & 1) || !take(rp, NCB, it)) return false;
       if (leader) {
-        const uint64_t db = kdesc(it, 0, 0);
+        const uint64_t da = kdesc(base + kOffQ, 0, kTileCb), db = kdesc(it, 0, 0);
         const uint32_t cbs = (uint32_t)rp * 128u, id = ptx::idesc_bf16(128, rp, false, false);
-        const uint32_t d = tmem + kTmS0 + 128 * (sidx_i & 1);
+        const uint32_t d = tmem + kTmS0 + 128 * (use_i & 1);
 #pragma unroll 1
-        for (int k = 0; k < D / 16; ++k) ptx::umma_bf16(d, kdesc(base + kOffQ, 0, kTileCb) + kstep(k, kTileCb), db + kstep(k, cbs), id, k > 0);
+        for (int k = 0; k < D / 16; ++k) ptx::umma_bf16(d, da + kstep(k, kTileCb), db + kstep(k, cbs), id, k > 0);
       }
       release();
       s_commit();
@@ -477,36 +551,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto g2 = [&](int rk) -> bool {
       const int rp = pad16(rk);
       uint32_t it;
-      if (!take(rp, 2, it)) return false;
+      if (!slot_free(use_i & 1) || !take(rp, 2, it)) return false;
       if (leader) {
-        const uint32_t d = tmem + kTmS0 + 128 * (sidx_i & 1);
+        const uint32_t d = tmem + kTmS0 + 128 * (use_i & 1);
         const uint64_t db = mndesc(it, 0, (uint32_t)rp * 128u);
+        const uint64_t dh = kdesc(base + kOffQtHi, 0, kTileCb), dl = kdesc(base + kOffQtLo, 0, kTileCb);
         for (int t = 0; t < rp / 16; ++t) {
           const uint64_t bd = db + (uint64_t)(t * 128);
-          ptx::umma_bf16(d, kdesc(base + kOffQtHi, 0, kTileCb) + kstep(t, kTileCb), bd, idS, t > 0);
-          ptx::umma_bf16(d, kdesc(base + kOffQtLo, 0, kTileCb) + kstep(t, kTileCb), bd, idS, 1);
+          ptx::umma_bf16(d, dh + kstep(t, kTileCb), bd, idS, t > 0);
+          ptx::umma_bf16(d, dl + kstep(t, kTileCb), bd, idS, 1);
         }
       }
       release();
       s_commit();
       return true;
     };
-    // G3: ã (+)= p · P_b, N = padded rank; `fresh` overwrites ã
-    auto g3 = [&](int rv, bool fresh) -> bool {
+    // G3: ã (+)= p · P_b, p packed in S slot s, N = padded rank; `fresh` overwrites ã
+    auto g3 = [&](int rv, bool fresh, uint32_t s) -> bool {
       const int rp = pad16(rv);
       uint32_t it;
       if (!take(rp, 2, it)) return false;
       if (leader) {
         const uint64_t db = kdesc(it, 0, 0);
         const uint32_t cbs = (uint32_t)rp * 128u, id = ptx::idesc_bf16(128, rp, false, false);
-#pragma unroll 1
+        const uint32_t a = tmem + kTmS0 + 128 * s;
+#pragma unroll
         for (int t = 0; t < kChunk / 16; ++t)
-          ptx::umma_bf16(tmem + kTmA, kdesc(base + kOffP, 0, kTileCb) + kstep(t, kTileCb), db + kstep(t, cbs), id, (t > 0 || !fresh) ? 1u : 0u);
+          ptx::umma_bf16_ta(tmem + kTmA, a + ta_col(t), db + kstep(t, cbs), id, (t > 0 || !fresh) ? 1u : 0u);
       }
       release();
+      p_commit(s);
       return true;
     };
-    // G4: acc (+)= ã · Q_bᵀ, ã in the P buffer, B MN-major, N = d
+    // G4: acc (+)= ã · Q_bᵀ, ã packed in TMEM, B MN-major, N = d
     auto g4 = [&](int rv, bool fresh) -> bool {
       const int rp = pad16(rv);
       uint32_t it;
@@ -514,48 +591,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (leader) {
         const uint64_t db = mndesc(it, 0, (uint32_t)rp * 128u);
         for (int t = 0; t < rp / 16; ++t)
-          ptx::umma_bf16(tmem + kTmAcc, kdesc(base + kOffP, 0, kTileCb) + kstep(t, kTileCb), db + (uint64_t)(t * 128), idD,
-                         (t > 0 || !fresh) ? 1u : 0u);
+          ptx::umma_bf16_ta(tmem + kTmAcc, tmem + kTmA + ta_col(t), db + (uint64_t)(t * 128), idD,
+                            (t > 0 || !fresh) ? 1u : 0u);
       }
       release();
+      commit(B_ACCDONE);
       return true;
     };
     // G2' (suffix): S = q · K_sufᵀ, B K-major over d, N = 128 tokens
     auto g2s = [&]() -> bool {
       uint32_t it;
-      if (!take(kChunk, NCB, it)) return false;
+      if (!slot_free(use_i & 1) || !take(kChunk, NCB, it)) return false;
       if (leader) {
-        const uint64_t db = kdesc(it, 0, 0);
-        const uint32_t d = tmem + kTmS0 + 128 * (sidx_i & 1), id = ptx::idesc_bf16(128, kChunk, false, false);
+        const uint64_t da = kdesc(base + kOffQ, 0, kTileCb), db = kdesc(it, 0, 0);
+        const uint32_t d = tmem + kTmS0 + 128 * (use_i & 1), id = ptx::idesc_bf16(128, kChunk, false, false);
 #pragma unroll
-        for (int t = 0; t < D / 16; ++t) ptx::umma_bf16(d, kdesc(base + kOffQ, 0, kTileCb) + kstep(t, kTileCb), db + kstep(t, kChunk * 128u), id, t > 0);
+        for (int t = 0; t < D / 16; ++t)
+          ptx::umma_bf16(d, da + kstep(t, kTileCb), db + kstep(t, kChunk * 128u), id, t > 0);
       }
       release();
       s_commit();
       return true;
     };
-    // G3' (suffix): acc (+)= p · V_suf, B MN-major, K = 128 tokens, N = d
-    auto g3s = [&](bool fresh) -> bool {
+    // G3' (suffix): acc (+)= p · V_suf, p packed in S slot s, B MN-major, K = 128 tokens, N = d
+    auto g3s = [&](bool fresh, uint32_t s) -> bool {
       uint32_t it;
       if (!take(kChunk, NCB, it)) return false;
       if (leader) {
         const uint64_t db = mndesc(it, 0, kChunk * 128u);
+        const uint32_t a = tmem + kTmS0 + 128 * s;
 #pragma unroll
         for (int t = 0; t < kChunk / 16; ++t)
-          ptx::umma_bf16(tmem + kTmAcc, kdesc(base + kOffP, 0, kTileCb) + kstep(t, kTileCb), db + (uint64_t)(t * 128), idD,
-                         (t > 0 || !fresh) ? 1u : 0u);
+          ptx::umma_bf16_ta(tmem + kTmAcc, a + ta_col(t), db + (uint64_t)(t * 128), idD, (t > 0 || !fresh) ? 1u : 0u);
       }
       release();
+      p_commit(s);
       return true;
-    };
-    auto commit = [&](int b) {
-      if (leader) ptx::umma_commit(bar(b));
     };
     auto wait_q = [&]() -> bool {
       const bool r = wait_bar(bar(B_QFULL), q_uses & 1, sh, p.status);
       ++q_uses;
       ptx::tc_fence_after();
       return r;
+    };
+    auto sync_p = [&]() -> uint32_t {  // the softmax warps' P of the next consumed use; returns its slot
+      const uint32_t s = use_c & 1;
+      sync_wg(kSigP0 + (int)s);
+      ++use_c;
+      return s;
     };
     bool bounds_ok = true;
     for (int si = s_begin; si < s_end && bounds_ok; ++si) {
@@ -592,6 +675,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             return true;
           };
           sync_wg(kSigQt);
+          ++use_c;
           if (ok) {
             ok = g2(bi.rk);
             if (ok && n >= 2) ok = g2(bi.rk);
@@ -599,16 +683,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (have_prev) {
             sync_wg(kSigAt);
-            if (ok) {
-              ok = g4(prev.rv, kb == 1);
-              commit(B_PEMPTY);
-            }
+            if (ok) ok = g4(prev.rv, kb == 1);
           }
           for (int j = 0; j < n; ++j) {
-            sync_wg(kSigP);
+            const uint32_t s = sync_p();
             if (ok) {
-              ok = g3(bi.rv, j == 0);
-              commit(j + 1 < n ? B_PEMPTY : B_ATFULL);
+              ok = g3(bi.rv, j == 0, s);
+              if (ok && j + 1 == n) commit(B_ATFULL);
               if (ok && j + 2 < n) ok = g2(bi.rk);
               else if (ok && j + 2 == n && next) ok = g1_next();
             }
@@ -622,11 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!bounds_ok) break;
         sync_wg(kSigAt);
-        if (ok) {
-          ok = g4(bi.rv, kb == 0);
-          commit(B_PEMPTY);
-          commit(B_ACCFULL);
-        }
+        if (ok) ok = g4(bi.rv, kb == 0);
       } else {
         const int n = sg.c1 - sg.c0;
         if (ok) {
@@ -635,230 +712,246 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok && n <= 2) commit(B_QEMPTY);
         }
         for (int j = 0; j < n; ++j) {
-          sync_wg(kSigP);
+          const uint32_t s = sync_p();
           if (ok) {
-            ok = g3s(j == 0);
-            commit(B_PEMPTY);
+            ok = g3s(j == 0, s);
             if (ok && j + 2 < n) {
               ok = g2s();
               if (ok && j + 2 == n - 1) commit(B_QEMPTY);
             }
           }
         }
-        if (ok) commit(B_ACCFULL);
+        if (ok) commit(B_ACCDONE);
       }
     }
     // drain: every MMA issued must complete before TMEM is freed
     commit(B_FINAL);
     __syncwarp();
     wait_bar(bar(B_FINAL), 0, sh, p.status, true);
+  }
   } else {
-    // ==================================================================== softmax warpgroup (warps 2..5)
-    // One thread per row and TMEM lane; signals the MMA warp through named barriers when its smem output
-    // (q̃, P or ã) is complete.
+  if (kRegSplit) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
+  {
+    // ==================================================================== softmax (warps 4..11)
+    // Two warpgroups split every 128-column tile by columns: warpgroup wg takes columns [64wg, 64wg + 64).
+    // Warp w serves TMEM lane quarter w & 3 (one thread per row); the two warps of a quarter exchange their
+    // row maxima through shared memory.  Signals reach the MMA warp through named barriers.
+    const int wg = (warp - kSoftWarp0) >> 2;
     const int quarter = warp & 3;
     const int row = 32 * quarter + lane;
     const uint32_t tl = tmem + ((uint32_t)(32 * quarter) << 16);
-    uint32_t sidx = 0, pk = 0, at_uses = 0, acc_uses = 0;  // consumption counters
+    const int pair_id = kPairBar0 + quarter;
+    uint32_t use = 0;                 // S-slot uses consumed
+    uint32_t sfree_odd = 0;           // bit s: B_SFREE[s] commits (as the MMA warp counts them) are odd
+    uint32_t at_uses = 0, accdone_n = 0, xpar = 0;
     bool ok = true;
     auto signal = [&](int id) {  // arrive on the MMA warp's named barrier `id` (does not wait)
       ptx::tc_fence_before();
-      asm volatile("bar.arrive %0, 160;" ::"r"(id) : "memory");
+      asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(kSigThreads) : "memory");
     };
-    // ---------------- softmax helpers (all four warps)
+    auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(pair_id) : "memory"); };
+    // Every helper below ends with its signal, also after a failed wait, so that all warps always execute
+    // the same sequence of named barriers (which have no time limit).
     // q̃ of a block (fp32, in the next S slot) → bf16 hi + lo in smem, columns >= r zeroed
-    // Every helper below ends with the warpgroup barrier, also after a failed wait, so that the four warps
-    // always execute the same sequence of named barriers (which have no time limit).
     auto convert_qt = [&](bool active, int rk) -> bool {
-      if (!wait_bar(bar(B_SFULL + (sidx & 1)), (sidx >> 1) & 1, sh, p.status)) {
-        ++sidx;
-        signal(kSigQt);
-        return false;
-      }
-      ptx::tc_fence_after();
-      const uint32_t src = tl + kTmS0 + 128 * (sidx & 1);
-      if (active) {
-        for (int c16 = 0; c16 < pad16(rk); c16 += 16) {
-          float v[16];
-          ptx::tmem_ld16(src + c16, v);
-          ptx::tmem_wait_ld();
-          uint32_t hi[8], lo[8];
+      const uint32_t s = use & 1;
+      const bool got = wait_bar(bar(B_SFULL + s), (use >> 1) & 1, sh, p.status);
+      ++use;
+      if (got) {
+        ptx::tc_fence_after();
+        const uint32_t src = tl + kTmS0 + 128 * s;
+        if (active) {
+#pragma unroll 1
+          for (int c16 = 16 * wg; c16 < pad16(rk); c16 += 32) {
+            float v[16];
+            ptx::tmem_ld16(src + c16, v);
+            ptx::tmem_wait_ld();
+            uint32_t hi[8], lo[8];
 #pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            const float a = (c16 + e < rk) ? v[e] : 0.f;
-            const float b2 = (c16 + e + 1 < rk) ? v[e + 1] : 0.f;
-            const uint32_t h2 = ptx::pack_bf16(a, b2);
-            hi[e / 2] = h2;
-            lo[e / 2] = ptx::pack_bf16(a - __uint_as_float(h2 << 16), b2 - __uint_as_float(h2 & 0xFFFF0000u));
+            for (int e = 0; e < 16; e += 2) {
+              const float a = (c16 + e < rk) ? v[e] : 0.f;
+              const float b2 = (c16 + e + 1 < rk) ? v[e + 1] : 0.f;
+              const uint32_t h2 = ptx::pack_bf16(a, b2);
+              hi[e / 2] = h2;
+              lo[e / 2] = ptx::pack_bf16(a - __uint_as_float(h2 << 16), b2 - __uint_as_float(h2 & 0xFFFF0000u));
+            }
+            st_tile8(base + kOffQtHi, row, c16, hi[0], hi[1], hi[2], hi[3]);
+            st_tile8(base + kOffQtHi, row, c16 + 8, hi[4], hi[5], hi[6], hi[7]);
+            st_tile8(base + kOffQtLo, row, c16, lo[0], lo[1], lo[2], lo[3]);
+            st_tile8(base + kOffQtLo, row, c16 + 8, lo[4], lo[5], lo[6], lo[7]);
           }
-          st_tile8(base + kOffQtHi, row, c16, hi[0], hi[1], hi[2], hi[3]);
-          st_tile8(base + kOffQtHi, row, c16 + 8, hi[4], hi[5], hi[6], hi[7]);
-          st_tile8(base + kOffQtLo, row, c16, lo[0], lo[1], lo[2], lo[3]);
-          st_tile8(base + kOffQtLo, row, c16 + 8, lo[4], lo[5], lo[6], lo[7]);
+          ptx::fence_async_smem();
         }
-        ptx::fence_async_smem();
       }
-      ++sidx;
       signal(kSigQt);
-      return true;
+      return got;
     };
-    // ã (fp32, TMEM) → bf16 in the P buffer (its last reader, G3, has completed), columns >= r zeroed
+    // ã (fp32, TMEM) → packed bf16 in place (warpgroup wg: columns [64wg, 64wg + 32)), ranks >= r zeroed
     auto convert_at = [&](bool active, int rv) -> bool {
-      if (!wait_bar(bar(B_ATFULL), at_uses & 1, sh, p.status)) {
-        ++at_uses;
-        signal(kSigAt);
-        return false;
-      }
+      const bool got = wait_bar(bar(B_ATFULL), at_uses & 1, sh, p.status);
       ++at_uses;
-      ptx::tc_fence_after();
-      if (active) {
-        for (int c16 = 0; c16 < pad16(rv); c16 += 16) {
-          float v[16];
-          ptx::tmem_ld16(tl + kTmA + c16, v);
-          ptx::tmem_wait_ld();
-          uint32_t wv[8];
+      ++accdone_n;  // the G4 this signal releases commits B_ACCDONE
+      if (got) {
+        ptx::tc_fence_after();
+        if (active && 64 * wg < pad16(rv)) {
+          // 32 columns at a time: packed half h lands on columns [16h, 16h + 16), which half 0 has read
 #pragma unroll
-          for (int e = 0; e < 16; e += 2)
-            wv[e / 2] = ptx::pack_bf16(c16 + e < rv ? v[e] : 0.f, c16 + e + 1 < rv ? v[e + 1] : 0.f);
-          st_tile8(base + kOffP, row, c16, wv[0], wv[1], wv[2], wv[3]);
-          st_tile8(base + kOffP, row, c16 + 8, wv[4], wv[5], wv[6], wv[7]);
+          for (int h = 0; h < 2; ++h) {
+            float v[32];
+            ptx::tmem_ld32(tl + kTmA + 64 * wg + 32 * h, v);
+            ptx::tmem_wait_ld();
+            uint32_t wv[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int r0 = 64 * wg + 32 * h + 2 * e;
+              wv[e] = ptx::pack_bf16(r0 < rv ? v[2 * e] : 0.f, r0 + 1 < rv ? v[2 * e + 1] : 0.f);
+            }
+            ptx::tmem_st16u(tl + kTmA + 64 * wg + 16 * h, wv);
+          }
+          ptx::tmem_wait_st();
         }
-        ptx::fence_async_smem();
       }
       signal(kSigAt);
-      return true;
+      return got;
     };
-    // one chunk of scores: online softmax, probabilities into the P buffer.  `rescale_at` / `rescale_acc`
-    // say whether ã / acc hold earlier chunks that a grown running max must rescale.
-    auto chunk = [&](bool active, int valid, bool& first_chunk, float& m_used, float& l, bool rescale_at,
-                     int rvp, bool rescale_acc) -> bool {
-      const uint32_t slot = sidx & 1;
-      if (!wait_bar(bar(B_SFULL + slot), (sidx >> 1) & 1, sh, p.status)) {
-        ++sidx;
-        ++pk;
-        signal(kSigP);
-        return false;
-      }
-      ptx::tc_fence_after();
-      ++sidx;
-      const uint32_t src = tl + kTmS0 + 128 * slot;
+    // One chunk of scores: online softmax, probabilities packed into the S slot's TMEM for G3.
+    // prev_chunk: the previous S-slot use was a chunk of this segment (its G3 wrote ã, or acc in a suffix);
+    // at_cols: padded rank of ã (0: no ã); acc_live: acc holds earlier results; acc_by_g4: by a G4.
+    auto chunk = [&](bool active, int valid, bool& first_chunk, float& m_used, float& l, bool prev_chunk,
+                     int at_cols, bool acc_live, bool acc_by_g4) -> bool {
+      const uint32_t s = use & 1, ps = s ^ 1;
+      // the pair barrier below runs whether or not the wait succeeded: it depends only on `active`,
+      // which both warps of a lane quarter share
+      const bool got = wait_bar(bar(B_SFULL + s), (use >> 1) & 1, sh, p.status);
+      if (got) ptx::tc_fence_after();
+      ++use;
+      const uint32_t src = tl + kTmS0 + 128 * s + 64 * wg;
       float alpha = 1.f;
       bool grow = false;
+      // The scores are read from TMEM twice, 32 columns at a time (max pass, then exp pass), so that few
+      // registers stay live across the exchange with the partner warp.
+      float v[32];
       if (active) {
-        // pass 1 over the scores (32 columns at a time, compact loop): the chunk's row max
-        float m8[8];
+        float mx = -INFINITY;
+        if (got) {
+          float m8[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
-#pragma unroll 1
-        for (int c32 = 0; c32 < kChunk; c32 += 32) {
-          float s[32];
-          ptx::tmem_ld32(src + c32, s);
-          ptx::tmem_wait_ld();
+          for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
 #pragma unroll
-          for (int t = 0; t < 32; t += 8)
+          for (int h = 0; h < 2; ++h) {
+            ptx::tmem_ld32(src + 32 * h, v);
+            ptx::tmem_wait_ld();
+            if (valid >= kChunk) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], c32 + t + e < valid ? s[t + e] : -INFINITY);
+              for (int i = 0; i < 32; ++i) m8[i & 7] = fmaxf(m8[i & 7], v[i]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                m8[i & 7] = fmaxf(m8[i & 7], 64 * wg + 32 * h + i < valid ? v[i] : -INFINITY);
+            }
+          }
+          mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          ptx::tmem_ld32(src, v);  // first half of the exp pass, in flight during the exchange
         }
-        float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        mx *= p.c;
+        sh->mx_x[xpar][wg][row] = mx;
+        pair_sync();
+        mx = fmaxf(mx, sh->mx_x[xpar][wg ^ 1][row]) * p.c;
         // keep the running max in use unless the chunk exceeds it by more than 2^8 (then rescale)
-        grow = !first_chunk && mx > m_used + 8.f;
+        grow = got && !first_chunk && mx > m_used + 8.f;
         if (grow) {
           alpha = ptx::ex2(m_used - mx);
           m_used = mx;
           l *= alpha;
         }
-        if (first_chunk) m_used = mx;
+        if (got && first_chunk) m_used = mx;
       }
-      if (pk > 0) {
-        // the previous chunk's G3 (or the previous block's G4, which read ã from the P buffer) has landed
-        if (!wait_bar(bar(B_PEMPTY), (pk - 1) & 1, sh, p.status)) {
-          ++pk;
-          signal(kSigP);
-          return false;
-        }
-        ptx::tc_fence_after();
-      }
+      xpar ^= 1;
+      first_chunk = false;
       if (__any_sync(0xffffffffu, grow)) {
-        // rare: rescale what this warp's rows accumulated so far (alpha = 1 for rows that did not grow)
-        if (rescale_at) {
-          for (int c16 = 0; c16 < rvp; c16 += 16) {
-            float v[16];
-            ptx::tmem_ld16(tl + kTmA + c16, v);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] *= alpha;
-            ptx::tmem_st16(tl + kTmA + c16, v);
-          }
+        // rare: rescale what this warp's rows accumulated so far (alpha = 1 for rows that did not grow),
+        // once the MMAs that wrote it have landed
+        bool w_ok = true;
+        if (prev_chunk) w_ok = wait_bar(bar(B_SFREE + ps), ((sfree_odd >> ps) & 1) ^ 1, sh, p.status);
+        if (w_ok && acc_by_g4) w_ok = wait_bar(bar(B_ACCDONE), (accdone_n - 1) & 1, sh, p.status);
+        ptx::tc_fence_after();
+        if (w_ok) {
+          if (prev_chunk && at_cols > 64 * wg) rescale_tmem(tl + kTmA + 64 * wg, min(at_cols - 64 * wg, 64), alpha);
+          if (acc_live) rescale_tmem(tl + kTmAcc + wg * (D / 2), D / 2, alpha);
+          ptx::tmem_wait_st();
         }
-        if (rescale_acc) {
-          for (int c16 = 0; c16 < D; c16 += 16) {
-            float v[16];
-            ptx::tmem_ld16(tl + kTmAcc + c16, v);
-            ptx::tmem_wait_ld();
+      }
+      if (active && got) {
+        // p = exp2(S·c − m) packed as bf16 over this warpgroup's columns of the slot, row sum in fp32.
+        // Packed half h lands on score columns [16h, 16h + 16) of this warpgroup, which were read before.
+        float ls0 = 0.f, ls1 = 0.f;
+        const float nm = -m_used;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] *= alpha;
-            ptx::tmem_st16(tl + kTmAcc + c16, v);
+        for (int h = 0; h < 2; ++h) {
+          if (h == 1) ptx::tmem_ld32(src + 32, v);
+          ptx::tmem_wait_ld();
+          if (valid < kChunk) {  // a ragged suffix chunk: zero the probabilities of the missing tokens
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 64 * wg + 32 * h + i < valid ? v[i] : -INFINITY;
           }
+          uint32_t pw[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float a = ptx::ex2(fmaf(v[2 * e], p.c, nm));
+            const float b2 = ptx::ex2(fmaf(v[2 * e + 1], p.c, nm));
+            if (e & 1) ls1 += a + b2;
+            else ls0 += a + b2;
+            pw[e] = ptx::pack_bf16(a, b2);
+          }
+          ptx::tmem_st16u(tl + kTmS0 + 128 * s + 64 * wg + 16 * h, pw);
         }
         ptx::tmem_wait_st();
+        l += ls0 + ls1;
       }
-      first_chunk = false;
-      if (active) {
-        // pass 2: p = exp2(S·c − m) as bf16 into the P buffer, row sum in fp32 (32 columns at a time)
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial row sums
-#pragma unroll 1
-        for (int c32 = 0; c32 < kChunk; c32 += 32) {
-          float s[32];
-          ptx::tmem_ld32(src + c32, s);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int g8 = 0; g8 < 4; ++g8) {
-            uint32_t wv[4];
-#pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-              const int t = c32 + 8 * g8 + e;
-              const float a = t < valid ? ptx::ex2(fmaf(s[8 * g8 + e], p.c, -m_used)) : 0.f;
-              const float b2 = t + 1 < valid ? ptx::ex2(fmaf(s[8 * g8 + e + 1], p.c, -m_used)) : 0.f;
-              ls[e / 2] += a + b2;
-              wv[e / 2] = ptx::pack_bf16(a, b2);
-            }
-            st_tile8(base + kOffP, row, c32 + 8 * g8, wv[0], wv[1], wv[2], wv[3]);
-          }
-        }
-        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-        ptx::fence_async_smem();
-      }
-      ++pk;
-      signal(kSigP);
-      return true;
+      sfree_odd ^= 1u << s;
+      signal(kSigP0 + (int)s);
+      return got;
     };
+    // The segment's acc goes to global memory through shared memory (the q̃ region, idle at a segment's
+    // end) and TMA tile stores: each 32-column block is staged as 128 rows × 128 B with the 128-byte
+    // swizzle, which the store undoes and which keeps the staging stores free of bank conflicts.
+    const bool storer = warp == kSoftWarp0 && lane == 0;
+    bool store_pending = false;
+    auto soft_sync = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(kSoftBar), "r"(256) : "memory"); };
     auto write_partial = [&](const Seg& sg, bool active, float m_used, float l) -> bool {
-      if (!wait_bar(bar(B_ACCFULL), acc_uses & 1, sh, p.status)) {
-        ++acc_uses;
-        return false;
-      }
-      ++acc_uses;
-      ptx::tc_fence_after();
+      const bool got = wait_bar(bar(B_ACCDONE), (accdone_n - 1) & 1, sh, p.status);
+      if (got) ptx::tc_fence_after();
       if (active) {
-        float* dst = p.part_acc + ((int64_t)sg.pid * 128 + row) * D;
-        for (int c16 = 0; c16 < D; c16 += 16) {
-          float v[16];
-          ptx::tmem_ld16(tl + kTmAcc + c16, v);
-          ptx::tmem_wait_ld();
-          if (row < sg.rows) {
+        if (got) {
 #pragma unroll
-            for (int e = 0; e < 16; e += 4)
-              *reinterpret_cast<float4*>(dst + c16 + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+          for (int c32 = 0; c32 < D / 2; c32 += 32) {
+            float v[32];
+            ptx::tmem_ld32(tl + kTmAcc + wg * (D / 2) + c32, v);
+            ptx::tmem_wait_ld();
+            const uint32_t blk = base + kOffQtHi + (uint32_t)((wg * (D / 2) + c32) / 32) * 16384u + (uint32_t)row * 128u;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              ptx::st_shared_v4(blk + (uint32_t)((j ^ (row & 7)) << 4), __float_as_uint(v[4 * j]),
+                                __float_as_uint(v[4 * j + 1]), __float_as_uint(v[4 * j + 2]),
+                                __float_as_uint(v[4 * j + 3]));
           }
         }
-        if (row < sg.rows) p.part_ml[(int64_t)sg.pid * 128 + row] = make_float2(m_used, l);
+        if (wg == 1) sh->l_x[row] = l;
+        pair_sync();  // unconditional for active warps (see chunk)
+        if (got && wg == 0 && row < sg.rows)
+          p.part_ml[(int64_t)sg.pid * 128 + row] = make_float2(m_used, l + sh->l_x[row]);
+      }
+      ptx::fence_async_smem();
+      soft_sync();
+      if (storer) {
+        for (int cb = 0; cb < D / 32; ++cb) ptx::tma_store_2d(&maps.pacc, base + kOffQtHi + 16384u * cb, 32 * cb, sg.pid * 128);
+        ptx::bulk_commit();
+        store_pending = true;
       }
       // acc is read before any MMA of the next segment writes it: those follow a later signal
-      return true;
+      return got;
     };
     auto fail_bounds = [&]() {
-      if (warp == 2 && lane == 0) atomicOr(p.status, kStatusDecodeBounds);
+      if (warp == kSoftWarp0 && lane == 0) atomicOr(p.status, kStatusDecodeBounds);
       sh->abort_flag = 1;
       return false;
     };
@@ -866,63 +959,66 @@ __global__ void __launch_bounds__(kThreads, 1)
     // The loops below depend only on the work list, never on `ok`: after a failure (an expired wait, which
     // also raises the CTA's abort flag so that later waits return at once) the warps still walk the same
     // steps and barriers, skipping the work, and then leave together.
+    // One walk serves both segment kinds, so that each helper is expanded once: a prefix segment runs, per
+    // block, q̃ → (the previous block's ã) → its chunks, and finally the last block's ã; a suffix segment
+    // runs its chunks.
     bool bounds_ok = true;
     for (int si = s_begin; si < s_end && bounds_ok; ++si) {
       const Seg sg = get_seg(p, sh, s_begin, si);
+      const bool pre = sg.type == 0;
       const bool active = 32 * quarter < sg.rows;  // a warp whose rows are all padding keeps the protocol only
+      if (si > s_begin) {  // the previous segment's bulk store has read the staging area (the q̃ region)
+        if (storer && store_pending) ptx::bulk_wait_read();
+        store_pending = false;
+        soft_sync();
+      }
       float m_used = -INFINITY, l = 0.f;
       bool first_chunk = true;
-      if (sg.type == 0) {
-        BlockWalk w{sg.c0, sg.c1, p.cpb};
-        BlockInfo bi, bn, prev;
-        int kb = 0;
-        bool have_prev = false;
-        if (!seg_block(p, sh, si - s_begin, kb, sg.h, w.block(), D, bi)) {
-          bounds_ok = fail_bounds();
-          break;
+      BlockWalk w{sg.c0, sg.c1, p.cpb};
+      BlockInfo bi{}, bn{}, prev{};
+      int kb = 0;
+      bool have_prev = false, done = false;
+      if (pre && !seg_block(p, sh, si - s_begin, kb, sg.h, w.block(), D, bi)) {
+        bounds_ok = fail_bounds();
+        break;
+      }
+      while (true) {
+        int n = sg.c1 - sg.c0;
+        bool next = false;
+        if (pre && !done) {
+          n = w.chunks();
+          next = w.has_next();
+          if (next && !seg_block(p, sh, si - s_begin, kb + 1, sg.h, w.block() + 1, D, bn)) {
+            bounds_ok = fail_bounds();
+            break;
+          }
+          ok = convert_qt(active, bi.rk) && ok;  // q̃ of this block to smem
         }
-        while (true) {
-          const int n = w.chunks();
-          const bool next = w.has_next();
-          bool next_is_last = false;
-          if (next) {
-            if (!seg_block(p, sh, si - s_begin, kb + 1, sg.h, w.block() + 1, D, bn)) {
-              bounds_ok = fail_bounds();
-              break;
-            }
-            BlockWalk w2 = w;
-            w2.next();
-            next_is_last = !w2.has_next();
-          }
-          // q̃ of this block to smem, then the first two S-slot uses
-          ok = convert_qt(active, bi.rk) && ok;
-          // the previous block's ã to smem and its expansion G4
-          if (have_prev) {
-            ok = convert_at(active, prev.rv) && ok;
-          }
-          for (int j = 0; j < n; ++j) {
-            ok = chunk(active, kChunk, first_chunk, m_used, l, j > 0, pad16(bi.rv), have_prev) && ok;
-          }
-          if (!next) break;
-          prev = bi;
-          have_prev = true;
+        if (have_prev) ok = convert_at(active, prev.rv) && ok;  // the previous block's ã for its G4
+        if (done) break;
+        for (int j = 0; j < n; ++j) {
+          const int valid = pre ? kChunk : min(kChunk, p.S - (sg.c0 + j) * kChunk);
+          ok = chunk(active, valid, first_chunk, m_used, l, j > 0, pre ? pad16(bi.rv) : 0, pre ? have_prev : j > 0,
+                     pre && have_prev) && ok;
+        }
+        if (!pre) break;
+        prev = bi;
+        have_prev = true;
+        if (next) {
           w.next();
           bi = bn;
           ++kb;
+        } else {
+          done = true;  // one more pass for the last block's ã
         }
-        if (!bounds_ok) break;
-        // the last block's ã and G4, then the segment's result
-        ok = convert_at(active, bi.rv) && ok;
-        ok = write_partial(sg, active, m_used, l) && ok;
-      } else {
-        const int n = sg.c1 - sg.c0;
-        for (int j = 0; j < n; ++j) {
-          const int valid = min(kChunk, p.S - (sg.c0 + j) * kChunk);
-          ok = chunk(active, valid, first_chunk, m_used, l, false, 0, j > 0) && ok;
-        }
-        ok = write_partial(sg, active, m_used, l) && ok;
       }
+      if (!bounds_ok) break;
+      if (!pre) ++accdone_n;  // the MMA warp commits B_ACCDONE after a suffix segment's last G3'
+      ok = write_partial(sg, active, m_used, l) && ok;
     }
+    if (storer && store_pending) ptx::bulk_wait_all();  // the last store has completed before the CTA exits
+  }
+
   }
 
   // ---- teardown: every role has drained its own async work; free TMEM
@@ -1027,6 +1123,64 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, c
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Prepares the decode kernel for head dimension d: its shared-memory size, and a check that the launch
+// allocates the registers that the kernel's register split (setmaxnreg) redistributes.
+cudaError_t prepare_kernel(int d) {
+  const void* kfn = d == 64 ? (const void*)decode_tc_kernel<64> : (const void*)decode_tc_kernel<128>;
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kfn);
+  if (e != cudaSuccess) return e;
+  if (kRegSplit && fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
+  return cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+}
+
+// The 2D and (for 128-column arrays) 3D maps of a [rows][width] bf16 array, boxes of 16/32/64/128 rows.
+bool make_row_maps(RowMaps* rm, const void* ptr, uint64_t width, uint64_t rows) {
+  std::memset(rm, 0, sizeof(RowMaps));
+  for (int hi = 0; hi < 4; ++hi) {
+    const uint32_t h = 16u << hi;
+    const uint64_t d2[2] = {width, rows}, s2[1] = {width * 2};
+    const uint32_t b2[2] = {64, h};
+    if (!make_map(&rm->m2[hi], ptr, 2, d2, s2, b2)) return false;
+    if (width == 128) {
+      const uint64_t d3[3] = {64, rows, 2}, s3[2] = {width * 2, 128};
+      const uint32_t b3[3] = {64, h, 2};
+      if (!make_map(&rm->m3[hi], ptr, 3, d3, s3, b3)) return false;
+    }
+  }
+  return true;
+}
+
+// Map of the partial accumulators: [rows][d] fp32, 128-row × 32-column boxes, 128-byte swizzle.
+bool make_pacc_map(CUtensorMap* m, float* part_acc, int64_t nseg, int d) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[2] = {(cuuint64_t)d, (cuuint64_t)std::max<int64_t>(1, nseg) * 128}, gs[1] = {(cuuint64_t)d * 4};
+  cuuint32_t bx[2] = {32, 128}, es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, part_acc, gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// Maps of one call's query and suffix arrays.
+bool make_call_maps(Maps* M, const DecodeShape& s, const TcInputs& in, int ipt) {
+  const int D = s.d, G = s.Hq / s.H;
+  const uint64_t dims[3] = {(uint64_t)D, (uint64_t)s.Hq, (uint64_t)s.Bq};
+  const uint64_t strd[2] = {(uint64_t)D * 2, (uint64_t)s.Hq * D * 2};
+  const uint32_t box_pre[3] = {64, (uint32_t)G, (uint32_t)ipt};
+  const uint32_t box_suf[3] = {64, (uint32_t)G, 1};
+  if (!make_map(&M->qpre, in.q, 3, dims, strd, box_pre)) return false;
+  if (!make_map(&M->qsuf, in.q, 3, dims, strd, box_suf)) return false;
+  if (s.S > 0) {
+    const uint64_t rows = (uint64_t)s.Bq * s.H * s.S;
+    if (!make_row_maps(&M->ksuf, in.K_suf, D, rows) || !make_row_maps(&M->vsuf, in.V_suf, D, rows)) return false;
+  } else {
+    M->ksuf = M->tok;  // never read
+    M->vsuf = M->tok;
+  }
+  return true;
+}
+
 }  // namespace
 
 struct TcPlan {
@@ -1038,7 +1192,8 @@ struct TcPlan {
   float2* part_ml = nullptr;
   const void* tok = nullptr;
   const void* dim = nullptr;
-  CUtensorMap map_tok, map_dim;
+  RowMaps map_tok, map_dim;
+  CUtensorMap map_pacc;
 };
 
 bool tc_supported(const DecodeShape& s) {
@@ -1057,8 +1212,18 @@ void tc_plan_destroy(TcPlan* plan) {
   delete plan;
 }
 
-// fixed per-chunk, per-block and per-suffix-unit times used to balance the work list (measured orders)
-constexpr double kChunkNs = 700.0, kBlockNs = 1500.0, kUnitNs = 1500.0;
+// Estimated time of one work atom, used to balance the work list across CTAs.  The weights come from a
+// least-squares fit of per-CTA run times on B200 against their work: a 128-token chunk costs about the
+// same whatever its ranks (softmax and MMA issue dominate its bytes), the first chunk of a block adds the
+// q̃ and ã round trips (G1, conversions, G4), the first chunk of a suffix unit adds a segment's partial.
+constexpr double kChunkNs = 1100.0, kBlockNs = 5400.0, kUnitNs = 1700.0, kBytesPerNs = 150.0;
+inline double prefix_atom_ns(int rk, int rv, int cc, int d) {
+  const double bytes = 2.0 * (rk + rv) * kChunk + (cc == 0 ? 2.0 * (rk + rv) * d : 0.0);
+  return bytes / kBytesPerNs + kChunkNs + (cc == 0 ? kBlockNs : 0.0);
+}
+inline double suffix_atom_ns(int c, int d) {
+  return 2.0 * 2.0 * kChunk * d / kBytesPerNs + kChunkNs + (c == 0 ? kUnitNs : 0.0);
+}
 
 static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& in) {
   const int H = s.H, nb = s.nb, D = s.d, G = s.Hq / s.H, Bq = s.Bq, S = s.S;
@@ -1079,17 +1244,12 @@ static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& 
     for (int rt = 0; rt < nrt; ++rt)
       for (int b = 0; b < nb; ++b) {
         const int rk = in.host_ranks[(size_t)(2 * h) * nb + b], rv = in.host_ranks[(size_t)(2 * h + 1) * nb + b];
-        // cost in nanoseconds: bytes at ~44 GB/s per SM, plus the fixed time of a chunk (softmax of
-        // 128 × 128 scores) and of a block (q̃ and ã round trips through TMEM and smem)
-        for (int cc = 0; cc < cpb; ++cc)
-          atoms.push_back({0, h, rt, b * cpb + cc,
-                           (2.0 * (rk + rv) * kChunk + (cc == 0 ? 2.0 * (rk + rv) * D : 0.0)) / 44.0 + kChunkNs +
-                               (cc == 0 ? kBlockNs : 0.0)});
+        for (int cc = 0; cc < cpb; ++cc) atoms.push_back({0, h, rt, b * cpb + cc, prefix_atom_ns(rk, rv, cc, D)});
       }
   for (int i = 0; i < Bq; ++i)
     for (int h = 0; h < H; ++h)
       for (int c = 0; c < nsc; ++c)
-        atoms.push_back({1, h, i, c, 2.0 * 2.0 * kChunk * D / 44.0 + kChunkNs + (c == 0 ? kUnitNs : 0.0)});
+        atoms.push_back({1, h, i, c, suffix_atom_ns(c, D)});
   double total = 0;
   for (auto& a : atoms) total += a.cost;
   const int grid = std::max(1, std::min(sms, (int)atoms.size()));
@@ -1166,23 +1326,15 @@ static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& 
   pl->nsegs = (int)segs.size();
   pl->ipt = ipt;
   pl->nrt = nrt;
-  // factor maps
+  // factor maps: the token factor as a [rows · n/128][128] array of 128-token slab rows, the dim factor
+  // as [rows][d]
   const uint64_t rows = (uint64_t)2 * H * in.pool_rows;
-  {
-    // the token factor as a [rows · n/128][128] array of 128-token slab rows
-    const uint64_t dims[2] = {(uint64_t)kChunk, rows * cpb}, st[1] = {(uint64_t)kChunk * 2};
-    const uint32_t box[2] = {64, 16};
-    if (!make_map(&pl->map_tok, in.tok, 2, dims, st, box)) return cudaErrorInvalidValue;
-  }
-  {
-    const uint64_t dims[2] = {(uint64_t)D, rows}, st[1] = {(uint64_t)D * 2};
-    const uint32_t box[2] = {64, 16};
-    if (!make_map(&pl->map_dim, in.dim, 2, dims, st, box)) return cudaErrorInvalidValue;
-  }
+  if (!make_row_maps(&pl->map_tok, in.tok, kChunk, rows * cpb)) return cudaErrorInvalidValue;
+  if (!make_row_maps(&pl->map_dim, in.dim, D, rows)) return cudaErrorInvalidValue;
+  if (!make_pacc_map(&pl->map_pacc, pl->part_acc, pl->nsegs, D)) return cudaErrorInvalidValue;
   pl->tok = in.tok;
   pl->dim = in.dim;
-  auto kfn = D == 64 ? (const void*)decode_tc_kernel<64> : (const void*)decode_tc_kernel<128>;
-  return cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  return prepare_kernel(D);
 }
 
 cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, void* out, cudaStream_t st,
@@ -1200,24 +1352,11 @@ cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, v
     *plan = pl;
   }
   const int D = s.d, G = s.Hq / s.H;
-  CUtensorMap mq_pre, mq_suf, mk, mv;
-  {
-    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)s.Hq, (uint64_t)s.Bq};
-    const uint64_t strd[2] = {(uint64_t)D * 2, (uint64_t)s.Hq * D * 2};
-    const uint32_t box_pre[3] = {64, (uint32_t)G, (uint32_t)pl->ipt};
-    const uint32_t box_suf[3] = {64, (uint32_t)G, 1};
-    if (!make_map(&mq_pre, in.q, 3, dims, strd, box_pre)) return cudaErrorInvalidValue;
-    if (!make_map(&mq_suf, in.q, 3, dims, strd, box_suf)) return cudaErrorInvalidValue;
-  }
-  if (s.S > 0) {
-    const uint64_t dims[2] = {(uint64_t)D, (uint64_t)s.Bq * s.H * s.S}, strd[1] = {(uint64_t)D * 2};
-    const uint32_t box[2] = {64, 16};
-    if (!make_map(&mk, in.K_suf, 2, dims, strd, box)) return cudaErrorInvalidValue;
-    if (!make_map(&mv, in.V_suf, 2, dims, strd, box)) return cudaErrorInvalidValue;
-  } else {
-    mk = pl->map_dim;
-    mv = pl->map_dim;
-  }
+  Maps maps;
+  maps.tok = pl->map_tok;
+  maps.dim = pl->map_dim;
+  maps.pacc = pl->map_pacc;
+  if (!make_call_maps(&maps, s, in, pl->ipt)) return cudaErrorInvalidValue;
   Params p;
   p.seg_first = pl->d_work;
   p.segs = reinterpret_cast<const Seg*>(pl->d_work + pl->off_segs);
@@ -1236,10 +1375,9 @@ cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, v
   cudaError_t e;
   if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
   if (D == 64)
-    decode_tc_kernel<64><<<pl->grid, kThreads, kSmemBytes, st>>>(pl->map_tok, pl->map_dim, mq_pre, mq_suf, mk, mv, p);
+    decode_tc_kernel<64><<<pl->grid, kThreads, kSmemBytes, st>>>(maps, p);
   else
-    decode_tc_kernel<128><<<pl->grid, kThreads, kSmemBytes, st>>>(pl->map_tok, pl->map_dim, mq_pre, mq_suf, mk, mv,
-                                                                   p);
+    decode_tc_kernel<128><<<pl->grid, kThreads, kSmemBytes, st>>>(maps, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (ev1 && (e = cudaEventRecord(ev1, st)) != cudaSuccess) return e;
@@ -1269,6 +1407,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 std::mutex g_noalloc_mu;
 void* g_noalloc_dev_ptr[kNoAllocMaxDevices];  // device address of g_noalloc_scratch, per device
+bool g_noalloc_ready[kNoAllocMaxDevices][2];  // decode kernel prepared on the device, per head dim (64, 128)
 int g_noalloc_host_words[kNoAllocMaxWords];   // work list staging, guarded by g_noalloc_mu
 
 // Byte-balanced work list as in build_plan, written into `w` without heap allocation.
@@ -1286,15 +1425,12 @@ int build_worklist_fixed(const DecodeShape& s, const int32_t* host_ranks, int gr
       for (int rt = 0; rt < nrt; ++rt)
         for (int b = 0; b < nb; ++b) {
           const int rk = host_ranks[(size_t)(2 * h) * nb + b], rv = host_ranks[(size_t)(2 * h + 1) * nb + b];
-          for (int cc = 0; cc < cpb; ++cc)
-            fn(0, h, rt, b * cpb + cc,
-               (2.0 * (rk + rv) * kChunk + (cc == 0 ? 2.0 * (rk + rv) * D : 0.0)) / 44.0 + kChunkNs +
-                   (cc == 0 ? kBlockNs : 0.0));
+          for (int cc = 0; cc < cpb; ++cc) fn(0, h, rt, b * cpb + cc, prefix_atom_ns(rk, rv, cc, D));
         }
     for (int i = 0; i < Bq; ++i)
       for (int h = 0; h < H; ++h)
         for (int c = 0; c < nsc; ++c)
-          fn(1, h, i, c, 2.0 * 2.0 * kChunk * D / 44.0 + kChunkNs + (c == 0 ? kUnitNs : 0.0));
+          fn(1, h, i, c, suffix_atom_ns(c, D));
   };
   double total = 0;
   for_each_atom([&](int, int, int, int, double cost) { total += cost; });
@@ -1383,9 +1519,10 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
     void* ptr = nullptr;
     if ((e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch)) != cudaSuccess) return e;
     g_noalloc_dev_ptr[dev] = ptr;
-    auto kfn = s.d == 64 ? (const void*)decode_tc_kernel<64> : (const void*)decode_tc_kernel<128>;
-    if ((e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes)) != cudaSuccess)
-      return e;
+  }
+  if (!g_noalloc_ready[dev][s.d == 64 ? 0 : 1]) {
+    if ((e = prepare_kernel(s.d)) != cudaSuccess) return e;
+    g_noalloc_ready[dev][s.d == 64 ? 0 : 1] = true;
   }
   unsigned char* scratch = static_cast<unsigned char*>(g_noalloc_dev_ptr[dev]);
   int sms = 148;
@@ -1413,35 +1550,12 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
       cudaSuccess)
     return e;
   const int D = s.d, G = s.Hq / s.H;
-  CUtensorMap map_tok, map_dim, mq_pre, mq_suf, mk, mv;
+  Maps maps;
   const uint64_t rows = (uint64_t)2 * s.H * in.pool_rows;
-  {
-    const uint64_t dims[2] = {(uint64_t)kChunk, rows * cpb}, strd[1] = {(uint64_t)kChunk * 2};
-    const uint32_t box[2] = {64, 16};
-    if (!make_map(&map_tok, in.tok, 2, dims, strd, box)) return cudaErrorInvalidValue;
-  }
-  {
-    const uint64_t dims[2] = {(uint64_t)D, rows}, strd[1] = {(uint64_t)D * 2};
-    const uint32_t box[2] = {64, 16};
-    if (!make_map(&map_dim, in.dim, 2, dims, strd, box)) return cudaErrorInvalidValue;
-  }
-  {
-    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)s.Hq, (uint64_t)s.Bq};
-    const uint64_t strd[2] = {(uint64_t)D * 2, (uint64_t)s.Hq * D * 2};
-    const uint32_t box_pre[3] = {64, (uint32_t)G, (uint32_t)ipt};
-    const uint32_t box_suf[3] = {64, (uint32_t)G, 1};
-    if (!make_map(&mq_pre, in.q, 3, dims, strd, box_pre)) return cudaErrorInvalidValue;
-    if (!make_map(&mq_suf, in.q, 3, dims, strd, box_suf)) return cudaErrorInvalidValue;
-  }
-  if (s.S > 0) {
-    const uint64_t dims[2] = {(uint64_t)D, (uint64_t)s.Bq * s.H * s.S}, strd[1] = {(uint64_t)D * 2};
-    const uint32_t box[2] = {64, 16};
-    if (!make_map(&mk, in.K_suf, 2, dims, strd, box)) return cudaErrorInvalidValue;
-    if (!make_map(&mv, in.V_suf, 2, dims, strd, box)) return cudaErrorInvalidValue;
-  } else {
-    mk = map_dim;
-    mv = map_dim;
-  }
+  if (!make_row_maps(&maps.tok, in.tok, kChunk, rows * cpb)) return cudaErrorInvalidValue;
+  if (!make_row_maps(&maps.dim, in.dim, D, rows)) return cudaErrorInvalidValue;
+  if (!make_pacc_map(&maps.pacc, part_acc, nsegs, D)) return cudaErrorInvalidValue;
+  if (!make_call_maps(&maps, s, in, ipt)) return cudaErrorInvalidValue;
   Params p;
   p.seg_first = d_work;
   p.segs = reinterpret_cast<const Seg*>(d_work + off_segs);
@@ -1458,9 +1572,9 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
   p.S = s.S;
   p.c = s.scale * 1.4426950408889634f;
   if (D == 64)
-    decode_tc_kernel<64><<<grid, kThreads, kSmemBytes, st>>>(map_tok, map_dim, mq_pre, mq_suf, mk, mv, p);
+    decode_tc_kernel<64><<<grid, kThreads, kSmemBytes, st>>>(maps, p);
   else
-    decode_tc_kernel<128><<<grid, kThreads, kSmemBytes, st>>>(map_tok, map_dim, mq_pre, mq_suf, mk, mv, p);
+    decode_tc_kernel<128><<<grid, kThreads, kSmemBytes, st>>>(maps, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (D == 64)
     combine_tc_kernel<64><<<dim3(s.Hq, s.Bq), 64, 0, st>>>(part_acc, part_ml, d_work + off_pre, d_work + off_suf,
