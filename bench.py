@@ -9,6 +9,7 @@ factors produced by milo_compress from a seeded synthetic cache.  Compression
 reported as compressions/s.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl milo|reference] [--workload NAME]
+  python bench.py --profile decode|compress [--calls N]   (a short run for ncu captures)
 
 Prints one JSON line on rank 0.  For N > 1 launch with torch.distributed.run;
 every rank decodes its own batch (independent problems, no collective on the
@@ -32,6 +33,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "compressed-KV decode tokens/s at Qwen2.5-7B shape; achieved HBM GB/s vs peak"
+# DRAM bytes read + written by one decode_tc_kernel launch on qwen2.5-7b-layer, from the ncu capture summarised
+# under profiles/ (decode_tc_kernel_qwen2.5-7b-layer); reset to None whenever the kernel changes.
+DECODE_TRAFFIC = {"qwen2.5-7b-layer": 42362112 + 67584}
 
 
 def _args():
@@ -43,6 +47,9 @@ def _args():
     p.add_argument("--workload", default="qwen2.5-7b-layer")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="bound of the CPU oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--profile", choices=["decode", "compress"], default=None,
+                   help="run only N calls of one phase on the workload (for profiler captures), no JSON contract")
+    p.add_argument("--calls", type=int, default=6)
     return p.parse_args()
 
 
@@ -360,7 +367,7 @@ def run_milo(a):
                        "l2": f"inputs rotated over {copies} copies ({copies * step_bytes / 1e6:.0f} MB > 3x L2)",
                        "launch": "CUDA graph of one pass over the copies"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                         "frac": achieved / peak, "traffic": DECODE_TRAFFIC.get(wl.name), "peak_kind": peak_kind,
                          "bytes_per_step": step_bytes, "kernel": "decode_tc_kernel" if dt == "bf16" else
                          "prefix_kernel", "kernel_ms": kernel_ms, "call_ms": per_call_ms,
                          "note": "achieved = algorithmic bytes per step / mean CUDA-event duration of the main "
@@ -382,8 +389,44 @@ def run_milo(a):
         torch.distributed.destroy_process_group()
 
 
+def run_profile(a):
+    """N eager calls of one phase on one GPU: what an ncu capture of that phase's kernels runs."""
+    import torch
+    torch.cuda.set_device(0)
+    import decode_attention_milo_b200 as milo
+    from synth import WORKLOADS, gen_layer
+    wl = WORKLOADS[a.workload]
+    dt = wl.dtype
+    L = gen_layer(wl)
+    dev = lambda x: _to_dev(x, dt, torch)
+    Kd, Vd = dev(L["K"]), dev(L["V"])
+    beta = wl.budgets[0]
+    t0 = time.time()
+    if a.profile == "compress":
+        for _ in range(a.calls):
+            f = milo.compress(Kd, Vd, wl.block_size, beta, wl.r_min)
+            torch.cuda.synchronize()
+            assert f.status()[0] == 0
+            f.close()
+    else:
+        f = milo.compress(Kd, Vd, wl.block_size, beta, wl.r_min)
+        q = dev(L["q"])
+        ks = dev(L["K_suf"]) if wl.suffix else None
+        vs = dev(L["V_suf"]) if wl.suffix else None
+        out = torch.empty_like(q)
+        for _ in range(a.calls):
+            milo.decode_attn(q, f, ks, vs, out=out)
+        torch.cuda.synchronize()
+        assert f.status()[0] == 0
+        f.close()
+    print(json.dumps({"profile": a.profile, "workload": wl.name, "calls": a.calls, "wall_s": time.time() - t0}))
+
+
 def main():
     a = _args()
+    if a.profile:
+        run_profile(a)
+        return
     if a.impl == "reference":
         run_reference(a)
     else:

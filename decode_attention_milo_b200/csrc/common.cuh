@@ -13,6 +13,7 @@ enum : uint32_t {
   kStatusCompressBounds = 2u,
   kStatusDecodeBounds = 4u,
   kStatusDecodeTimeout = 8u,
+  kStatusCompressTimeout = 16u,
 };
 
 __device__ __forceinline__ float to_f32(float x) { return x; }

@@ -5,7 +5,7 @@
 // block's keys and values separately at low rank; §4.3 sets each block's rank
 // from its entropy under a fixed total budget.  Four kernels per layer, all on
 // the caller's stream:
-//   gram     G_b = X_bᵀ X_b in fp32                       (one CTA per block)
+//   gram     G_b = X_bᵀ X_b in fp32  (bf16 blocks: tensor cores, gram_tc.cu; fp32: here, one CTA per block)
 //   jacobi   one-sided Jacobi on G_b: eigenvalues λ_i = σ_i², eigenvectors B_b,
 //            sorted descending                            (one CTA per block)
 //   alloc    H_b = −Σ p ln p (p = λ/Σλ, fp64), w_b = e^{H_b}, quotas
@@ -368,7 +368,14 @@ cudaError_t run(const CompressShape& s, const CompressBuffers& bf, cudaStream_t 
   const T* K = static_cast<const T*>(bf.K);
   const T* V = static_cast<const T*>(bf.V);
   dim3 grid(s.nb, 2 * s.H);
-  gram_kernel<T, D><<<grid, kThreads, 0, st>>>(K, V, s.T, s.n, s.nb, bf.gram);
+  // bf16 blocks: Gram on the tensor cores (gram_tc.cu); fp32 blocks: on the CUDA cores
+  const cudaError_t ge = launch_gram_tc(s, K, V, bf.gram, bf.status, st);
+  if (ge == cudaErrorNotSupported) {
+    cudaGetLastError();
+    gram_kernel<T, D><<<grid, kThreads, 0, st>>>(K, V, s.T, s.n, s.nb, bf.gram);
+  } else if (ge != cudaSuccess) {
+    return ge;
+  }
   const size_t jsm = (2 * D * D + D) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(jacobi_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)jsm);
   if (e != cudaSuccess) return e;

@@ -35,6 +35,10 @@ struct CompressBuffers {
 };
 
 cudaError_t launch_compress(const CompressShape& s, const CompressBuffers& b, cudaStream_t st);
+// Tensor-core Gram of bf16 blocks (d in {64, 128}, n % 128 == 0); cudaErrorNotSupported otherwise.
+bool gram_tc_supported(const CompressShape& s);
+cudaError_t launch_gram_tc(const CompressShape& s, const void* K, const void* V, float* gram, uint32_t* status,
+                           cudaStream_t st);
 
 // Rank-space decode on CUDA cores (any dtype; the fp32 path and a cross-check for bf16).
 struct DecodeShape {

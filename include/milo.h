@@ -203,7 +203,7 @@ milo_status milo_factors_describe(const milo_factors* f, milo_factors_desc* desc
  * Synchronises the device and returns the first error recorded by a kernel
  * for f (MILO_OK if none).  *host_bits (optional) receives the raw bit mask:
  * 1 = Jacobi did not converge, 2 = compress bounds check, 4 = decode bounds
- * check, 8 = decode wait expired.
+ * check, 8 = decode wait expired, 16 = compress (Gram) wait expired.
  */
 milo_status milo_factors_status(const milo_factors* f, uint32_t* host_bits);
 
