@@ -35,7 +35,7 @@ sys.path.insert(0, ROOT)
 METRIC = "compressed-KV decode tokens/s at Qwen2.5-7B shape; achieved HBM GB/s vs peak"
 # DRAM bytes read + written by one decode_tc_kernel launch on qwen2.5-7b-layer, from the ncu capture summarised
 # under profiles/ (decode_tc_kernel_qwen2.5-7b-layer); reset to None whenever the kernel changes.
-DECODE_TRAFFIC = {"qwen2.5-7b-layer": 42362112 + 67584}
+DECODE_TRAFFIC = {"qwen2.5-7b-layer": 42166528 + 42752}
 
 
 def _args():

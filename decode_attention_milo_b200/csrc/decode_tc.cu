@@ -272,7 +272,7 @@ struct Producer {
   // `rows` (multiple of 16, <= 128) rows × `ncb` 64-column blocks at row y0 → one item, laid out
   // [cb][rows][128 B].  A power-of-two height over two column blocks is one 3D load; other heights are
   // 2D loads of 128/64/32/16 rows per column block.
-  __device__ bool item(const RowMaps& m, int64_t y0, int rows, int ncb) {
+  __device__ __noinline__ bool item(const RowMaps& m, int64_t y0, int rows, int ncb) {
     const uint32_t bytes = (uint32_t)rows * 128u * ncb;
     const uint32_t i = ring.n;
     const uint32_t head = ring.head;  // end of the newest item in flight
@@ -795,7 +795,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tc_fence_after();
         if (active && 64 * wg < pad16(rv)) {
           // 32 columns at a time: packed half h lands on columns [16h, 16h + 16), which half 0 has read
-#pragma unroll
+#pragma unroll 1
           for (int h = 0; h < 2; ++h) {
             float v[32];
             ptx::tmem_ld32(tl + kTmA + 64 * wg + 32 * h, v);
@@ -837,7 +837,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float m8[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
-#pragma unroll
+#pragma unroll 1
           for (int h = 0; h < 2; ++h) {
             ptx::tmem_ld32(src + 32 * h, v);
             ptx::tmem_wait_ld();
@@ -885,7 +885,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Packed half h lands on score columns [16h, 16h + 16) of this warpgroup, which were read before.
         float ls0 = 0.f, ls1 = 0.f;
         const float nm = -m_used;
-#pragma unroll
+#pragma unroll 1
         for (int h = 0; h < 2; ++h) {
           if (h == 1) ptx::tmem_ld32(src + 32, v);
           ptx::tmem_wait_ld();
@@ -922,7 +922,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (got) ptx::tc_fence_after();
       if (active) {
         if (got) {
-#pragma unroll
+#pragma unroll 1
           for (int c32 = 0; c32 < D / 2; c32 += 32) {
             float v[32];
             ptx::tmem_ld32(tl + kTmAcc + wg * (D / 2) + c32, v);
@@ -1216,7 +1216,7 @@ void tc_plan_destroy(TcPlan* plan) {
 // least-squares fit of per-CTA run times on B200 against their work: a 128-token chunk costs about the
 // same whatever its ranks (softmax and MMA issue dominate its bytes), the first chunk of a block adds the
 // q̃ and ã round trips (G1, conversions, G4), the first chunk of a suffix unit adds a segment's partial.
-constexpr double kChunkNs = 1100.0, kBlockNs = 5400.0, kUnitNs = 1700.0, kBytesPerNs = 150.0;
+constexpr double kChunkNs = 1000.0, kBlockNs = 3000.0, kUnitNs = 1700.0, kBytesPerNs = 150.0;
 inline double prefix_atom_ns(int rk, int rv, int cc, int d) {
   const double bytes = 2.0 * (rk + rv) * kChunk + (cc == 0 ? 2.0 * (rk + rv) * d : 0.0);
   return bytes / kBytesPerNs + kChunkNs + (cc == 0 ? kBlockNs : 0.0);
