@@ -134,6 +134,34 @@ def _dist():
     return world, rank, local
 
 
+def _max_over_ranks(x, world):
+    """Max of a float over all ranks (the job's time is its slowest rank's); identity on one rank."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _job_value(world, batch, steps, ms):
+    """Whole-job decode tokens/s: every rank decodes `batch` tokens per step; `ms` is the max over ranks."""
+    return world * batch * steps / (ms / 1e3)
+
+
+def _config(wl, world, ranks_total=None, **extra):
+    """The workload description shared by both arms' JSON lines."""
+    c = {"workload": wl.name, "batch": wl.batch, "kv_heads": wl.kv_heads, "q_heads": wl.q_heads,
+         "head_dim": wl.head_dim, "context": wl.context, "block_size": wl.block_size, "suffix": wl.suffix,
+         "budget": wl.budgets[0], "r_min": wl.r_min, "parallelism": f"replica x{world}"}
+    if ranks_total is not None:
+        c["ranks_total"] = int(ranks_total)
+    c.update(extra)
+    return c
+
+
 def _to_dev(a, dt, torch):
     if dt == "f32":
         return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
@@ -179,13 +207,18 @@ def _cpu_baseline(wl, L, seconds):
 
 
 def run_reference(a):
-    """The oracle timed on the host cores: `steps` bounded decode steps after `warmup`."""
+    """The oracle timed on the host cores: `steps` bounded decode steps after `warmup` (rank 0 only)."""
     world, rank, _ = _dist()
     if rank != 0:
         return
     from synth import WORKLOADS, gen_layer
     import oracle
     from synth import from_storage
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
+    except Exception:  # pragma: no cover
+        pass
     wl = WORKLOADS[a.workload]
     L = gen_layer(wl)
     dt = wl.dtype
@@ -204,14 +237,12 @@ def run_reference(a):
         oracle.decode_attention(q[sl], lay, Ks[sl], Vs[sl])
     el = time.perf_counter() - t0
     value = a.steps * per / el
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference", "n_gpus": a.gpus,
+    sample = f"{per} of {wl.batch} queries per step, fp64 NumPy oracle, 1 BLAS thread"
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference", "n_gpus": world,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * el / a.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "batch_per_step": per, "kv_heads": wl.kv_heads,
-                       "q_heads": wl.q_heads, "head_dim": wl.head_dim, "context": wl.context,
-                       "block_size": wl.block_size, "suffix": wl.suffix, "budget": wl.budgets[0]},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{per} of {wl.batch} queries per step, fp64 NumPy oracle"},
+            "config": _config(wl, world),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -298,13 +329,9 @@ def run_milo(a):
         torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = _max_over_ranks(e0.elapsed_time(e1), world)
     ms_step = ms / steps
-    value = world * wl.batch * steps / (ms / 1e3)
+    value = _job_value(world, wl.batch, steps, ms)
     per_call_ms = ms_step  # every step is one milo_decode_attn call
     kernels_per_call = sets[0].decode_launches(wl.batch, wl.q_heads, S)
 
@@ -342,11 +369,7 @@ def run_milo(a):
         hout.copy_(outs[c].view(hout.dtype), non_blocking=True)
     f1.record(st)
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = _max_over_ranks(f0.elapsed_time(f1), world)
     h2d = hq.numel() * hq.element_size() + (2 * hk.numel() * hk.element_size() if S else 0)
     d2h = hout.numel() * hout.element_size()
 
@@ -360,12 +383,9 @@ def run_milo(a):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
             "warmup": reps_w * copies, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": dt, "data": "synthetic",
-            "config": {"workload": wl.name, "batch": wl.batch, "kv_heads": wl.kv_heads, "q_heads": wl.q_heads,
-                       "head_dim": wl.head_dim, "context": wl.context, "block_size": wl.block_size,
-                       "suffix": wl.suffix, "budget": beta, "r_min": wl.r_min,
-                       "ranks_total": int(ranks.sum()), "parallelism": f"replica x{world}",
-                       "l2": f"inputs rotated over {copies} copies ({copies * step_bytes / 1e6:.0f} MB > 3x L2)",
-                       "launch": "CUDA graph of one pass over the copies"},
+            "config": _config(wl, world, ranks.sum(),
+                              l2=f"inputs rotated over {copies} copies ({copies * step_bytes / 1e6:.0f} MB > 3x L2)",
+                              launch="CUDA graph of one pass over the copies"),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": DECODE_TRAFFIC.get(wl.name), "peak_kind": peak_kind,
                          "bytes_per_step": step_bytes, "kernel": "decode_tc_kernel" if dt == "bf16" else
@@ -373,7 +393,7 @@ def run_milo(a):
                          "note": "achieved = algorithmic bytes per step / mean CUDA-event duration of the main "
                                  "decode kernel (events recorded by the library right before and after it, "
                                  f"{kt_steps} eager launches over the rotated copies)"},
-            "e2e": {"value": world * wl.batch * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+            "e2e": {"value": _job_value(world, wl.batch, e2e_steps, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "compress": {"compressions_per_s": 1e3 / statistics.median(comp), "ms": statistics.median(comp),
                          "unit": "whole-layer compressions/s"},

@@ -68,6 +68,8 @@ def load_library(path: str | None = None):
     L.milo_decode_attn_noalloc.argtypes = [vp, i32, i32, vp, vp, vp, i32, f32, vp, vp]
     L.milo_decode_launches.restype = i32
     L.milo_decode_launches.argtypes = [vp, i32, i32, i32]
+    L.milo_decode_worklist.restype = i32
+    L.milo_decode_worklist.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, i64, vp]
     L.milo_factors_ranks.restype = i32
     L.milo_factors_ranks.argtypes = [vp, vp]
     L.milo_factors_describe.restype = i32
@@ -238,3 +240,23 @@ def import_factors(dtype: int, num_kv_heads: int, context: int, head_dim: int, b
                                               dim.ctypes.data_as(ctypes.c_void_p), _stream_ptr(stream),
                                               ctypes.byref(h)), "milo_factors_import")
     return Factors(h)
+
+
+def decode_worklist(ranks, block_size: int, head_dim: int, batch: int, num_q_heads: int, suffix_len: int,
+                    num_ctas: int) -> dict:
+    """The bf16 decode's work list for host ranks [2H][nb] (milo_decode_worklist; host only, no GPU)."""
+    import numpy as np
+    r = np.ascontiguousarray(ranks, dtype=np.int32)
+    H, nb = r.shape[0] // 2, r.shape[1]
+    cap = 1 << 22
+    out = np.zeros(cap, dtype=np.int32)
+    info = np.zeros(8, dtype=np.int64)
+    _check(load_library().milo_decode_worklist(r.ctypes.data, H, nb, block_size, head_dim, batch, num_q_heads,
+                                               suffix_len, num_ctas, out.ctypes.data, cap, info.ctypes.data),
+           "milo_decode_worklist")
+    nwords, nsegs, grid, off_segs, off_pre, off_suf, ipt, nrt = (int(x) for x in info)
+    return {"seg_first": out[:grid + 1].copy(),
+            "segs": out[off_segs:off_segs + 8 * nsegs].reshape(nsegs, 8).copy(),
+            "pre_range": out[off_pre:off_pre + 2 * H * nrt].reshape(H * nrt, 2).copy(),
+            "suf_range": out[off_suf:off_suf + 2 * batch * H].reshape(batch * H, 2).copy(),
+            "items_per_tile": ipt, "tiles": nrt, "words": nwords}

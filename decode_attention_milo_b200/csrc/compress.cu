@@ -22,6 +22,9 @@ namespace milo {
 namespace {
 
 constexpr int kThreads = 256;
+// Jacobi runs one CTA per block with 128 KB of shared memory (one CTA per SM), so it uses more warps to hide
+// the latency of each round: 16 warps, 4 column pairs per warp per round (d = 128).
+constexpr int kJThreads = 512;
 constexpr float kJacobiTol = 1e-5f;  // relative orthogonality |a_p·a_q| / (|a_p||a_q|)
 
 template <typename T>
@@ -85,7 +88,7 @@ __device__ __forceinline__ void rr_pair(int D, int s, int k, int& p, int& q) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads) jacobi_kernel(const float* __restrict__ gram, int nb, int max_sweeps,
+__global__ void __launch_bounds__(kJThreads) jacobi_kernel(const float* __restrict__ gram, int nb, int max_sweeps,
                                                          float* __restrict__ eigvals, float* __restrict__ eigvecs,
                                                          uint32_t* status) {
   constexpr int E = D / 32;  // elements per lane of one column
@@ -95,13 +98,13 @@ __global__ void __launch_bounds__(kThreads) jacobi_kernel(const float* __restric
   float* lam = W + D * D;   // D
   const int blk = blockIdx.x + blockIdx.y * nb;
   const float* G = gram + (int64_t)blk * D * D;
-  for (int e = threadIdx.x; e < D * D; e += kThreads) {
+  for (int e = threadIdx.x; e < D * D; e += kJThreads) {
     A[e] = G[e];  // G symmetric: row-major == column-major
     W[e] = (e / D == e % D) ? 1.f : 0.f;
   }
   __syncthreads();
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  constexpr int NW = kThreads / 32;
+  constexpr int NW = kJThreads / 32;
   constexpr int PP = (D / 2) / NW;  // column pairs per warp per round
   bool converged = false;
   for (int sweep = 0; sweep < max_sweeps; ++sweep) {
@@ -159,7 +162,7 @@ __global__ void __launch_bounds__(kThreads) jacobi_kernel(const float* __restric
   }
   if (!converged && threadIdx.x == 0) atomicOr(status, kStatusNoConvergence);
   // eigenvalue of column j = |G w_j| = norm of A's column j
-  for (int j = warp; j < D; j += kThreads / 32) {
+  for (int j = warp; j < D; j += kJThreads / 32) {
     float ss = 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -171,7 +174,7 @@ __global__ void __launch_bounds__(kThreads) jacobi_kernel(const float* __restric
   }
   __syncthreads();
   // sort descending by counting (ties: lower column first)
-  for (int j = warp; j < D; j += kThreads / 32) {
+  for (int j = warp; j < D; j += kJThreads / 32) {
     const float lj = lam[j];
     int rank = 0;
     for (int i = lane; i < D; i += 32) rank += (lam[i] > lj) || (lam[i] == lj && i < j);
@@ -379,7 +382,7 @@ cudaError_t run(const CompressShape& s, const CompressBuffers& bf, cudaStream_t 
   const size_t jsm = (2 * D * D + D) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(jacobi_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)jsm);
   if (e != cudaSuccess) return e;
-  jacobi_kernel<D><<<grid, kThreads, jsm, st>>>(bf.gram, s.nb, s.max_sweeps, bf.eigvals, bf.eigvecs, bf.status);
+  jacobi_kernel<D><<<grid, kJThreads, jsm, st>>>(bf.gram, s.nb, s.max_sweeps, bf.eigvals, bf.eigvecs, bf.status);
   const size_t asm_ = (size_t)s.nb * (3 * sizeof(double) + sizeof(int));
   e = cudaFuncSetAttribute(alloc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asm_);
   if (e != cudaSuccess) return e;

@@ -1196,11 +1196,12 @@ struct TcPlan {
   CUtensorMap map_pacc;
 };
 
-bool tc_supported(const DecodeShape& s) {
+bool tc_shape_ok(const DecodeShape& s) {
   const int G = s.Hq / s.H;
-  return s.bf16 && (s.d == 64 || s.d == 128) && s.n % kChunk == 0 && G >= 1 && G <= 128 && s.Hq % s.H == 0 &&
-         encode_fn() != nullptr;
+  return s.bf16 && (s.d == 64 || s.d == 128) && s.n % kChunk == 0 && G >= 1 && G <= 128 && s.Hq % s.H == 0;
 }
+
+bool tc_supported(const DecodeShape& s) { return tc_shape_ok(s) && encode_fn() != nullptr; }
 
 int tc_launches(const DecodeShape&) { return 2; }
 
@@ -1225,193 +1226,12 @@ inline double suffix_atom_ns(int c, int d) {
   return 2.0 * 2.0 * kChunk * d / kBytesPerNs + kChunkNs + (c == 0 ? kUnitNs : 0.0);
 }
 
-static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& in) {
-  const int H = s.H, nb = s.nb, D = s.d, G = s.Hq / s.H, Bq = s.Bq, S = s.S;
-  const int cpb = s.n / kChunk;
-  const int ipt = std::min(Bq, 128 / G);
-  const int nrt = (Bq + ipt - 1) / ipt;
-  const int nsc = (S + kChunk - 1) / kChunk;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // atoms in processing order with their byte cost
-  struct Atom {
-    int type, h, tile, c;
-    double cost;
-  };
-  std::vector<Atom> atoms;
-  for (int h = 0; h < H; ++h)
-    for (int rt = 0; rt < nrt; ++rt)
-      for (int b = 0; b < nb; ++b) {
-        const int rk = in.host_ranks[(size_t)(2 * h) * nb + b], rv = in.host_ranks[(size_t)(2 * h + 1) * nb + b];
-        for (int cc = 0; cc < cpb; ++cc) atoms.push_back({0, h, rt, b * cpb + cc, prefix_atom_ns(rk, rv, cc, D)});
-      }
-  for (int i = 0; i < Bq; ++i)
-    for (int h = 0; h < H; ++h)
-      for (int c = 0; c < nsc; ++c)
-        atoms.push_back({1, h, i, c, suffix_atom_ns(c, D)});
-  double total = 0;
-  for (auto& a : atoms) total += a.cost;
-  const int grid = std::max(1, std::min(sms, (int)atoms.size()));
-  std::vector<Seg> segs;
-  std::vector<int> seg_first(grid + 1, 0);
-  std::vector<int> pre_range(2 * H * nrt, 0), suf_range(2 * Bq * H, 0);
-  double cum = 0;
-  int cta = 0;
-  for (size_t a = 0; a < atoms.size(); ++a) {
-    const Atom& at = atoms[a];
-    const double mid = cum + 0.5 * at.cost;
-    cum += at.cost;
-    while (cta + 1 < grid && mid >= total * (cta + 1) / grid) {
-      ++cta;
-      seg_first[cta] = (int)segs.size();
-    }
-    const bool cont = !segs.empty() && seg_first[cta] < (int)segs.size() && segs.back().type == at.type &&
-                      segs.back().h == at.h && segs.back().tile == at.tile && segs.back().c1 == at.c;
-    if (cont) {
-      segs.back().c1 = at.c + 1;
-    } else {
-      Seg sg{};
-      sg.type = at.type;
-      sg.h = at.h;
-      sg.tile = at.tile;
-      sg.c0 = at.c;
-      sg.c1 = at.c + 1;
-      sg.pid = (int)segs.size();
-      sg.rows = at.type == 0 ? std::min(ipt, Bq - at.tile * ipt) * G : G;
-      segs.push_back(sg);
-    }
-  }
-  for (int k = cta + 1; k <= grid; ++k) seg_first[k] = (int)segs.size();
-  // partial ranges per output row group (segments of one (h, tile) / (i, h) are consecutive)
-  for (int h = 0; h < H; ++h)
-    for (int rt = 0; rt < nrt; ++rt) pre_range[2 * (h * nrt + rt)] = pre_range[2 * (h * nrt + rt) + 1] = -1;
-  for (int i = 0; i < Bq; ++i)
-    for (int h = 0; h < H; ++h) suf_range[2 * (i * H + h)] = suf_range[2 * (i * H + h) + 1] = 0;
-  for (auto& sg : segs) {
-    int* r = sg.type == 0 ? &pre_range[2 * (sg.h * nrt + sg.tile)] : &suf_range[2 * (sg.tile * H + sg.h)];
-    if (sg.type == 0 && r[0] < 0) r[0] = sg.pid;
-    if (sg.type == 1 && r[1] == 0 && r[0] == 0) r[0] = sg.pid;
-    r[1] = sg.pid + 1;
-  }
-  for (int i = 0; i < 2 * H * nrt; ++i)
-    if (pre_range[i] < 0) pre_range[i] = 0;
-  for (int h = 0; h < H; ++h)
-    for (int i = 0; i < Bq; ++i) {
-      const int rt = i / ipt;
-      const int parts = pre_range[2 * (h * nrt + rt) + 1] - pre_range[2 * (h * nrt + rt)] +
-                        suf_range[2 * (i * H + h) + 1] - suf_range[2 * (i * H + h)];
-      if (parts > kMaxParts) return cudaErrorInvalidValue;
-    }
-  pl->off_segs = grid + 1;
-  pl->off_pre = pl->off_segs + (int)segs.size() * (int)(sizeof(Seg) / sizeof(int));
-  pl->off_suf = pl->off_pre + 2 * H * nrt;
-  const int nwords = pl->off_suf + 2 * Bq * H;
-  std::vector<int> host(nwords);
-  std::copy(seg_first.begin(), seg_first.end(), host.begin());
-  std::memcpy(host.data() + pl->off_segs, segs.data(), segs.size() * sizeof(Seg));
-  std::copy(pre_range.begin(), pre_range.end(), host.begin() + pl->off_pre);
-  std::copy(suf_range.begin(), suf_range.end(), host.begin() + pl->off_suf);
-  cudaError_t e;
-  if ((e = cudaMalloc((void**)&pl->d_work, nwords * sizeof(int))) != cudaSuccess) return e;
-  if ((e = cudaMemcpy(pl->d_work, host.data(), nwords * sizeof(int), cudaMemcpyHostToDevice)) != cudaSuccess)
-    return e;
-  const size_t np = std::max<size_t>(1, segs.size());
-  if ((e = cudaMalloc((void**)&pl->part_acc, np * 128 * D * sizeof(float))) != cudaSuccess) return e;
-  if ((e = cudaMalloc((void**)&pl->part_ml, np * 128 * sizeof(float2))) != cudaSuccess) return e;
-  pl->Bq = Bq;
-  pl->Hq = s.Hq;
-  pl->S = S;
-  pl->grid = grid;
-  pl->nsegs = (int)segs.size();
-  pl->ipt = ipt;
-  pl->nrt = nrt;
-  // factor maps: the token factor as a [rows · n/128][128] array of 128-token slab rows, the dim factor
-  // as [rows][d]
-  const uint64_t rows = (uint64_t)2 * H * in.pool_rows;
-  if (!make_row_maps(&pl->map_tok, in.tok, kChunk, rows * cpb)) return cudaErrorInvalidValue;
-  if (!make_row_maps(&pl->map_dim, in.dim, D, rows)) return cudaErrorInvalidValue;
-  if (!make_pacc_map(&pl->map_pacc, pl->part_acc, pl->nsegs, D)) return cudaErrorInvalidValue;
-  pl->tok = in.tok;
-  pl->dim = in.dim;
-  return prepare_kernel(D);
-}
-
-cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, void* out, cudaStream_t st,
-                      cudaEvent_t ev0, cudaEvent_t ev1) {
-  TcPlan* pl = *plan;
-  if (!pl || pl->Bq != s.Bq || pl->Hq != s.Hq || pl->S != s.S || pl->tok != in.tok) {
-    tc_plan_destroy(pl);
-    *plan = nullptr;
-    pl = new TcPlan();
-    cudaError_t e = build_plan(pl, s, in);
-    if (e != cudaSuccess) {
-      tc_plan_destroy(pl);
-      return e;
-    }
-    *plan = pl;
-  }
-  const int D = s.d, G = s.Hq / s.H;
-  Maps maps;
-  maps.tok = pl->map_tok;
-  maps.dim = pl->map_dim;
-  maps.pacc = pl->map_pacc;
-  if (!make_call_maps(&maps, s, in, pl->ipt)) return cudaErrorInvalidValue;
-  Params p;
-  p.seg_first = pl->d_work;
-  p.segs = reinterpret_cast<const Seg*>(pl->d_work + pl->off_segs);
-  p.ranks = in.ranks;
-  p.row_offsets = in.row_offsets;
-  p.part_acc = pl->part_acc;
-  p.part_ml = pl->part_ml;
-  p.status = in.status;
-  p.nb = s.nb;
-  p.cpb = s.n / kChunk;
-  p.H = s.H;
-  p.G = G;
-  p.ipt = pl->ipt;
-  p.S = s.S;
-  p.c = s.scale * 1.4426950408889634f;
-  cudaError_t e;
-  if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
-  if (D == 64)
-    decode_tc_kernel<64><<<pl->grid, kThreads, kSmemBytes, st>>>(maps, p);
-  else
-    decode_tc_kernel<128><<<pl->grid, kThreads, kSmemBytes, st>>>(maps, p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  if (ev1 && (e = cudaEventRecord(ev1, st)) != cudaSuccess) return e;
-  const int* pre = pl->d_work + pl->off_pre;
-  const int* suf = pl->d_work + pl->off_suf;
-  if (D == 64)
-    combine_tc_kernel<64><<<dim3(s.Hq, s.Bq), 64, 0, st>>>(pl->part_acc, pl->part_ml, pre, suf, s.H, s.Hq, pl->ipt,
-                                                          pl->nrt, static_cast<__nv_bfloat16*>(out));
-  else
-    combine_tc_kernel<128><<<dim3(s.Hq, s.Bq), 128, 0, st>>>(pl->part_acc, pl->part_ml, pre, suf, s.H, s.Hq,
-                                                            pl->ipt, pl->nrt, static_cast<__nv_bfloat16*>(out));
-  return cudaGetLastError();
-}
-
-
-// ================================================================================================
-// Decode without allocation: the same kernels, with their scratch (work list and partials) in a
-// fixed device array.  See milo_decode_attn_noalloc in milo.h.
-// ================================================================================================
-namespace {
-
-constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB, held by every device that loads us
-constexpr int kNoAllocMaxWords = 1 << 18;                  // host-side work-list staging (1 MiB)
-constexpr int kNoAllocMaxDevices = 64;
-
-static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
-
-std::mutex g_noalloc_mu;
-void* g_noalloc_dev_ptr[kNoAllocMaxDevices];  // device address of g_noalloc_scratch, per device
-bool g_noalloc_ready[kNoAllocMaxDevices][2];  // decode kernel prepared on the device, per head dim (64, 128)
-int g_noalloc_host_words[kNoAllocMaxWords];   // work list staging, guarded by g_noalloc_mu
-
-// Byte-balanced work list as in build_plan, written into `w` without heap allocation.
-// Returns the number of words used, or -1 if `cap` words are not enough.
+// The decode work list, written into `w` without heap allocation: atoms (one 128-token chunk of one KV head's
+// row tile, or one chunk of one query's suffix) in processing order, cut into `grid` runs of about equal
+// estimated time; consecutive atoms of one (head, tile) or (query, head) in a run form a segment.  Layout of
+// `w`: seg_first [grid + 1] | segments | pre_range [2·H·nrt] | suf_range [2·Bq·H] (each range: the partial
+// slots [first, end) of one output row group).  Returns the number of words used, or -1 if `cap` is too small
+// or a row would have more than kMaxParts partials.
 int build_worklist_fixed(const DecodeShape& s, const int32_t* host_ranks, int grid, int* w, int cap, int& nsegs,
                          int& off_segs, int& off_pre, int& off_suf, int& ipt_out, int& nrt_out) {
   const int H = s.H, nb = s.nb, D = s.d, G = s.Hq / s.H, Bq = s.Bq, S = s.S;
@@ -1502,7 +1322,150 @@ int build_worklist_fixed(const DecodeShape& s, const int32_t* host_ranks, int gr
   return nwords;
 }
 
+// CTAs of the decode kernel: one per SM, fewer when there are fewer atoms.
+int plan_grid(const DecodeShape& s, int sms) {
+  const int cpb = s.n / kChunk, nsc = (s.S + kChunk - 1) / kChunk;
+  const int ipt = std::min(s.Bq, 128 / (s.Hq / s.H));
+  const int64_t natoms =
+      (int64_t)s.H * ((s.Bq + ipt - 1) / ipt) * s.nb * cpb + (int64_t)s.Bq * s.H * nsc;
+  return (int)std::max<int64_t>(1, std::min<int64_t>(sms, natoms));
+}
+// Words a work list can need at most (every atom its own segment).
+int64_t worklist_cap(const DecodeShape& s, int grid) {
+  const int cpb = s.n / kChunk, nsc = (s.S + kChunk - 1) / kChunk;
+  const int ipt = std::min(s.Bq, 128 / (s.Hq / s.H)), nrt = (s.Bq + ipt - 1) / ipt;
+  const int64_t natoms = (int64_t)s.H * nrt * s.nb * cpb + (int64_t)s.Bq * s.H * nsc;
+  return grid + 1 + natoms * (int64_t)(sizeof(Seg) / sizeof(int)) + 2LL * s.H * nrt + 2LL * s.Bq * s.H;
+}
+
+static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& in) {
+  const int D = s.d;
+  const int cpb = s.n / kChunk;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = plan_grid(s, sms);
+  const int64_t cap = worklist_cap(s, grid);
+  if (cap > (int64_t)1 << 30) return cudaErrorInvalidValue;
+  std::vector<int> host((size_t)cap);
+  int nsegs = 0, off_segs = 0, off_pre = 0, off_suf = 0, ipt = 0, nrt = 0;
+  const int nwords = build_worklist_fixed(s, in.host_ranks, grid, host.data(), (int)cap, nsegs, off_segs, off_pre,
+                                          off_suf, ipt, nrt);
+  if (nwords < 0) return cudaErrorInvalidValue;
+  pl->off_segs = off_segs;
+  pl->off_pre = off_pre;
+  pl->off_suf = off_suf;
+  cudaError_t e;
+  if ((e = cudaMalloc((void**)&pl->d_work, nwords * sizeof(int))) != cudaSuccess) return e;
+  if ((e = cudaMemcpy(pl->d_work, host.data(), nwords * sizeof(int), cudaMemcpyHostToDevice)) != cudaSuccess)
+    return e;
+  const size_t np = std::max<size_t>(1, (size_t)nsegs);
+  if ((e = cudaMalloc((void**)&pl->part_acc, np * 128 * D * sizeof(float))) != cudaSuccess) return e;
+  if ((e = cudaMalloc((void**)&pl->part_ml, np * 128 * sizeof(float2))) != cudaSuccess) return e;
+  pl->Bq = s.Bq;
+  pl->Hq = s.Hq;
+  pl->S = s.S;
+  pl->grid = grid;
+  pl->nsegs = nsegs;
+  pl->ipt = ipt;
+  pl->nrt = nrt;
+  // factor maps: the token factor as a [rows · n/128][128] array of 128-token slab rows, the dim factor
+  // as [rows][d]
+  const uint64_t rows = (uint64_t)2 * s.H * in.pool_rows;
+  if (!make_row_maps(&pl->map_tok, in.tok, kChunk, rows * cpb)) return cudaErrorInvalidValue;
+  if (!make_row_maps(&pl->map_dim, in.dim, D, rows)) return cudaErrorInvalidValue;
+  if (!make_pacc_map(&pl->map_pacc, pl->part_acc, pl->nsegs, D)) return cudaErrorInvalidValue;
+  pl->tok = in.tok;
+  pl->dim = in.dim;
+  return prepare_kernel(D);
+}
+
+cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, void* out, cudaStream_t st,
+                      cudaEvent_t ev0, cudaEvent_t ev1) {
+  TcPlan* pl = *plan;
+  if (!pl || pl->Bq != s.Bq || pl->Hq != s.Hq || pl->S != s.S || pl->tok != in.tok) {
+    tc_plan_destroy(pl);
+    *plan = nullptr;
+    pl = new TcPlan();
+    cudaError_t e = build_plan(pl, s, in);
+    if (e != cudaSuccess) {
+      tc_plan_destroy(pl);
+      return e;
+    }
+    *plan = pl;
+  }
+  const int D = s.d, G = s.Hq / s.H;
+  Maps maps;
+  maps.tok = pl->map_tok;
+  maps.dim = pl->map_dim;
+  maps.pacc = pl->map_pacc;
+  if (!make_call_maps(&maps, s, in, pl->ipt)) return cudaErrorInvalidValue;
+  Params p;
+  p.seg_first = pl->d_work;
+  p.segs = reinterpret_cast<const Seg*>(pl->d_work + pl->off_segs);
+  p.ranks = in.ranks;
+  p.row_offsets = in.row_offsets;
+  p.part_acc = pl->part_acc;
+  p.part_ml = pl->part_ml;
+  p.status = in.status;
+  p.nb = s.nb;
+  p.cpb = s.n / kChunk;
+  p.H = s.H;
+  p.G = G;
+  p.ipt = pl->ipt;
+  p.S = s.S;
+  p.c = s.scale * 1.4426950408889634f;
+  cudaError_t e;
+  if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
+  if (D == 64)
+    decode_tc_kernel<64><<<pl->grid, kThreads, kSmemBytes, st>>>(maps, p);
+  else
+    decode_tc_kernel<128><<<pl->grid, kThreads, kSmemBytes, st>>>(maps, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (ev1 && (e = cudaEventRecord(ev1, st)) != cudaSuccess) return e;
+  const int* pre = pl->d_work + pl->off_pre;
+  const int* suf = pl->d_work + pl->off_suf;
+  if (D == 64)
+    combine_tc_kernel<64><<<dim3(s.Hq, s.Bq), 64, 0, st>>>(pl->part_acc, pl->part_ml, pre, suf, s.H, s.Hq, pl->ipt,
+                                                          pl->nrt, static_cast<__nv_bfloat16*>(out));
+  else
+    combine_tc_kernel<128><<<dim3(s.Hq, s.Bq), 128, 0, st>>>(pl->part_acc, pl->part_ml, pre, suf, s.H, s.Hq,
+                                                            pl->ipt, pl->nrt, static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError();
+}
+
+
+// ================================================================================================
+// Decode without allocation: the same kernels, with their scratch (work list and partials) in a
+// fixed device array.  See milo_decode_attn_noalloc in milo.h.
+// ================================================================================================
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB, held by every device that loads us
+constexpr int kNoAllocMaxWords = 1 << 18;                  // host-side work-list staging (1 MiB)
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_dev_ptr[kNoAllocMaxDevices];  // device address of g_noalloc_scratch, per device
+bool g_noalloc_ready[kNoAllocMaxDevices][2];  // decode kernel prepared on the device, per head dim (64, 128)
+int g_noalloc_host_words[kNoAllocMaxWords];   // work list staging, guarded by g_noalloc_mu
+
 }  // namespace
+
+int tc_worklist(const DecodeShape& s, const int32_t* host_ranks, int sms, int* w, int64_t cap, int64_t* info) {
+  if (cap > INT32_MAX) cap = INT32_MAX;
+  const int grid = plan_grid(s, sms);
+  int nsegs = 0, off_segs = 0, off_pre = 0, off_suf = 0, ipt = 0, nrt = 0;
+  const int nwords =
+      build_worklist_fixed(s, host_ranks, grid, w, (int)cap, nsegs, off_segs, off_pre, off_suf, ipt, nrt);
+  if (nwords < 0) return -1;
+  const int64_t v[8] = {nwords, nsegs, grid, off_segs, off_pre, off_suf, ipt, nrt};
+  for (int i = 0; i < 8; ++i) info[i] = v[i];
+  return nwords;
+}
 
 size_t tc_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 
@@ -1527,11 +1490,8 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
   unsigned char* scratch = static_cast<unsigned char*>(g_noalloc_dev_ptr[dev]);
   int sms = 148;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  const int cpb = s.n / kChunk, nsc = (s.S + kChunk - 1) / kChunk;
-  const int64_t natoms = (int64_t)s.H * ((s.Bq + std::min(s.Bq, 128 / (s.Hq / s.H)) - 1) /
-                                         std::min(s.Bq, 128 / (s.Hq / s.H))) * s.nb * cpb +
-                         (int64_t)s.Bq * s.H * nsc;
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sms, natoms));
+  const int cpb = s.n / kChunk;
+  const int grid = plan_grid(s, sms);
   int nsegs = 0, off_segs = 0, off_pre = 0, off_suf = 0, ipt = 0, nrt = 0;
   const int nwords = build_worklist_fixed(s, in.host_ranks, grid, g_noalloc_host_words, kNoAllocMaxWords, nsegs,
                                           off_segs, off_pre, off_suf, ipt, nrt);

@@ -23,6 +23,8 @@ struct TcInputs {
   const int32_t* host_ranks;  // [2H][nb]
 };
 
+// The shape check alone (no CUDA call): bf16, d in {64, 128}, n % 128 == 0, GQA group <= 128.
+bool tc_shape_ok(const DecodeShape& s);
 bool tc_supported(const DecodeShape& s);
 int tc_launches(const DecodeShape& s);
 // ev0 / ev1 (optional) are recorded on `st` right before and right after the main decode kernel.
@@ -35,5 +37,8 @@ void tc_plan_destroy(TcPlan* plan);
 cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* out, cudaStream_t st,
                               bool* too_large);
 size_t tc_noalloc_scratch_bytes();
+// The work list for ranks / shape on a GPU with `sms` SMs into w[cap] (host only); info as in
+// milo_decode_worklist.  Returns the words used, or -1 if cap is too small.
+int tc_worklist(const DecodeShape& s, const int32_t* host_ranks, int sms, int* w, int64_t cap, int64_t* info);
 
 }  // namespace milo

@@ -304,6 +304,22 @@ void milo_factors_destroy(milo_factors* f) {
   delete f;
 }
 
+milo_status milo_decode_worklist(const int32_t* host_ranks, int32_t num_kv_heads, int32_t num_blocks,
+                                 int32_t block_size, int32_t head_dim, int32_t batch, int32_t num_q_heads,
+                                 int32_t suffix_len, int32_t num_ctas, int32_t* out, int64_t capacity,
+                                 int64_t* info) {
+  if (!host_ranks || !out || !info || num_kv_heads <= 0 || num_blocks <= 0 || block_size <= 0 || head_dim <= 0 ||
+      batch <= 0 || num_q_heads <= 0 || suffix_len < 0 || num_ctas <= 0 || capacity <= 0 ||
+      num_q_heads % num_kv_heads != 0)
+    return MILO_ERR_INVALID_ARGUMENT;
+  for (int64_t i = 0; i < 2LL * num_kv_heads * num_blocks; ++i)
+    if (host_ranks[i] < 1 || host_ranks[i] > head_dim) return MILO_ERR_INVALID_ARGUMENT;
+  milo::DecodeShape ds{num_kv_heads, num_blocks, block_size, head_dim, batch, num_q_heads, suffix_len, true, 1.f};
+  if (!milo::tc_shape_ok(ds)) return MILO_ERR_UNSUPPORTED;
+  if (milo::tc_worklist(ds, host_ranks, num_ctas, out, capacity, info) < 0) return MILO_ERR_UNSUPPORTED;
+  return MILO_OK;
+}
+
 int32_t milo_decode_launches(const milo_factors* f, int32_t batch, int32_t num_q_heads, int32_t suffix_len) {
   if (!f || batch <= 0 || num_q_heads <= 0 || suffix_len < 0 || num_q_heads % f->H != 0)
     return -(int32_t)MILO_ERR_INVALID_ARGUMENT;

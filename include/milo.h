@@ -193,6 +193,28 @@ milo_status milo_decode_attn_noalloc(const void* q, int32_t batch, int32_t num_q
  */
 int32_t milo_decode_launches(const milo_factors* f, int32_t batch, int32_t num_q_heads, int32_t suffix_len);
 
+/*
+ * Host only (no GPU, no CUDA call): the work list that the bf16 tensor-core decode builds for these ranks
+ * and this decode shape on a GPU with num_ctas SMs (one CTA per SM, fewer when there are fewer chunks
+ * than SMs), for inspection and testing.  The
+ * decode splits the compressed prefix of each (KV head, row tile) into 128-token chunks and each query's
+ * suffix into 128-token chunks (the rank-space decode of page "MILO", §4.4), and cuts the sequence of
+ * chunks into one run per CTA of about equal estimated time.
+ *   host_ranks  [2H][nb] int32 (per head: K ranks, then V ranks), each in [1, head_dim]; caller-owned.
+ *   out         capacity int32 words, written: seg_first [CTAs + 1] | segments, 8 words each
+ *               {kind (0 prefix, 1 suffix), KV head, row tile (prefix) or query (suffix), first chunk,
+ *               end chunk, partial slot, valid rows, 0} | pre_range [2·H·tiles] | suf_range [2·batch·H]
+ *               (each range: the [first, end) partial slots of one output row group).
+ *   info        8 int64, written: {words used, segments, CTAs, offset of the segments, offset of
+ *               pre_range, offset of suf_range, query items per row tile, row tiles per head}.
+ * Errors: MILO_ERR_INVALID_ARGUMENT for a bad shape or rank, MILO_ERR_UNSUPPORTED for a shape the
+ * tensor-core decode does not take or a capacity that is too small.
+ */
+milo_status milo_decode_worklist(const int32_t* host_ranks, int32_t num_kv_heads, int32_t num_blocks,
+                                 int32_t block_size, int32_t head_dim, int32_t batch, int32_t num_q_heads,
+                                 int32_t suffix_len, int32_t num_ctas, int32_t* out, int64_t capacity,
+                                 int64_t* info);
+
 /* Copies the ranks [2H][nb] to host memory. Synchronises the compress stream. */
 milo_status milo_factors_ranks(const milo_factors* f, int32_t* host_ranks);
 
