@@ -24,6 +24,14 @@ def _setup(name, beta=None, batch=None, suffix=None, q_scale=1.0, seed_override=
     lay = stored_layer(oracle.compress_layer(K, V, wl.block_size, beta, wl.r_min), dt)
     q = L["q"]
     Ks, Vs = L["K_suf"], L["V_suf"]
+    if batch is not None and batch > q.shape[0]:
+        # more queries than the workload draws: append sign-flipped, rescaled copies (distinct rows, each
+        # with its own copy of a suffix)
+        from synth import to_storage
+        reps = -(-batch // q.shape[0])
+        qf = from_storage(q, dt)
+        q = to_storage(np.concatenate([qf * (-0.6) ** k for k in range(reps)]), dt)
+        Ks, Vs = np.concatenate([Ks] * reps), np.concatenate([Vs] * reps)
     if batch is not None:
         q, Ks, Vs = q[:batch], Ks[:batch], Vs[:batch]
     if suffix is not None:
@@ -67,6 +75,14 @@ def test_decode_sharp_softmax_7b():
 
 @pytest.mark.parametrize("batch,suffix", [(1, 0), (3, 7), (16, 0), (5, 129)])
 def test_decode_ragged_shapes_7b(batch, suffix):
+    wl, dt, lay, f, q, Ks, Vs = _setup("qwen2.5-7b-layer", batch=batch, suffix=suffix)
+    out, want = _run(wl, dt, lay, f, q, Ks, Vs)
+    assert rel_l2(out, want) <= TOL[dt]
+
+
+@pytest.mark.parametrize("batch,suffix", [(40, 100), (19, 0)])
+def test_decode_several_row_tiles_7b(batch, suffix):
+    """More query rows than one 128-row tile per KV head (GQA group 7: 18 queries per tile)."""
     wl, dt, lay, f, q, Ks, Vs = _setup("qwen2.5-7b-layer", batch=batch, suffix=suffix)
     out, want = _run(wl, dt, lay, f, q, Ks, Vs)
     assert rel_l2(out, want) <= TOL[dt]
