@@ -165,17 +165,17 @@ __device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, Shared
   for (uint32_t i = 1;; ++i) {
     if (__all_sync(0xffffffffu, ptx::mbar_try_wait(bar, parity))) return true;
     if ((i & 63) == 0) {
-      int verdict = 0;  // 0 keep waiting, 1 aborted elsewhere, 2 timed out
+      int outcome = 0;  // 0 keep waiting, 1 aborted elsewhere, 2 timed out
       if ((threadIdx.x & 31) == 0) {
-        if (!drain && *(volatile int*)&sh->abort_flag) verdict = 1;
-        else if (ptx::globaltimer() - t0 > kWaitNs) verdict = 2;
+        if (!drain && *(volatile int*)&sh->abort_flag) outcome = 1;
+        else if (ptx::globaltimer() - t0 > kWaitNs) outcome = 2;
       }
-      verdict = __shfl_sync(0xffffffffu, verdict, 0);
-      if (verdict == 2 && (threadIdx.x & 31) == 0) {
+      outcome = __shfl_sync(0xffffffffu, outcome, 0);
+      if (outcome == 2 && (threadIdx.x & 31) == 0) {
         atomicOr(status, kStatusDecodeTimeout);
         *(volatile int*)&sh->abort_flag = 1;
       }
-      if (verdict) return false;
+      if (outcome) return false;
     }
   }
 }
