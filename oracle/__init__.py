@@ -17,6 +17,9 @@ page is silent.
 from .milo import (  # noqa: F401
     BudgetError,
     allocate_ranks,
+    allocate_ranks_greedy,
+    allocate_ranks_random,
+    allocate_ranks_uniform,
     block_svd,
     compress_layer,
     compress_pool,

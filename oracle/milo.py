@@ -115,6 +115,57 @@ def allocate_ranks(w, R: int, r_min: int, d: int):
     return ranks, q, lam
 
 
+def allocate_ranks_greedy(sigma, R: int, r_min: int, d: int) -> np.ndarray:
+    """Greedy marginal-gain allocation, the form §4.3 describes in words.
+
+    The allocation starts every block at the minimum rank and then hands out the
+    remaining rank units one at a time, each to the block with the largest marginal
+    gain.  Reading of "marginal information gain": the share of the block's spectral
+    energy carried by its next component, g_b(i) = σ_{b,i}² / Σ_j σ_{b,j}² for
+    i = r_b + 1 (the distribution whose entropy H_b is), so blocks whose spectrum decays
+    slowly keep receiving units; ties go to the lower block index; a block at rank d
+    takes no more.  sigma: [nb][d] singular values per block, descending.
+
+    Returns ranks int64[nb].  Raises BudgetError if R < nb · r_min; R >= nb · d gives d
+    everywhere.
+    """
+    sigma = np.asarray(sigma, dtype=np.float64)
+    nb = sigma.shape[0]
+    if R < nb * r_min:
+        raise BudgetError(f"total rank {R} < {nb} blocks x r_min {r_min}")
+    if R >= nb * d:
+        return np.full(nb, d, dtype=np.int64)
+    energy = sigma[:, :d] ** 2
+    tot = energy.sum(axis=1)
+    share = np.divide(energy, tot[:, None], out=np.zeros_like(energy), where=tot[:, None] > 0)
+    ranks = np.full(nb, r_min, dtype=np.int64)
+    for _ in range(R - nb * r_min):
+        gain = np.where(ranks < d, share[np.arange(nb), np.minimum(ranks, d - 1)], -np.inf)
+        b = int(np.argmax(gain))  # first maximum: ties to the lower block index
+        ranks[b] += 1
+    return ranks
+
+
+def allocate_ranks_uniform(nb: int, R: int, r_min: int, d: int) -> np.ndarray:
+    """Uniform baseline of §5.3's allocation comparison: every block floor(R / nb), the
+    R mod nb leftover units to the lowest block indices, within [r_min, d]."""
+    if R < nb * r_min:
+        raise BudgetError(f"total rank {R} < {nb} blocks x r_min {r_min}")
+    if R >= nb * d:
+        return np.full(nb, d, dtype=np.int64)
+    ranks = np.full(nb, R // nb, dtype=np.int64)
+    ranks[: R % nb] += 1
+    return ranks
+
+
+def allocate_ranks_random(nb: int, R: int, r_min: int, d: int, rng) -> np.ndarray:
+    """Random baseline of §5.3's allocation comparison: ranks proportional to weights drawn
+    uniformly from [1, d] (the range of e^{H_b}), with the same water-filling and rounding
+    as the entropy rule.  rng: a numpy Generator (the caller seeds it)."""
+    w = rng.uniform(1.0, float(d), size=nb)
+    return allocate_ranks(w, R, r_min, d)[0]
+
+
 def compress_pool(x: np.ndarray, n: int, beta: float, r_min: int) -> dict:
     """Compress one pool [T][d]: partition, per-block SVD, entropy, ranks, factors.
 

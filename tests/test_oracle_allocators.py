@@ -1,0 +1,94 @@
+"""Oracle pins for the allocators of MILO §4.3 and §5.3 beyond the entropy rule.
+
+§4.3 describes the allocation as greedy: start at the minimum rank and give each remaining
+rank unit to the block with the largest marginal gain.  §5.3 compares entropy allocation with
+uniform and random allocation under the same total budget.  These tests pin the oracle's
+versions: hand-derived worked examples (tests/golden), exact optimality of the greedy on small
+problems (brute force over every rank vector), invariants, and the baselines' definitions.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from synth import WORKLOADS, gen_block_f64
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "greedy_alloc_worked_examples.json")
+
+
+def _shares(sigma):
+    e = np.asarray(sigma, dtype=np.float64) ** 2
+    t = e.sum(axis=1, keepdims=True)
+    return np.divide(e, t, out=np.zeros_like(e), where=t > 0)
+
+
+def _captured(sigma, ranks):
+    s = _shares(sigma)
+    return sum(s[b, :r].sum() for b, r in enumerate(ranks))
+
+
+def test_greedy_worked_examples():
+    for case in json.load(open(GOLDEN))["cases"]:
+        got = oracle.allocate_ranks_greedy(case["sigma"], case["R"], case["r_min"], case["d"])
+        assert list(got) == case["ranks"], case["name"]
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_greedy_is_optimal_by_brute_force(seed):
+    """The greedy maximises the captured energy shares Σ_b Σ_{i<=r_b} g_b(i) over every rank vector
+    with Σ r = R and r_min <= r <= d (each block's shares are non-increasing, so greedy is exact)."""
+    rng = np.random.default_rng(seed)
+    nb, d, r_min = 3, 6, 1
+    sigma = np.sort(rng.exponential(1.0, size=(nb, d)) ** rng.uniform(0.5, 3.0, size=(nb, 1)), axis=1)[:, ::-1]
+    R = int(rng.integers(nb * r_min + 1, nb * d))
+    got = oracle.allocate_ranks_greedy(sigma, R, r_min, d)
+    best = max(_captured(sigma, r) for r in itertools.product(range(r_min, d + 1), repeat=nb) if sum(r) == R)
+    assert got.sum() == R
+    assert _captured(sigma, got) == pytest.approx(best, rel=1e-12)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_greedy_invariants(seed):
+    rng = np.random.default_rng(100 + seed)
+    nb, d = int(rng.integers(2, 40)), int(rng.choice([64, 128]))
+    r_min = int(rng.integers(1, 8))
+    sigma = np.sort(rng.exponential(1.0, size=(nb, d)), axis=1)[:, ::-1]
+    R = int(rng.integers(nb * r_min, nb * d))
+    r = oracle.allocate_ranks_greedy(sigma, R, r_min, d)
+    assert r.sum() == R and r.min() >= r_min and r.max() <= d
+    assert np.array_equal(oracle.allocate_ranks_greedy(sigma * 7.5, R, r_min, d), r)  # scale-free shares
+    assert list(oracle.allocate_ranks_greedy(sigma, nb * r_min, r_min, d)) == [r_min] * nb
+    assert list(oracle.allocate_ranks_greedy(sigma, nb * d + 3, r_min, d)) == [d] * nb
+    with pytest.raises(oracle.BudgetError):
+        oracle.allocate_ranks_greedy(sigma, nb * r_min - 1, r_min, d)
+
+
+def test_greedy_gives_slower_decay_more_rank_noise_free():
+    wl = WORKLOADS["tiny"]
+    taus = [1.5, 3.0, 6.0, 12.0]
+    sig = np.array([oracle.block_svd(gen_block_f64(wl, 0, 0, 0, b, t, noise_std=0.0))[0] for b, t in enumerate(taus)])
+    n, d = wl.block_size, wl.head_dim
+    R = oracle.rank_total(0.5, len(taus) * n, n, d)
+    r = oracle.allocate_ranks_greedy(sig, R, 4, d)
+    assert r.sum() == R and np.all(np.diff(r) >= 0)
+
+
+def test_uniform_baseline():
+    assert list(oracle.allocate_ranks_uniform(4, 10, 1, 8)) == [3, 3, 2, 2]
+    assert list(oracle.allocate_ranks_uniform(3, 12, 4, 64)) == [4, 4, 4]
+    assert list(oracle.allocate_ranks_uniform(2, 40, 4, 16)) == [16, 16]
+    # the same as the entropy rule's water-filling with equal weights
+    for nb, R in [(5, 23), (64, 3276), (7, 7 * 128 - 1)]:
+        want = oracle.allocate_ranks(np.ones(nb), R, 4, 128)[0]
+        assert np.array_equal(oracle.allocate_ranks_uniform(nb, R, 4, 128), want)
+
+
+def test_random_baseline_is_a_valid_seeded_allocation():
+    a = oracle.allocate_ranks_random(64, 3276, 4, 128, np.random.default_rng(5))
+    b = oracle.allocate_ranks_random(64, 3276, 4, 128, np.random.default_rng(5))
+    assert np.array_equal(a, b) and a.sum() == 3276 and a.min() >= 4 and a.max() <= 128
+    assert not np.array_equal(a, oracle.allocate_ranks_uniform(64, 3276, 4, 128))
