@@ -31,4 +31,4 @@ from .milo import (  # noqa: F401
     stored_factors,
 )
 from .hestenes import hestenes_svd  # noqa: F401
-from .tiefree import cut_gap, tiefree_taus  # noqa: F401
+from .tiefree import cut_gap, greedy_cut_gap, tiefree_taus  # noqa: F401

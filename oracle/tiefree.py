@@ -32,6 +32,27 @@ def cut_gap(quotas: np.ndarray, R: int) -> tuple[float, int]:
     return float(frac[order[rem - 1]] - frac[order[rem]]), int(order[rem])
 
 
+def greedy_cut_gap(sigma, R: int, r_min: int, d: int) -> float:
+    """Margin of the greedy marginal-gain allocation (allocate_ranks_greedy).
+
+    The greedy hands the R − nb·r_min free units to the largest next-component shares; its
+    result only changes where the smallest share it took meets the largest share it left
+    (across blocks, with blocks already at d excluded).  Returns that difference (inf when
+    no unit is free or none is left), so a GPU whose shares are off by less than half of it
+    makes the same choices."""
+    sigma = np.asarray(sigma, dtype=np.float64)
+    nb = sigma.shape[0]
+    if R <= nb * r_min or R >= nb * d:
+        return float("inf")
+    e = sigma[:, :d] ** 2
+    t = e.sum(axis=1, keepdims=True)
+    share = np.divide(e, t, out=np.zeros_like(e), where=t > 0)
+    free = share[:, r_min:d]  # candidate units i = r_min+1 .. d of every block (0-based columns r_min..d-1)
+    vals = np.sort(free.ravel())[::-1]
+    k = R - nb * r_min
+    return float(vals[k - 1] - vals[k])
+
+
 def _block_entropy(wl, layer, head, tensor, b, tau):
     x = wlmod.gen_block_f64(wl, layer, head, tensor, b, tau)
     if tensor == wlmod.KEY:

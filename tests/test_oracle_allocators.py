@@ -92,3 +92,27 @@ def test_random_baseline_is_a_valid_seeded_allocation():
     b = oracle.allocate_ranks_random(64, 3276, 4, 128, np.random.default_rng(5))
     assert np.array_equal(a, b) and a.sum() == 3276 and a.min() >= 4 and a.max() <= 128
     assert not np.array_equal(a, oracle.allocate_ranks_uniform(64, 3276, 4, 128))
+
+
+def test_greedy_cut_gap_predicts_stability():
+    """Perturbing every share by less than half the cut gap leaves the greedy ranks unchanged; the
+    gap is the difference between the smallest share taken and the largest share left."""
+    rng = np.random.default_rng(11)
+    nb, d, r_min = 8, 16, 2
+    sigma = np.sort(rng.exponential(1.0, size=(nb, d)) ** 1.5, axis=1)[:, ::-1]
+    R = 60
+    r = oracle.allocate_ranks_greedy(sigma, R, r_min, d)
+    gap = oracle.greedy_cut_gap(sigma, R, r_min, d)
+    s = _shares(sigma)
+    taken = [s[b, i] for b in range(nb) for i in range(r_min, r[b])]
+    left = [s[b, i] for b in range(nb) for i in range(r[b], d)]
+    assert gap == pytest.approx(min(taken) - max(left), abs=1e-15)
+    assert gap > 0
+    for k in range(20):
+        # multiplicative noise on the energies that moves every share by less than gap / 2
+        eps = 0.2 * gap * rng.uniform(-1, 1, size=sigma.shape)
+        e = sigma ** 2
+        s2 = e / e.sum(axis=1, keepdims=True) + eps
+        sig2 = np.sqrt(np.maximum(s2, 0) * e.sum(axis=1, keepdims=True))
+        assert np.array_equal(oracle.allocate_ranks_greedy(sig2, R, r_min, d), r)
+    assert oracle.greedy_cut_gap(sigma, nb * r_min, r_min, d) == float("inf")
