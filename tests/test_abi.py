@@ -72,3 +72,33 @@ def test_import_rejects_unequal_pools():
                                    tok.ctypes.data_as(ctypes.c_void_p), tok.ctypes.data_as(ctypes.c_void_p),
                                    None, ctypes.byref(out))
     assert code == 1
+
+
+def test_every_status_code_has_a_string():
+    lib = milo.load_library()
+    seen = set()
+    for code in range(8):
+        s = lib.milo_status_string(code)
+        assert s and s not in seen, code
+        seen.add(s)
+    assert lib.milo_status_string(99)  # unknown codes still get a string
+
+
+def test_host_only_calls_reject_bad_arguments():
+    import numpy as np
+    lib = milo.load_library()
+    assert lib.milo_decode_launches(None, 1, 28, 0) == -1
+    assert lib.milo_decode_attn_noalloc(None, 1, 2, None, None, None, 0, 0.0, None, None) == 1
+    ranks = np.full((8, 4), 16, dtype=np.int32)
+    out = np.zeros(1 << 12, dtype=np.int32)
+    info = np.zeros(8, dtype=np.int64)
+    call = lambda **kw: lib.milo_decode_worklist(
+        ranks.ctypes.data, kw.get("H", 4), 4, kw.get("n", 512), 128, kw.get("B", 16), kw.get("Hq", 28),
+        kw.get("S", 0), kw.get("ctas", 148), out.ctypes.data, kw.get("cap", out.size), info.ctypes.data)
+    assert call() == 0 and info[0] > 0 and info[1] >= 1
+    assert call(Hq=27) == 1        # query heads not a multiple of KV heads
+    assert call(B=0) == 1
+    assert call(ctas=0) == 1
+    assert call(S=-1) == 1
+    assert call(n=384 + 64) == 2   # block size not a multiple of 128
+    assert call(cap=4) == 2        # output too small
