@@ -123,6 +123,7 @@ class Factors:
 
     def __init__(self, handle: ctypes.c_void_p):
         self._h = handle
+        self._shape = None
 
     @property
     def handle(self):
@@ -134,6 +135,13 @@ class Factors:
         d = _Desc()
         _check(load_library().milo_factors_describe(self.handle, ctypes.byref(d)), "milo_factors_describe")
         return {name: getattr(d, name) for name, _ in _Desc._fields_}
+
+    def shape(self) -> tuple[int, int, int]:
+        """(KV heads, head dim, dtype code) of the factors (cached: they never change)."""
+        if self._shape is None:
+            d = self.describe()
+            self._shape = (d["num_kv_heads"], d["head_dim"], d["dtype"])
+        return self._shape
 
     def ranks(self) -> np.ndarray:
         d = self.describe()
@@ -180,19 +188,39 @@ def compress(K, V, block_size: int, budget: float, r_min: int = 4, max_sweeps: i
     return Factors(h)
 
 
-def decode_attn(q, factors: Factors, K_suf=None, V_suf=None, scale: float = 0.0, out=None, stream=None):
-    """One decode step: q [B][Hq][d] → out [B][Hq][d]. Suffix K/V [B][H][S][d] or None. See milo_decode_attn."""
+def _decode_args(q, factors: Factors, K_suf, V_suf, out):
+    """Checks the shapes and dtypes of one decode call against the factors (the C ABI takes no q shape or
+    dtype beyond batch and heads, so a mismatched tensor would be read or written past its end) and
+    returns (batch, q heads, suffix length, out)."""
     import torch
-    if q.dim() != 3:
-        raise ValueError("q must be [batch][q_heads][d]")
-    B, Hq, d = q.shape
+    H, d, dt = factors.shape()
+    want = torch.bfloat16 if dt == BF16 else torch.float32
+    if q.dim() != 3 or q.shape[2] != d or q.shape[1] % H != 0 or q.shape[0] < 1:
+        raise ValueError(f"q must be [batch][q_heads][{d}] with q_heads a multiple of {H}, got {tuple(q.shape)}")
+    if q.dtype != want:
+        raise ValueError(f"q must have the factors' dtype {want}, got {q.dtype}")
+    B, Hq, _ = q.shape
     S = 0
-    if K_suf is not None:
-        if V_suf is None or K_suf.shape != V_suf.shape or K_suf.dim() != 4 or K_suf.shape[0] != B:
-            raise ValueError("K_suf and V_suf must both be [batch][kv_heads][S][d]")
+    if K_suf is not None or V_suf is not None:
+        if K_suf is None or V_suf is None:
+            raise ValueError("K_suf and V_suf must be given together")
+        if K_suf.dim() != 4 or tuple(K_suf.shape) != tuple(V_suf.shape) or tuple(K_suf.shape[:2]) != (B, H) \
+                or K_suf.shape[3] != d:
+            raise ValueError(f"K_suf and V_suf must both be [{B}][{H}][S][{d}], got {tuple(K_suf.shape)} and "
+                             f"{tuple(V_suf.shape)}")
+        if K_suf.dtype != want or V_suf.dtype != want:
+            raise ValueError(f"K_suf and V_suf must have the factors' dtype {want}")
         S = K_suf.shape[2]
     if out is None:
         out = torch.empty_like(q)
+    elif tuple(out.shape) != tuple(q.shape) or out.dtype != want:
+        raise ValueError(f"out must be {tuple(q.shape)} of dtype {want}, got {tuple(out.shape)} {out.dtype}")
+    return B, Hq, S, out
+
+
+def decode_attn(q, factors: Factors, K_suf=None, V_suf=None, scale: float = 0.0, out=None, stream=None):
+    """One decode step: q [B][Hq][d] → out [B][Hq][d]. Suffix K/V [B][H][S][d] or None. See milo_decode_attn."""
+    B, Hq, S, out = _decode_args(q, factors, K_suf, V_suf, out)
     _check(load_library().milo_decode_attn(_dev_ptr(q, "q"), B, Hq, factors.handle,
                                            _dev_ptr(K_suf, "K_suf") if S else None,
                                            _dev_ptr(V_suf, "V_suf") if S else None, S, float(scale),
@@ -203,8 +231,7 @@ def decode_attn(q, factors: Factors, K_suf=None, V_suf=None, scale: float = 0.0,
 def decode_attn_profiled(q, factors: Factors, K_suf, V_suf, out, event_before, event_after, scale: float = 0.0,
                          stream=None):
     """decode_attn that records two torch.cuda.Event objects around the main decode kernel."""
-    B, Hq, _ = q.shape
-    S = 0 if K_suf is None else K_suf.shape[2]
+    B, Hq, S, out = _decode_args(q, factors, K_suf, V_suf, out)
     _check(load_library().milo_decode_attn_profiled(
         _dev_ptr(q, "q"), B, Hq, factors.handle, _dev_ptr(K_suf, "K_suf") if S else None,
         _dev_ptr(V_suf, "V_suf") if S else None, S, float(scale), _dev_ptr(out, "out"), _stream_ptr(stream),
@@ -215,11 +242,7 @@ def decode_attn_profiled(q, factors: Factors, K_suf, V_suf, out, event_before, e
 
 def decode_attn_noalloc(q, factors: Factors, K_suf=None, V_suf=None, scale: float = 0.0, out=None, stream=None):
     """decode_attn through milo_decode_attn_noalloc: the library allocates nothing (bf16 factors only)."""
-    import torch
-    B, Hq, _ = q.shape
-    S = 0 if K_suf is None else K_suf.shape[2]
-    if out is None:
-        out = torch.empty_like(q)
+    B, Hq, S, out = _decode_args(q, factors, K_suf, V_suf, out)
     _check(load_library().milo_decode_attn_noalloc(
         _dev_ptr(q, "q"), B, Hq, factors.handle, _dev_ptr(K_suf, "K_suf") if S else None,
         _dev_ptr(V_suf, "V_suf") if S else None, S, float(scale), _dev_ptr(out, "out"), _stream_ptr(stream)),

@@ -32,7 +32,10 @@ struct milo_factors {
   cudaEvent_t ready = nullptr;  // recorded after the factors are written
   // decode scratch, owned here and reused by later calls
   std::mutex mu;
+  // host copy of the ranks for the work-list builder: sized when the object is made, filled (one
+  // synchronisation) by the first decode call, so that no later call allocates or waits for it
   std::vector<int32_t> host_ranks;
+  bool host_ranks_valid = false;
   float* partials = nullptr;
   size_t partials_floats = 0;
   milo::TcPlan* tc_plan = nullptr;
@@ -69,6 +72,10 @@ void free_all(milo_factors* f) {
   if (f->ready) cudaEventDestroy(f->ready);
   milo::tc_plan_destroy(f->tc_plan);
 }
+
+// Blocks per pool that milo_compress takes: its allocation step holds 28 bytes per block of a pool in
+// shared memory (224 KB at this limit, within the 227 KB a CTA may use).
+constexpr int kMaxAllocBlocks = 8192;
 
 bool valid_dtype(int32_t dt) { return dt == MILO_F32 || dt == MILO_BF16; }
 
@@ -111,6 +118,8 @@ milo_status milo_compress(const void* K, const void* V, int32_t dtype, int32_t n
   if (!(budget > 0.0) || !isfinite(budget) || max_sweeps < 0 || (flags & ~MILO_KEEP_INTERMEDIATES))
     return MILO_ERR_INVALID_ARGUMENT;
   const int nb = (int)(context / block_size);
+  // the allocation kernel keeps 28 bytes per block of a pool in shared memory
+  if (nb > kMaxAllocBlocks) return MILO_ERR_UNSUPPORTED;
   const double Rd = floor(budget * (double)(context * head_dim) / (double)(block_size + head_dim));
   if (Rd < (double)nb * r_min) return MILO_ERR_BUDGET;
   const int64_t full = (int64_t)nb * head_dim;
@@ -130,6 +139,7 @@ milo_status milo_compress(const void* K, const void* V, int32_t dtype, int32_t n
   f->dtype = dtype;
   f->flags = flags;
   const int P = 2 * num_kv_heads;
+  f->host_ranks.assign((size_t)P * nb, 0);
   const size_t rows = (size_t)P * f->pool_rows;
   const size_t nblk = (size_t)P * nb;
   const size_t dd = (size_t)head_dim * head_dim;
@@ -252,6 +262,7 @@ milo_status milo_factors_import(int32_t dtype, int32_t num_kv_heads, int64_t con
   if ((e = cudaEventRecord(f->ready, s)) != cudaSuccess) return fail(e);
   if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return fail(e);
   f->host_ranks.assign(host_ranks, host_ranks + (size_t)P * nb);
+  f->host_ranks_valid = true;
   *out = f;
   return MILO_OK;
 }
@@ -348,11 +359,11 @@ static milo_status decode_impl(const void* q, int32_t batch, int32_t num_q_heads
   milo::DecodeShape ds{f->H, f->nb, f->n, f->d, batch, num_q_heads, suffix_len, f->dtype == MILO_BF16, sc};
   milo::DecodeBuffers db{q, K_suffix, V_suffix, f->ranks, f->row_offsets, f->tok, f->dim, nullptr, out, f->status};
   if (f->dtype == MILO_BF16 && milo::tc_supported(ds)) {
-    if (f->host_ranks.empty()) {
-      f->host_ranks.resize((size_t)2 * f->H * f->nb);
+    if (!f->host_ranks_valid) {
       MILO_CUDA(cudaStreamSynchronize(s));
       MILO_CUDA(cudaMemcpy(f->host_ranks.data(), f->ranks, f->host_ranks.size() * sizeof(int32_t),
                            cudaMemcpyDeviceToHost));
+      f->host_ranks_valid = true;
     }
     milo::TcInputs in{q,        K_suffix, V_suffix,     f->tok,       f->dim,
                       f->ranks, f->row_offsets, f->status, f->pool_rows, f->host_ranks.data()};
@@ -378,10 +389,6 @@ milo_status milo_decode_attn(const void* q, int32_t batch, int32_t num_q_heads, 
                      nullptr);
 }
 
-// Host staging of the ranks for milo_decode_attn_noalloc when the factor object has no host copy yet.
-static int32_t g_noalloc_ranks[1 << 16];
-static std::mutex g_noalloc_ranks_mu;
-
 milo_status milo_decode_attn_noalloc(const void* q, int32_t batch, int32_t num_q_heads, const milo_factors* fc,
                                      const void* K_suffix, const void* V_suffix, int32_t suffix_len, float scale,
                                      void* out, void* stream) {
@@ -394,22 +401,20 @@ milo_status milo_decode_attn_noalloc(const void* q, int32_t batch, int32_t num_q
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)f->d);
   milo::DecodeShape ds{f->H, f->nb, f->n, f->d, batch, num_q_heads, suffix_len, f->dtype == MILO_BF16, sc};
   if (f->dtype != MILO_BF16 || !milo::tc_supported(ds)) return MILO_ERR_UNSUPPORTED;
-  const size_t nranks = (size_t)2 * f->H * f->nb;
-  if (nranks > sizeof(g_noalloc_ranks) / sizeof(int32_t)) return MILO_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   std::lock_guard<std::mutex> lock(f->mu);
-  std::lock_guard<std::mutex> lock_r(g_noalloc_ranks_mu);
-  const int32_t* host_ranks = f->host_ranks.empty() ? nullptr : f->host_ranks.data();
-  if (!host_ranks) {
+  if (!f->host_ranks_valid) {
+    // the host copy was sized when the factor object was made: filling it allocates nothing
     MILO_CUDA(cudaEventSynchronize(f->ready));
-    MILO_CUDA(cudaMemcpy(g_noalloc_ranks, f->ranks, nranks * sizeof(int32_t), cudaMemcpyDeviceToHost));
-    host_ranks = g_noalloc_ranks;
+    MILO_CUDA(cudaMemcpy(f->host_ranks.data(), f->ranks, f->host_ranks.size() * sizeof(int32_t),
+                         cudaMemcpyDeviceToHost));
+    f->host_ranks_valid = true;
   }
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   MILO_CUDA(cudaStreamIsCapturing(s, &cap));
   if (cap == cudaStreamCaptureStatusNone) MILO_CUDA(cudaStreamWaitEvent(s, f->ready, 0));
   milo::TcInputs in{q,        K_suffix, V_suffix,     f->tok,       f->dim,
-                    f->ranks, f->row_offsets, f->status, f->pool_rows, host_ranks};
+                    f->ranks, f->row_offsets, f->status, f->pool_rows, f->host_ranks.data()};
   bool too_large = false;
   const cudaError_t e = milo::tc_decode_noalloc(ds, in, out, s, &too_large);
   if (too_large) return MILO_ERR_UNSUPPORTED;

@@ -101,7 +101,8 @@ typedef struct {
  * pool (clamped to [r_min, d], largest-remainder rounding), and the
  * projection U_b = X_b·B_b[:, :r_b].
  *   K, V        device [H][T][d] in `dtype`; read only.
- *   block_size  n: T % n == 0, n % 128 == 0, n >= d.
+ *   block_size  n: T % n == 0, n % 128 == 0, n >= d; at most 8192 blocks
+ *               (T / n) per pool, else MILO_ERR_UNSUPPORTED.
  *   head_dim    d ∈ {64, 128}.
  *   budget      storage budget > 0 (fraction of the raw cache; > 1 allowed).
  *   r_min       1 <= r_min <= d; MILO_ERR_BUDGET if R < nb*r_min.
@@ -159,10 +160,10 @@ milo_status milo_decode_attn_profiled(const void* q, int32_t batch, int32_t num_
  * milo_decode_attn_noalloc — milo_decode_attn for callers that cannot allocate
  * device memory.  The pages have no counterpart: it is a deployment variant.
  * Who needs it: code that runs where cudaMalloc is not allowed or not wanted —
- * while a stream is being captured in global mode (cudaMalloc is illegal there),
- * inside an engine whose allocator owns all device memory and forbids side
- * allocations, or on a latency-critical path that cannot afford the device-wide
- * synchronisation cudaMalloc implies.  milo_decode_attn allocates its work list
+ * inside a serving engine whose allocator owns all device memory and forbids
+ * side allocations (a cudaMalloc there can fail, or take memory the engine has
+ * promised elsewhere), or on a latency-critical path that cannot afford the
+ * device-wide synchronisation that cudaMalloc and cudaFree imply.  milo_decode_attn allocates its work list
  * and partials on the first call for a shape; this entry point allocates nothing
  * (no cudaMalloc, cudaFree, or allocating library routine) and keeps both in one
  * fixed array in device memory of MILO_NOALLOC_SCRATCH_BYTES (32 MiB) that every
@@ -174,8 +175,10 @@ milo_status milo_decode_attn_profiled(const void* q, int32_t batch, int32_t num_
  *   exceed the array returns MILO_ERR_UNSUPPORTED before anything is launched.
  *   Set-up: the first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current); make that first call
- *   before any stream capture.  If the factor object has never been decoded,
- *   the call synchronises once on the factors to read their ranks.
+ *   before any stream capture.  The first decode call of a factor object
+ *   (through this entry point or milo_decode_attn) synchronises once on the
+ *   factors to read their ranks into a host copy that was sized when the
+ *   object was made; later calls neither synchronise nor allocate for it.
  *   Sharing: every call on a device uses the same array and leaves its contents
  *   behind; each call writes every scratch word it reads, so nothing has to
  *   start at zero, but calls that overlap on the GPU (different streams, or

@@ -49,6 +49,7 @@ def _compress(lib, **kw):
     (dict(T=32769), 1), (dict(n=100), 1), (dict(n=64), 1), (dict(r_min=0), 1), (dict(r_min=129), 1),
     (dict(budget=0.0), 1), (dict(budget=float("nan")), 1), (dict(sweeps=-1), 1), (dict(flags=8), 1),
     (dict(budget=0.001), 3),
+    (dict(T=8193 * 512, H=1), 2),  # more blocks per pool than the allocation step holds in shared memory
 ])
 def test_compress_rejects_bad_arguments(kw, code):
     assert _compress(milo.load_library(), **kw) == code
@@ -102,3 +103,39 @@ def test_host_only_calls_reject_bad_arguments():
     assert call(S=-1) == 1
     assert call(n=384 + 64) == 2   # block size not a multiple of 128
     assert call(cap=4) == 2        # output too small
+
+
+def test_python_decode_checks_shapes_before_the_library():
+    """The binding rejects a q, out or suffix whose shape or dtype does not match the factors (the C ABI takes
+    no q shape or dtype beyond batch and heads) before any library call."""
+    import torch
+
+    class FakeFactors(milo.Factors):
+        def __init__(self):
+            super().__init__(None)
+            self._shape = (4, 128, milo.BF16)  # 4 KV heads, d = 128, bf16
+
+        def close(self):
+            pass
+
+    f = FakeFactors()
+    bf = torch.bfloat16
+    good_q = torch.zeros(2, 28, 128, dtype=bf)
+    bad = [
+        dict(q=torch.zeros(2, 28, 64, dtype=bf)),                       # head dim
+        dict(q=torch.zeros(2, 27, 128, dtype=bf)),                      # q heads not a multiple of 4
+        dict(q=torch.zeros(2, 28, 128, dtype=torch.float32)),           # dtype
+        dict(q=torch.zeros(28, 128, dtype=bf)),                         # rank
+        dict(out=torch.zeros(2, 28, 64, dtype=bf)),                     # out shape
+        dict(out=torch.zeros(2, 28, 128, dtype=torch.float32)),         # out dtype
+        dict(K_suf=torch.zeros(2, 4, 8, 128, dtype=bf)),                # V_suf missing
+        dict(K_suf=torch.zeros(2, 4, 8, 128, dtype=bf), V_suf=torch.zeros(2, 4, 9, 128, dtype=bf)),
+        dict(K_suf=torch.zeros(3, 4, 8, 128, dtype=bf), V_suf=torch.zeros(3, 4, 8, 128, dtype=bf)),
+        dict(K_suf=torch.zeros(2, 4, 8, 64, dtype=bf), V_suf=torch.zeros(2, 4, 8, 64, dtype=bf)),
+    ]
+    for kw in bad:
+        args = dict(q=good_q, K_suf=None, V_suf=None, out=None)
+        args.update(kw)
+        for fn in (milo.decode_attn, milo.decode_attn_noalloc):
+            with pytest.raises(ValueError):
+                fn(args["q"], f, args["K_suf"], args["V_suf"], out=args["out"])

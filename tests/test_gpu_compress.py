@@ -14,7 +14,7 @@ import numpy as np
 import pytest
 
 import oracle
-from milo_testutil import factor_arrays, from_torch, rel_l2, to_torch, untok_slabs
+from milo_testutil import assert_close, factor_arrays, from_torch, to_torch, untok_slabs
 from synth import WORKLOADS, from_storage, gen_layer
 
 pytestmark = pytest.mark.gpu
@@ -30,7 +30,7 @@ def delta(wl):
 E2E_TOL = {"f32": 1e-4, "bf16": 2e-2}
 
 
-@functools.lru_cache(maxsize=4)
+@functools.lru_cache(maxsize=3)
 def _inputs_and_oracle(name, beta, layer):
     """Tie-free generator inputs and the oracle's compression of them (cached across tests)."""
     wl = WORKLOADS[name]
@@ -39,15 +39,16 @@ def _inputs_and_oracle(name, beta, layer):
     dt = wl.dtype
     K, V = from_storage(L["K"], dt), from_storage(L["V"], dt)
     ref = oracle.compress_layer(K, V, wl.block_size, beta, wl.r_min)
-    return L, K, V, ref
+    return L, ref
 
 
 def _compress_both(name, beta=None, layer=0, keep=True):
     import decode_attention_milo_b200 as milo
     wl = WORKLOADS[name]
     beta = wl.budgets[0] if beta is None else beta
-    L, K, V, ref = _inputs_and_oracle(name, beta, layer)
+    L, ref = _inputs_and_oracle(name, beta, layer)
     dt = wl.dtype
+    K, V = from_storage(L["K"], dt), from_storage(L["V"], dt)
     f = milo.compress(to_torch(L["K"], dt), to_torch(L["V"], dt), wl.block_size, beta, wl.r_min,
                       keep_intermediates=keep)
     return wl, dt, L, K, V, ref, f
@@ -121,7 +122,7 @@ def test_end_to_end_decode(name):
                                       to_torch(L["V_suf"], dt) if S else None))
     want = oracle.decode_attention(from_storage(L["q"], dt), ref, from_storage(L["K_suf"], dt),
                                    from_storage(L["V_suf"], dt))
-    assert rel_l2(out, want) <= E2E_TOL[dt]
+    assert_close(out, want, E2E_TOL[dt], f"{name} end to end")
 
 
 def test_full_rank_budget_reproduces_attention_7b():
@@ -137,7 +138,7 @@ def test_full_rank_budget_reproduces_attention_7b():
     out = from_torch(milo.decode_attn(to_torch(q, dt), f, to_torch(Ks, dt), to_torch(Vs, dt)))
     want = oracle.decode_attention_dense(from_storage(q, dt), from_storage(L["K"], dt), from_storage(L["V"], dt),
                                          from_storage(Ks, dt), from_storage(Vs, dt))
-    assert rel_l2(out, want) <= E2E_TOL[dt]
+    assert_close(out, want, E2E_TOL[dt], "full rank vs dense attention")
 
 
 def test_sweep_limit_reports_no_convergence():
@@ -150,15 +151,37 @@ def test_sweep_limit_reports_no_convergence():
     assert code == 4 and bits & 1
 
 
-@pytest.mark.parametrize("name,beta", [("qwen2.5-7b-stack", 0.5), ("qwen2.5-32b-stack", 0.25),
-                                       ("qwen2.5-32b-stack", 0.75)])
-def test_stack_layer_ranks_bit_exact(name, beta):
-    """One full layer of the stacked workloads (each layer is an independent call)."""
+STACK_CASES = [("qwen2.5-7b-stack", 0.5), ("qwen2.5-32b-stack", 0.25), ("qwen2.5-32b-stack", 0.5),
+               ("qwen2.5-32b-stack", 0.75)]
+
+
+def _tile_sample(wl):
+    """Queries at the first and last item of every row tile of the decode (128 // G queries per tile)."""
+    ipt = min(wl.batch, 128 // wl.group)
+    s = set()
+    for t0 in range(0, wl.batch, ipt):
+        s |= {t0, min(wl.batch, t0 + ipt) - 1}
+    return sorted(s)
+
+
+@pytest.mark.parametrize("name,beta", STACK_CASES)
+def test_stack_layer_ranks_and_end_to_end(name, beta):
+    """One full layer of a stacked workload (each layer is an independent call): ranks bit-exact, then GPU
+    decode of the whole batch and suffix on the GPU's own factors against the oracle's fp64 pipeline, on
+    queries that span every row tile."""
+    import decode_attention_milo_b200 as milo
     wl, dt, L, K, V, ref, f = _compress_both(name, beta=beta, layer=1, keep=True)
     assert f.status()[0] == 0
     pools = _ref_pools(ref)
     qerr = np.abs(factor_arrays(f)["quotas"] - np.array([p["quotas"] for p in pools])).max()
     print(f"{name} beta={beta}: max |quota_gpu - quota_oracle| = {qerr:.2e}")
     assert qerr < delta(wl) / 2
-    want = np.array([p["ranks"] for p in pools])
-    assert np.array_equal(f.ranks(), want)
+    want_ranks = np.array([p["ranks"] for p in pools])
+    assert np.array_equal(f.ranks(), want_ranks)
+    out = from_torch(milo.decode_attn(to_torch(L["q"], dt), f, to_torch(L["K_suf"], dt),
+                                      to_torch(L["V_suf"], dt)))
+    assert f.status()[0] == 0
+    idx = _tile_sample(wl)
+    want = oracle.decode_attention(from_storage(L["q"][idx], dt), ref, from_storage(L["K_suf"][idx], dt),
+                                   from_storage(L["V_suf"][idx], dt))
+    assert_close(out[idx], want, E2E_TOL[dt], f"{name} beta {beta} end to end")
