@@ -15,13 +15,17 @@ Every function states the passage it follows and the reading taken where the
 page is silent.
 """
 from .milo import (  # noqa: F401
+    ALLOC_RULES,
+    POOL_SCOPES,
     BudgetError,
+    allocate_blocks,
     allocate_ranks,
     allocate_ranks_greedy,
     allocate_ranks_random,
     allocate_ranks_uniform,
     block_svd,
     compress_layer,
+    compress_layer_rule,
     compress_pool,
     decode_attention,
     decode_attention_dense,

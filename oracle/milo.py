@@ -210,6 +210,88 @@ def compress_layer(K: np.ndarray, V: np.ndarray, n: int, beta: float, r_min: int
                 V=[compress_pool(V[h], n, beta, r_min) for h in range(H)])
 
 
+ALLOC_RULES = ("entropy", "greedy", "uniform", "weights")
+POOL_SCOPES = ("pool", "layer")
+
+
+def allocate_blocks(rule: str, sigma, R: int, r_min: int, d: int, weights=None):
+    """Ranks of a set of blocks under one allocation rule, summing to R.
+
+    The rules are the entropy rule of §4.3 (ranks ∝ exp(H_b), water-filling and largest
+    remainder), the greedy marginal-gain form §4.3 describes in words, and the two baselines
+    §5.3 compares against: uniform, and random (ranks ∝ weights drawn by the caller, passed
+    in as `weights`, with the entropy rule's water-filling).  sigma: [nb][d] singular values.
+
+    Returns (ranks int64[nb], quotas float64[nb] or None for the rules without quotas).
+    """
+    sigma = np.asarray(sigma, dtype=np.float64)
+    nb = sigma.shape[0]
+    if rule == "entropy":
+        w = np.exp([spectral_entropy(s) for s in sigma])
+        r, q, _ = allocate_ranks(w, R, r_min, d)
+        return r, q
+    if rule == "weights":
+        r, q, _ = allocate_ranks(np.asarray(weights, dtype=np.float64), R, r_min, d)
+        return r, q
+    if rule == "greedy":
+        return allocate_ranks_greedy(sigma, R, r_min, d), None
+    if rule == "uniform":
+        return allocate_ranks_uniform(nb, R, r_min, d), None
+    raise ValueError(rule)
+
+
+def compress_layer_rule(K: np.ndarray, V: np.ndarray, n: int, beta: float, r_min: int, rule: str = "entropy",
+                        scope: str = "pool", weights=None) -> dict:
+    """Compress one layer with a chosen allocation rule and budget scope.
+
+    scope "pool": each (KV head, K|V) pool gets R = floor(beta·T·d/(n+d)) rank units
+    (compress_layer with the entropy rule).  scope "layer": the layer's pools share one
+    budget, P·R units over all P·nb blocks (the "global rank budget" of §4.3 taken over the
+    layer), with the blocks in the order pool p = 2h + t (t = 0 keys, 1 values), then block.
+    weights: [P][nb] for rule "weights".  Factors are computed as in compress_pool.
+    Returns compress_layer's structure; each pool also carries its own rank sum as "R", and
+    the layer dict carries "R_total".
+    """
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    H, T, d = K.shape
+    if T % n:
+        raise ValueError("context length must be a multiple of the block size")
+    nb = T // n
+    P = 2 * H
+    xs = [(K if p % 2 == 0 else V)[p // 2] for p in range(P)]
+    svd = [[block_svd(x[b * n:(b + 1) * n]) for b in range(nb)] for x in xs]
+    sig = np.array([[s for s, _ in pool] for pool in svd])  # [P][nb][d]
+    R = rank_total(beta, T, n, d)
+    w = None if weights is None else np.asarray(weights, dtype=np.float64).reshape(P, nb)
+    ranks = np.zeros((P, nb), dtype=np.int64)
+    quotas = np.full((P, nb), np.nan)
+    if scope == "pool":
+        for p in range(P):
+            r, q = allocate_blocks(rule, sig[p], R, r_min, d, None if w is None else w[p])
+            ranks[p] = r
+            if q is not None:
+                quotas[p] = q
+    elif scope == "layer":
+        r, q = allocate_blocks(rule, sig.reshape(P * nb, -1), P * R, r_min, d, None if w is None else w.ravel())
+        ranks[:] = r.reshape(P, nb)
+        if q is not None:
+            quotas[:] = q.reshape(P, nb)
+    else:
+        raise ValueError(scope)
+    pools = []
+    for p in range(P):
+        U, B = [], []
+        for b in range(nb):
+            br = svd[p][b][1][:, :int(ranks[p, b])]
+            U.append(xs[p][b * n:(b + 1) * n] @ br)
+            B.append(br)
+        ent = np.array([spectral_entropy(s) for s in sig[p]])
+        pools.append(dict(sigma=sig[p], entropy=ent, weights=np.exp(ent), R=int(ranks[p].sum()), quotas=quotas[p],
+                          ranks=ranks[p], U=U, B=B, n=n, d=d))
+    return dict(K=pools[0::2], V=pools[1::2], R_total=int(ranks.sum()))
+
+
 def reconstruct_pool(pool: dict) -> np.ndarray:
     """Dense [T][d] reconstruction Σ_b U_b · B_bᵀ stacked over blocks."""
     return np.concatenate([u @ b.T for u, b in zip(pool["U"], pool["B"])], axis=0)

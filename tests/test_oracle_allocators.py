@@ -116,3 +116,89 @@ def test_greedy_cut_gap_predicts_stability():
         sig2 = np.sqrt(np.maximum(s2, 0) * e.sum(axis=1, keepdims=True))
         assert np.array_equal(oracle.allocate_ranks_greedy(sig2, R, r_min, d), r)
     assert oracle.greedy_cut_gap(sigma, nb * r_min, r_min, d) == float("inf")
+
+
+# ---------------------------------------------------------------- rules and budget scope of a whole layer
+
+def _tiny_layer(scale_v=1.0):
+    from synth import from_storage, gen_layer
+    wl = WORKLOADS["tiny"]
+    L = gen_layer(wl)
+    return wl, from_storage(L["K"], wl.dtype), from_storage(L["V"], wl.dtype) * scale_v
+
+
+def test_layer_scope_worked_example():
+    """Hand-derived: 2 pools x 2 blocks, d = 8, r_min = 1, weights [1, 2 | 3, 2].
+    Layer budget 12: lam = 12 / 8 = 1.5, quotas [1.5, 3, 4.5, 3], floors sum 11, the one extra unit goes to
+    the largest fractional part (0.5, a tie between blocks 0 and 2, to the lower index): [2, 3 | 4, 3].
+    Per pool, 6 each: pool 0 lam = 2, quotas [2, 4]; pool 1 lam = 1.2, quotas [3.6, 2.4], floors 5, the
+    extra unit to fraction 0.6: [2, 4 | 4, 2]."""
+    sig = np.ones((4, 8))
+    r, q = oracle.allocate_blocks("weights", sig, 12, 1, 8, weights=[1, 2, 3, 2])
+    assert list(r) == [2, 3, 4, 3] and np.allclose(q, [1.5, 3, 4.5, 3])
+    r0, _ = oracle.allocate_blocks("weights", sig[:2], 6, 1, 8, weights=[1, 2])
+    r1, _ = oracle.allocate_blocks("weights", sig[2:], 6, 1, 8, weights=[3, 2])
+    assert list(r0) + list(r1) == [2, 4, 4, 2]
+
+
+def test_pool_scope_entropy_is_compress_layer():
+    wl, K, V = _tiny_layer()
+    a = oracle.compress_layer(K, V, wl.block_size, 0.5, wl.r_min)
+    b = oracle.compress_layer_rule(K, V, wl.block_size, 0.5, wl.r_min, "entropy", "pool")
+    for t in ("K", "V"):
+        for pa, pb in zip(a[t], b[t]):
+            assert np.array_equal(pa["ranks"], pb["ranks"])
+            assert np.allclose(pa["quotas"], pb["quotas"], rtol=0, atol=1e-12)
+            for ua, ub in zip(pa["U"], pb["U"]):
+                assert np.array_equal(ua, ub)
+
+
+@pytest.mark.parametrize("rule", ["entropy", "greedy", "uniform"])
+def test_layer_scope_invariants(rule):
+    wl, K, V = _tiny_layer()
+    n, d, T = wl.block_size, wl.head_dim, wl.context
+    R = oracle.rank_total(0.5, T, n, d)
+    lay = oracle.compress_layer_rule(K, V, n, 0.5, wl.r_min, rule, "layer")
+    ranks = np.array([p["ranks"] for t in ("K", "V") for p in lay[t]])
+    assert lay["R_total"] == ranks.sum() == 2 * wl.kv_heads * R
+    assert ranks.min() >= wl.r_min and ranks.max() <= d
+    if rule != "uniform":  # entropy and energy shares do not change when a pool is scaled
+        lay2 = oracle.compress_layer_rule(K * 3.0, V, n, 0.5, wl.r_min, rule, "layer")
+        ranks2 = np.array([p["ranks"] for t in ("K", "V") for p in lay2[t]])
+        assert np.array_equal(ranks, ranks2)
+    else:
+        P, nb = ranks.shape
+        want = np.full(P * nb, (P * R) // (P * nb))
+        want[: (P * R) % (P * nb)] += 1
+        assert np.array_equal(ranks.ravel(), want)
+
+
+@pytest.mark.parametrize("rule", ["entropy", "greedy"])
+def test_layer_scope_with_identical_pools_matches_pool_scope(rule):
+    """When every pool holds the same data, sharing the budget over the layer changes nothing: the quotas
+    (or shares) repeat per pool, and the tie-break by index hands each repeated unit to every pool alike."""
+    wl, K, _ = _tiny_layer()
+    n = wl.block_size
+    a = oracle.compress_layer_rule(K, K, n, 0.5, wl.r_min, rule, "pool")
+    b = oracle.compress_layer_rule(K, K, n, 0.5, wl.r_min, rule, "layer")
+    for t in ("K", "V"):
+        for pa, pb in zip(a[t], b[t]):
+            assert np.array_equal(pa["ranks"], pb["ranks"])
+
+
+def test_layer_scope_greedy_is_optimal_by_brute_force():
+    """Over a layer the greedy still maximises the captured energy shares (brute force, 2 pools x 2 blocks)."""
+    rng = np.random.default_rng(7)
+    d, r_min = 5, 1
+    sigma = np.sort(rng.exponential(1.0, size=(4, d)) ** 2.0, axis=1)[:, ::-1]
+    for R in range(5, 4 * d):
+        got, _ = oracle.allocate_blocks("greedy", sigma, R, r_min, d)
+        best = max(_captured(sigma, r) for r in itertools.product(range(r_min, d + 1), repeat=4) if sum(r) == R)
+        assert got.sum() == R
+        assert _captured(sigma, got) == pytest.approx(best, rel=1e-12)
+
+
+def test_weights_rule_with_equal_weights_is_uniform():
+    sig = np.ones((64, 128))
+    r, _ = oracle.allocate_blocks("weights", sig, 3276, 4, 128, weights=np.full(64, 9.0))
+    assert np.array_equal(r, oracle.allocate_ranks_uniform(64, 3276, 4, 128))
