@@ -241,7 +241,7 @@ def allocate_blocks(rule: str, sigma, R: int, r_min: int, d: int, weights=None):
 
 
 def compress_layer_rule(K: np.ndarray, V: np.ndarray, n: int, beta: float, r_min: int, rule: str = "entropy",
-                        scope: str = "pool", weights=None) -> dict:
+                        scope: str = "pool", weights=None, ranks=None) -> dict:
     """Compress one layer with a chosen allocation rule and budget scope.
 
     scope "pool": each (KV head, K|V) pool gets R = floor(beta·T·d/(n+d)) rank units
@@ -249,6 +249,8 @@ def compress_layer_rule(K: np.ndarray, V: np.ndarray, n: int, beta: float, r_min
     budget, P·R units over all P·nb blocks (the "global rank budget" of §4.3 taken over the
     layer), with the blocks in the order pool p = 2h + t (t = 0 keys, 1 values), then block.
     weights: [P][nb] for rule "weights".  Factors are computed as in compress_pool.
+    ranks: optional [P][nb] integers that replace the allocation (factors at given ranks, to
+    compare outputs once the integer decisions have been compared on their own).
     Returns compress_layer's structure; each pool also carries its own rank sum as "R", and
     the layer dict carries "R_total".
     """
@@ -264,9 +266,12 @@ def compress_layer_rule(K: np.ndarray, V: np.ndarray, n: int, beta: float, r_min
     sig = np.array([[s for s, _ in pool] for pool in svd])  # [P][nb][d]
     R = rank_total(beta, T, n, d)
     w = None if weights is None else np.asarray(weights, dtype=np.float64).reshape(P, nb)
+    given = ranks
     ranks = np.zeros((P, nb), dtype=np.int64)
     quotas = np.full((P, nb), np.nan)
-    if scope == "pool":
+    if given is not None:
+        ranks[:] = np.asarray(given, dtype=np.int64).reshape(P, nb)
+    elif scope == "pool":
         for p in range(P):
             r, q = allocate_blocks(rule, sig[p], R, r_min, d, None if w is None else w[p])
             ranks[p] = r
@@ -308,15 +313,21 @@ def stored_factors(pool: dict, cast) -> dict:
 # ---------------------------------------------------------------- decode
 
 def decode_attention(q: np.ndarray, layer: dict, K_suf: np.ndarray, V_suf: np.ndarray,
-                     scale: float | None = None) -> np.ndarray:
+                     scale: float | None = None, block_mask=None) -> np.ndarray:
     """Softmax decode attention over the compressed prefix and the per-query suffix, in rank space.
 
     §4.4 inference attends over the low-rank caches.  With K_b ≈ U_b·B_bᵀ the
     scores of block b are (q · B_b) · U_bᵀ and with V_b ≈ P_b·Q_bᵀ the block's
     value sum is (p · P_b) · Q_bᵀ, so no block is expanded to n×d.
-    Readings: every block is attended (no selection); scale = 1/sqrt(d); no
-    RoPE; query head hq reads KV head hq // (Hq / H); the prefix is shared by
-    every query and one softmax runs over prefix ∪ that query's suffix.
+    Readings: every block is attended unless block_mask says otherwise;
+    scale = 1/sqrt(d); no RoPE; query head hq reads KV head hq // (Hq / H); the
+    prefix is shared by every query and one softmax runs over prefix ∪ that
+    query's suffix.
+
+    Block selection (§4.4: decoding retrieves the selected blocks and attends
+    sparsely): block_mask [H][nb] of booleans, True = attended; the blocks of a
+    KV head that are not selected take no part in that head's softmax, for
+    every query.  None selects every block.
 
     q [Bq][Hq][d]; layer = compress_layer(...) output (possibly with stored
     factors); K_suf, V_suf [Bq][H][S][d] (S may be 0).  Returns [Bq][Hq][d].
@@ -329,6 +340,10 @@ def decode_attention(q: np.ndarray, layer: dict, K_suf: np.ndarray, V_suf: np.nd
     out = np.zeros((Bq, Hq, d))
     for h in range(H):
         kp, vp = layer["K"][h], layer["V"][h]
+        if block_mask is not None:
+            keep = [b for b in range(len(kp["U"])) if block_mask[h][b]]
+            kp = dict(U=[kp["U"][b] for b in keep], B=[kp["B"][b] for b in keep])
+            vp = dict(U=[vp["U"][b] for b in keep], B=[vp["B"][b] for b in keep])
         for i in range(Bq):
             for g in range(G):
                 hq = h * G + g

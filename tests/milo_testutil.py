@@ -105,18 +105,18 @@ def factor_arrays(f) -> dict:
     """Host copies of a factor object's arrays, as fp64 / int numpy arrays."""
     import torch
     d = f.describe()
-    H2, nb, n, dd, rows = 2 * d["num_kv_heads"], d["num_blocks"], d["block_size"], d["head_dim"], d["pool_rows"]
+    H2, nb, n, dd, total = 2 * d["num_kv_heads"], d["num_blocks"], d["block_size"], d["head_dim"], d["total_rows"]
     bf = d["dtype"] == 1
     out = dict(desc=d)
     out["ranks"] = device_view(d["ranks"], (H2, nb), "<i4").cpu().numpy()
     out["row_offsets"] = device_view(d["row_offsets"], (H2, nb + 1), "<i8").cpu().numpy()
     if bf:
-        tok = device_view(d["tok"], (H2 * rows * n,), "<i2").cpu().numpy().view(np.uint16)
-        dim = device_view(d["dim"], (H2 * rows, dd), "<i2").cpu().numpy().view(np.uint16)
+        tok = device_view(d["tok"], (total * n,), "<i2").cpu().numpy().view(np.uint16)
+        dim = device_view(d["dim"], (total, dd), "<i2").cpu().numpy().view(np.uint16)
         out["tok"], out["dim"] = from_storage(tok, "bf16"), from_storage(dim, "bf16")
     else:
-        out["tok"] = device_view(d["tok"], (H2 * rows * n,), "<f4").cpu().numpy().astype(np.float64)
-        out["dim"] = device_view(d["dim"], (H2 * rows, dd), "<f4").cpu().numpy().astype(np.float64)
+        out["tok"] = device_view(d["tok"], (total * n,), "<f4").cpu().numpy().astype(np.float64)
+        out["dim"] = device_view(d["dim"], (total, dd), "<f4").cpu().numpy().astype(np.float64)
     if d["eigvals"]:
         out["eigvals"] = device_view(d["eigvals"], (H2, nb, dd), "<f4").cpu().numpy().astype(np.float64)
         out["entropy"] = device_view(d["entropy"], (H2, nb), "<f8").cpu().numpy()

@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol():
     assert {"milo_compress", "milo_decode_attn"} <= names
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.milo_abi_version() == 1
+    assert lib.milo_abi_version() == 2
     assert lib.milo_status_string(0) == b"ok"
     assert lib.milo_status_string(3).startswith(b"budget")
 
@@ -55,6 +55,36 @@ def test_compress_rejects_bad_arguments(kw, code):
     assert _compress(milo.load_library(), **kw) == code
 
 
+def _compress_rule(lib, rule=0, scope=0, weights=None, **kw):
+    args = dict(K=1, V=1, dtype=1, H=4, T=32768, d=128, n=512, budget=0.5, r_min=4)
+    args.update(kw)
+    out = ctypes.c_void_p(123)
+    w = None if weights is None else weights.ctypes.data_as(ctypes.c_void_p)
+    code = lib.milo_compress_rule(ctypes.c_void_p(args["K"]), ctypes.c_void_p(args["V"]), args["dtype"], args["H"],
+                                  args["T"], args["d"], args["n"], args["budget"], args["r_min"], 0, 0, rule, scope,
+                                  w, None, ctypes.byref(out))
+    assert out.value is None
+    return code
+
+
+def test_compress_rule_rejects_bad_arguments():
+    import numpy as np
+    lib = milo.load_library()
+    w = np.ones(2 * 4 * 64)
+    assert _compress_rule(lib, rule=4) == 1                      # unknown rule
+    assert _compress_rule(lib, scope=2) == 1                     # unknown scope
+    assert _compress_rule(lib, rule=3) == 1                      # weights rule without weights
+    assert _compress_rule(lib, rule=0, weights=w) == 1           # weights given to another rule
+    bad = w.copy()
+    bad[5] = 0.0
+    assert _compress_rule(lib, rule=3, weights=bad) == 1         # weights must be > 0
+    bad[5] = float("nan")
+    assert _compress_rule(lib, rule=3, weights=bad) == 1
+    # a layer-wide budget allocates over all 2H·nb blocks at once: 16 heads x 2 x 512 blocks is too many
+    assert _compress_rule(lib, scope=1, H=16, T=512 * 512) == 2
+    assert _compress_rule(lib, rule=1, budget=0.001) == 3
+
+
 def test_decode_rejects_null_arguments():
     lib = milo.load_library()
     assert lib.milo_decode_attn(None, 1, 2, None, None, None, 0, 0.0, None, None) == 1
@@ -63,16 +93,17 @@ def test_decode_rejects_null_arguments():
     lib.milo_factors_destroy(None)
 
 
-def test_import_rejects_unequal_pools():
+def test_import_rejects_ranks_out_of_range():
     import numpy as np
     lib = milo.load_library()
-    ranks = np.array([[4, 5], [4, 4]], dtype=np.int32)  # pool sums differ
     tok = np.zeros(64 * 512, dtype=np.uint16)
-    out = ctypes.c_void_p()
-    code = lib.milo_factors_import(1, 1, 1024, 64, 512, 4, ranks.ctypes.data_as(ctypes.c_void_p),
-                                   tok.ctypes.data_as(ctypes.c_void_p), tok.ctypes.data_as(ctypes.c_void_p),
-                                   None, ctypes.byref(out))
-    assert code == 1
+    for bad in (0, 65):
+        ranks = np.array([[4, bad], [4, 4]], dtype=np.int32)
+        out = ctypes.c_void_p()
+        code = lib.milo_factors_import(1, 1, 1024, 64, 512, 4, ranks.ctypes.data_as(ctypes.c_void_p),
+                                       tok.ctypes.data_as(ctypes.c_void_p), tok.ctypes.data_as(ctypes.c_void_p),
+                                       None, ctypes.byref(out))
+        assert code == 1
 
 
 def test_every_status_code_has_a_string():

@@ -144,3 +144,40 @@ def test_scale_argument():
     c = oracle.decode_attention(q, lay, Ks, Vs, scale=0.5)
     assert np.array_equal(a, b)
     assert not np.allclose(b, c)
+
+
+# ---------------------------------------------------------------- block selection (§4.4: selected blocks only)
+
+def test_block_selection_equals_attention_over_the_selected_blocks():
+    """Selecting blocks {0, 2} of four equals brute-force softmax over those blocks' reconstructed rows and
+    the suffix; selecting every block equals the unmasked decode."""
+    wl, K, V, q, Ks, Vs = _tiny_inputs(suffix=12, batch=2)
+    lay = oracle.compress_layer(K, V, wl.block_size, 0.5, wl.r_min)
+    n = wl.block_size
+    Kr = oracle.reconstruct_pool(lay["K"][0])
+    Vr = oracle.reconstruct_pool(lay["V"][0])
+    mask = [[True, False, True, False]]
+    rows = np.concatenate([np.arange(b * n, (b + 1) * n) for b in (0, 2)])
+    got = oracle.decode_attention(q, lay, Ks, Vs, block_mask=mask)
+    want = _brute_force(q, Kr[rows][None], Vr[rows][None], Ks, Vs, 1.0 / 8.0)
+    assert np.allclose(got, want, rtol=1e-11, atol=1e-15)
+    every = oracle.decode_attention(q, lay, Ks, Vs, block_mask=[[True] * 4])
+    assert np.array_equal(every, oracle.decode_attention(q, lay, Ks, Vs))
+
+
+def test_block_selection_full_rank_is_exact_attention_on_the_selected_rows():
+    wl, K, V, q, Ks, Vs = _tiny_inputs(suffix=8)
+    beta = (wl.block_size + wl.head_dim) / wl.block_size
+    lay = oracle.compress_layer(K, V, wl.block_size, beta, wl.r_min)
+    n = wl.block_size
+    got = oracle.decode_attention(q, lay, Ks, Vs, block_mask=[[False, True, False, False]])
+    want = _sdpa(q, K[:, n:2 * n], V[:, n:2 * n], Ks, Vs, 1.0 / 8.0)
+    assert np.allclose(got, want, rtol=1e-10, atol=1e-14)
+
+
+def test_no_block_selected_leaves_the_suffix():
+    wl, K, V, q, Ks, Vs = _tiny_inputs(suffix=5)
+    lay = oracle.compress_layer(K, V, wl.block_size, 0.5, wl.r_min)
+    got = oracle.decode_attention(q, lay, Ks, Vs, block_mask=[[False] * 4])
+    want = _sdpa(q, K[:, :0], V[:, :0], Ks, Vs, 1.0 / 8.0)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-15)
