@@ -33,9 +33,17 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "compressed-KV decode tokens/s at Qwen2.5-7B shape; achieved HBM GB/s vs peak"
-# DRAM bytes read + written by one decode_tc_kernel launch on qwen2.5-7b-layer, from the ncu capture summarised
-# under profiles/ (decode_tc_kernel_qwen2.5-7b-layer); reset to None whenever the kernel changes.
-DECODE_TRAFFIC = {"qwen2.5-7b-layer": 42166528 + 42752}
+# DRAM bytes (read + written) of one launch of the main decode kernel, measured with ncu, per workload, keyed by
+# the SHA-256 prefix of the kernel's source file at the time of the capture.  A different digest means the
+# kernel has changed since the counters were taken, and the line reports traffic as null.
+DECODE_TRAFFIC = {}
+
+
+def _source_digest() -> str:
+    import hashlib
+    path = os.path.join(ROOT, "decode_attention_milo_b200", "csrc", "decode_tc.cu")
+    with open(path, "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:12]
 
 
 def _args():
@@ -170,6 +178,56 @@ def _to_dev(a, dt, torch):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
 
 
+def _device_ints(torch, ptr, n):
+    """Host copy of n int32 values at a library-owned device address."""
+    class _A:
+        __cuda_array_interface__ = {"shape": (n,), "typestr": "<i4", "data": (int(ptr), False), "version": 3,
+                                    "strides": None}
+    return torch.as_tensor(_A(), device="cuda").cpu().numpy()
+
+
+def _fp32_peak_tflops(torch):
+    """FP32 FMA peak from the unit counts: SMs x 128 FP32 lanes x 2 flops x max SM clock."""
+    props = torch.cuda.get_device_properties(0)
+    mhz = None
+    try:
+        import pynvml as nv
+        nv.nvmlInit()
+        mhz = nv.nvmlDeviceGetMaxClockInfo(nv.nvmlDeviceGetHandleByIndex(torch.cuda.current_device()),
+                                           nv.NVML_CLOCK_SM)
+    except Exception:
+        mhz = 1965
+    return props.multi_processor_count * 128 * 2 * mhz * 1e6 / 1e12, mhz
+
+
+def _compress_roofline(torch, wl, esize, ranks, sweeps, kern, peak_gbs):
+    """Per-kernel fraction of roofline for one whole-layer compression (median CUDA-event times)."""
+    H, T, d, n, nb = wl.kv_heads, wl.context, wl.head_dim, wl.block_size, wl.num_blocks
+    nblk = 2 * H * nb
+    x_bytes = 2 * H * T * d * esize                          # K and V, read once
+    gram_bytes = x_bytes + nblk * d * d * 4                  # + the fp32 Gram matrices written
+    rsum = int(ranks.sum())
+    proj_bytes = x_bytes + rsum * d * 4 + rsum * (n + d) * esize  # + eigenvectors used, factors written
+    pairs = d * (d - 1) // 2
+    jac_flops = float(np.sum(sweeps)) * pairs * 18 * d     # per pair: 3 dot products (6d) + 4 column updates (12d)
+    fp32_tf, mhz = _fp32_peak_tflops(torch)
+    med = {k: statistics.median(v) for k, v in kern.items()}
+
+    def hbm(bytes_, ms):
+        gbs = bytes_ / (ms / 1e3) / 1e9
+        return {"ms": ms, "bytes": bytes_, "achieved": gbs, "peak": peak_gbs, "unit": "GB/s", "frac": gbs / peak_gbs}
+    jt = jac_flops / (med["jacobi"] / 1e3) / 1e12
+    return {
+        "gram": dict(hbm(gram_bytes, med["gram"]), bound="hbm"),
+        "jacobi": {"bound": "alu", "ms": med["jacobi"], "flops": jac_flops, "achieved": jt, "peak": fp32_tf,
+                   "unit": "TFLOP/s", "frac": jt / fp32_tf, "sweeps_mean": float(np.mean(sweeps)),
+                   "sweeps_max": int(np.max(sweeps)),
+                   "peak_note": f"FP32 FMA: SMs x 128 lanes x 2 flops x {mhz} MHz; flops count full sweeps"},
+        "alloc": {"ms": med["alloc"]},
+        "project": dict(hbm(proj_bytes, med["project"]), bound="hbm"),
+    }
+
+
 def _algorithmic_bytes(ranks, wl, esize):
     """Bytes one decode step must move: factors at their ranks (read once, shared by the batch),
     the per-query suffix K and V, q and out."""
@@ -179,8 +237,75 @@ def _algorithmic_bytes(ranks, wl, esize):
     return factors + suffix + qo
 
 
+def _oracle_layer(wl, L):
+    """The oracle's compression of the workload's layer (fp64, stored factors as the decode reads them)."""
+    import oracle
+    from synth import from_storage
+    dt = wl.dtype
+    K, V = from_storage(L["K"], dt), from_storage(L["V"], dt)
+    return oracle.compress_layer(K, V, wl.block_size, wl.budgets[0], wl.r_min)
+
+
+def _save_layer(lay, path):
+    """Writes the oracle layer's per-pool factors to .npy files that worker processes map read-only."""
+    os.makedirs(path, exist_ok=True)
+    H = len(lay["K"])
+    for t in ("K", "V"):
+        for h in range(H):
+            pool = lay[t][h]
+            np.save(os.path.join(path, f"{t}{h}_ranks.npy"), np.asarray(pool["ranks"], dtype=np.int64))
+            np.save(os.path.join(path, f"{t}{h}_U.npy"), np.concatenate([u.T for u in pool["U"]], axis=0))
+            np.save(os.path.join(path, f"{t}{h}_B.npy"), np.concatenate([b.T for b in pool["B"]], axis=0))
+    return H
+
+
+def _load_layer(path, H):
+    lay = {"K": [], "V": []}
+    for t in ("K", "V"):
+        for h in range(H):
+            ranks = np.load(os.path.join(path, f"{t}{h}_ranks.npy"))
+            U = np.load(os.path.join(path, f"{t}{h}_U.npy"), mmap_mode="r")
+            B = np.load(os.path.join(path, f"{t}{h}_B.npy"), mmap_mode="r")
+            off = np.concatenate([[0], np.cumsum(ranks)])
+            lay[t].append({"U": [np.asarray(U[a:b]).T for a, b in zip(off[:-1], off[1:])],
+                           "B": [np.asarray(B[a:b]).T for a, b in zip(off[:-1], off[1:])]})
+    return lay
+
+
+def _cpu_worker(path, H, wl_name, k, seconds, ready, start, results):
+    """One host core: decodes single queries of the workload with the oracle until `seconds` elapse."""
+    try:
+        try:
+            from threadpoolctl import threadpool_limits
+            threadpool_limits(1)
+        except Exception:  # pragma: no cover
+            pass
+        import oracle
+        from synth import WORKLOADS
+        wl = WORKLOADS[wl_name]
+        lay = _load_layer(path, H)
+        q, Ks, Vs = (np.load(os.path.join(path, f"{x}.npy"), mmap_mode="r") for x in ("q", "K_suf", "V_suf"))
+    except Exception as exc:  # pragma: no cover - reported to the parent, which stops waiting
+        ready.put(("error", repr(exc)))
+        return
+    ready.put(("ready", k))
+    start.wait()
+    n = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        i = (k + n) % wl.batch
+        oracle.decode_attention(np.asarray(q[i:i + 1]), lay, np.asarray(Ks[i:i + 1]), np.asarray(Vs[i:i + 1]))
+        n += 1
+    results.put((k, n, time.perf_counter() - t0))
+
+
 def _cpu_baseline(wl, L, seconds):
-    """The fp64 oracle, as it stands, on this host: whole decode steps until `seconds` elapse."""
+    """The fp64 oracle, as it stands, on this host.  One core: whole decode steps of the batch until `seconds`
+    elapse.  All cores: one process per core (spawned), each decoding single queries for `seconds`."""
+    import multiprocessing as mp
+    import shutil
+    import tempfile
+
     import oracle
     from synth import from_storage
     try:
@@ -189,8 +314,7 @@ def _cpu_baseline(wl, L, seconds):
     except Exception:  # pragma: no cover
         limiter = None
     dt = wl.dtype
-    K, V = from_storage(L["K"], dt), from_storage(L["V"], dt)
-    lay = oracle.compress_layer(K, V, wl.block_size, wl.budgets[0], wl.r_min)
+    lay = _oracle_layer(wl, L)
     q = from_storage(L["q"], dt)
     Ks, Vs = from_storage(L["K_suf"], dt), from_storage(L["V_suf"], dt)
     steps = 0
@@ -201,11 +325,48 @@ def _cpu_baseline(wl, L, seconds):
         if time.perf_counter() - t0 >= seconds:
             break
     el = time.perf_counter() - t0
-    if limiter is not None:
-        limiter.unregister() if hasattr(limiter, "unregister") else None
-    return {"value": steps * wl.batch / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{steps} whole decode steps of {wl.name} (batch {wl.batch}) in {el:.1f} s, fp64 NumPy, "
-                      f"1 BLAS thread"}
+    one = {"value": steps * wl.batch / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+           "sample": f"{steps} whole decode steps of {wl.name} (batch {wl.batch}) in {el:.1f} s, fp64 NumPy, "
+                     f"1 BLAS thread"}
+    del limiter
+    cores = min(len(os.sched_getaffinity(0)), 64)
+    tmp = tempfile.mkdtemp(prefix="milo_oracle_")
+    try:
+        H = _save_layer(lay, tmp)
+        for x, a in (("q", q), ("K_suf", Ks), ("V_suf", Vs)):
+            np.save(os.path.join(tmp, f"{x}.npy"), a)
+        ctx = mp.get_context("spawn")
+        ready, results, start = ctx.Queue(), ctx.Queue(), ctx.Event()
+        procs = [ctx.Process(target=_cpu_worker, args=(tmp, H, wl.name, k, seconds, ready, start, results))
+                 for k in range(cores)]
+        for pr in procs:
+            pr.start()
+        try:
+            for _ in procs:
+                tag, what = ready.get(timeout=180)
+                if tag == "error":
+                    raise RuntimeError(f"oracle worker failed to start: {what}")
+        except BaseException:
+            for pr in procs:
+                pr.terminate()
+            raise
+        start.set()
+        got = [results.get(timeout=120 + 4 * seconds) for _ in procs]
+        for pr in procs:
+            pr.join(timeout=60)
+        done = sum(n for _, n, _ in got)
+        wall = max(t for _, _, t in got)
+        many = {"value": done / wall, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                "sample": f"{done} single-query decodes of {wl.name} over {cores} processes (one per core, spawned, "
+                          f"1 BLAS thread each) in {wall:.1f} s, fp64 NumPy"}
+    except Exception as exc:  # pragma: no cover - reported, not fatal to the GPU line
+        many = {"value": None, "unit": "tokens/s", "cores": cores, "kind": "oracle", "error": repr(exc)}
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)
+    # the line's cpu_baseline is the all-core figure; the one-core figure sits beside it
+    out = dict(many) if many.get("value") else dict(one)
+    out["one_core"] = one
+    return out
 
 
 def run_reference(a):
@@ -269,17 +430,28 @@ def run_milo(a):
     beta = wl.budgets[0]
     S = wl.suffix
 
-    # --- compression, timed (one "compression" = the whole layer's K and V)
-    comp = []
+    # --- compression, timed (one "compression" = the whole layer's K and V), with each kernel's share
+    comp, kern = [], {k: [] for k in ("gram", "jacobi", "alloc", "project")}
+    sweeps = None
     for i in range(4):
         st = torch.cuda.current_stream()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        for e in evs:  # torch creates the CUDA event on its first record
+            e.record(st)
+        torch.cuda.synchronize()
         e0.record(st)
-        f = milo.compress(Kd, Vd, wl.block_size, beta, wl.r_min)
+        f = milo.compress_profiled(Kd, Vd, wl.block_size, beta, evs, wl.r_min)
         e1.record(st)
         torch.cuda.synchronize()
         if i:
             comp.append(e0.elapsed_time(e1))
+            for k, name in enumerate(kern):
+                kern[name].append(evs[k].elapsed_time(evs[k + 1]))
+        if i == 3:
+            d = f.describe()
+            sweeps = _device_ints(torch, d["sweeps"], 2 * wl.kv_heads * wl.num_blocks)
+            comp_ranks = f.ranks()
         f.close()
 
     # --- decode inputs, rotated over enough copies that the working set exceeds 3x L2
@@ -303,35 +475,55 @@ def run_milo(a):
     for f in sets:
         assert f.status()[0] == 0
 
-    # capture one pass over all copies in a CUDA graph (the pages' launch-overhead remedy)
-    g = torch.cuda.CUDAGraph()
-    cap = torch.cuda.Stream()
-    cap.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(cap):
-        with torch.cuda.graph(g, stream=cap):
-            for c in range(copies):
-                milo.decode_attn(qs[c], sets[c], ks[c], vs[c], out=outs[c])
+    # CUDA graphs (the pages' launch-overhead remedy): one of a whole pass over the copies and one of the
+    # first (steps mod copies) of them, so that warm-up and every timed window run exactly the steps asked.
+    def capture(ncopies):
+        if ncopies == 0:
+            return None
+        g_ = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(g_, stream=cap):
+                for c in range(ncopies):
+                    milo.decode_attn(qs[c], sets[c], ks[c], vs[c], out=outs[c])
+        torch.cuda.synchronize()
+        return g_
+    g_full = capture(copies)
+    g_rest = {r: capture(r) for r in {a.steps % copies, a.warmup % copies} if r}
+
+    def run_steps(k):
+        for _ in range(k // copies):
+            g_full.replay()
+        if k % copies:
+            g_rest[k % copies].replay()
+
+    run_steps(a.warmup)
     torch.cuda.synchronize()
-    reps_w = max(1, math.ceil(a.warmup / copies))
-    reps = max(1, math.ceil(a.steps / copies))
-    steps = reps * copies
-    for _ in range(reps_w):
-        g.replay()
+    steps = a.steps
+    # repeated timed windows of `steps` steps each (the median is reported), enough of them that the clock
+    # sampler sees the GPU under load for at least ~0.3 s
+    probe_e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    probe_e[0].record()
+    run_steps(steps)
+    probe_e[1].record()
     torch.cuda.synchronize()
+    windows = max(5, min(2000, math.ceil(300.0 / max(probe_e[0].elapsed_time(probe_e[1]), 1e-3))))
     if world > 1:
+        windows = int(_max_over_ranks(windows, world))
         torch.distributed.barrier()
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    wev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(windows)]
     with ClockSampler(torch.cuda.current_device()) as clk:
-        e0.record(st)
-        for _ in range(reps):
-            g.replay()
-        e1.record(st)
+        for e0, e1 in wev:
+            e0.record(st)
+            run_steps(steps)
+            e1.record(st)
         torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    ms = _max_over_ranks(e0.elapsed_time(e1), world)
+    ms = _max_over_ranks(statistics.median(e0.elapsed_time(e1) for e0, e1 in wev), world)
     ms_step = ms / steps
     value = _job_value(world, wl.batch, steps, ms)
     per_call_ms = ms_step  # every step is one milo_decode_attn call
@@ -394,13 +586,14 @@ def run_milo(a):
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
-            "warmup": reps_w * copies, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": a.warmup, "ms_per_step": ms_step, "timed_windows": windows, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": dt, "data": "synthetic",
             "config": _config(wl, world, ranks.sum(),
                               l2=f"inputs rotated over {copies} copies ({copies * step_bytes / 1e6:.0f} MB > 3x L2)",
-                              launch="CUDA graph of one pass over the copies"),
+                              launch="CUDA graphs over the copies; median of the timed windows"),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": DECODE_TRAFFIC.get(wl.name), "peak_kind": peak_kind,
+                         "frac": achieved / peak, "traffic": DECODE_TRAFFIC.get((wl.name, _source_digest())),
+                         "peak_kind": peak_kind,
                          "bytes_per_step": step_bytes, "kernel": "decode_tc_kernel" if dt == "bf16" else
                          "prefix_kernel", "kernel_ms": kernel_ms, "call_ms": per_call_ms,
                          "note": "achieved = algorithmic bytes per step / mean CUDA-event duration of the main "
@@ -409,13 +602,16 @@ def run_milo(a):
             "e2e": {"value": _job_value(world, wl.batch, e2e_steps, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "compress": {"compressions_per_s": 1e3 / statistics.median(comp), "ms": statistics.median(comp),
-                         "unit": "whole-layer compressions/s"},
+                         "unit": "whole-layer compressions/s",
+                         "roofline": _compress_roofline(torch, wl, esize, comp_ranks, sweeps, kern, peak)},
             "gpu_launches": kernels_per_call * steps,
+            "gpu_launches_note": f"{kernels_per_call} kernels per decode call x {steps} steps of one timed window "
+                                 f"({windows} windows timed, the median reported)",
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    del g
+    del g_full, g_rest
     for f in sets:
         f.close()
     if world > 1:

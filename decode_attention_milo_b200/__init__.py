@@ -17,6 +17,8 @@ __all__ = ["F32", "BF16", "MiloError", "Factors", "compress", "decode_attn", "im
 
 F32, BF16 = 0, 1
 KEEP_INTERMEDIATES = 1
+ALLOC_RULES = {"entropy": 0, "greedy": 1, "uniform": 2, "weights": 3}
+POOL_SCOPES = {"pool": 0, "layer": 1}
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
 
@@ -34,10 +36,11 @@ class _Desc(ctypes.Structure):
     _fields_ = [
         ("num_kv_heads", ctypes.c_int32), ("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
         ("head_dim", ctypes.c_int32), ("context", ctypes.c_int64), ("r_min", ctypes.c_int32),
-        ("pool_rows", ctypes.c_int32), ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("pool_rows", ctypes.c_int32), ("dtype", ctypes.c_int32), ("alloc_rule", ctypes.c_int32),
+        ("pool_scope", ctypes.c_int32), ("reserved", ctypes.c_int32), ("total_rows", ctypes.c_int64),
         ("ranks", ctypes.c_void_p), ("row_offsets", ctypes.c_void_p), ("tok", ctypes.c_void_p),
         ("dim", ctypes.c_void_p), ("eigvals", ctypes.c_void_p), ("eigvecs", ctypes.c_void_p),
-        ("entropy", ctypes.c_void_p), ("quotas", ctypes.c_void_p),
+        ("entropy", ctypes.c_void_p), ("quotas", ctypes.c_void_p), ("sweeps", ctypes.c_void_p),
     ]
 
 
@@ -60,10 +63,18 @@ def load_library(path: str | None = None):
     L.milo_status_string.argtypes = [i32]
     L.milo_compress.restype = i32
     L.milo_compress.argtypes = [vp, vp, i32, i32, i64, i32, i32, f64, i32, i32, u32, vp, ctypes.POINTER(vp)]
+    L.milo_compress_rule.restype = i32
+    L.milo_compress_rule.argtypes = [vp, vp, i32, i32, i64, i32, i32, f64, i32, i32, u32, i32, i32, vp, vp,
+                                     ctypes.POINTER(vp)]
+    L.milo_compress_profiled.restype = i32
+    L.milo_compress_profiled.argtypes = [vp, vp, i32, i32, i64, i32, i32, f64, i32, i32, u32, vp,
+                                         ctypes.POINTER(vp), ctypes.POINTER(vp)]
     L.milo_decode_attn.restype = i32
     L.milo_decode_attn.argtypes = [vp, i32, i32, vp, vp, vp, i32, f32, vp, vp]
     L.milo_decode_attn_profiled.restype = i32
     L.milo_decode_attn_profiled.argtypes = [vp, i32, i32, vp, vp, vp, i32, f32, vp, vp, vp, vp]
+    L.milo_decode_attn_select.restype = i32
+    L.milo_decode_attn_select.argtypes = [vp, i32, i32, vp, vp, vp, i32, f32, vp, vp, vp]
     L.milo_decode_attn_noalloc.restype = i32
     L.milo_decode_attn_noalloc.argtypes = [vp, i32, i32, vp, vp, vp, i32, f32, vp, vp]
     L.milo_decode_launches.restype = i32
@@ -80,7 +91,7 @@ def load_library(path: str | None = None):
     L.milo_factors_import.argtypes = [i32, i32, i64, i32, i32, i32, vp, vp, vp, vp, ctypes.POINTER(vp)]
     L.milo_factors_destroy.restype = None
     L.milo_factors_destroy.argtypes = [vp]
-    if L.milo_abi_version() != 1:
+    if L.milo_abi_version() != 2:
         raise RuntimeError("libmilo.so ABI version mismatch")
     _lib = L
     return L
@@ -188,6 +199,44 @@ def compress(K, V, block_size: int, budget: float, r_min: int = 4, max_sweeps: i
     return Factors(h)
 
 
+def compress_rule(K, V, block_size: int, budget: float, rule: str = "entropy", scope: str = "pool",
+                  weights=None, r_min: int = 4, max_sweeps: int = 0, keep_intermediates: bool = False,
+                  stream=None) -> Factors:
+    """compress() with an allocation rule ("entropy", "greedy", "uniform", "weights") and budget scope
+    ("pool" or "layer"); weights: host [2H][nb] array for the "weights" rule. See milo_compress_rule."""
+    if K.shape != V.shape or K.dim() != 3 or K.dtype != V.dtype:
+        raise ValueError("K and V must both be [H][T][d] with the same dtype")
+    H, T, d = K.shape
+    w = None
+    if weights is not None:
+        w = np.ascontiguousarray(weights, dtype=np.float64)
+        if w.size != 2 * H * (T // block_size):
+            raise ValueError("weights must hold [2H][nb] values")
+    h = ctypes.c_void_p()
+    flags = KEEP_INTERMEDIATES if keep_intermediates else 0
+    _check(load_library().milo_compress_rule(
+        _dev_ptr(K, "K"), _dev_ptr(V, "V"), _dtype_code(K), H, T, d, block_size, float(budget), r_min, max_sweeps,
+        flags, ALLOC_RULES[rule], POOL_SCOPES[scope], None if w is None else w.ctypes.data_as(ctypes.c_void_p),
+        _stream_ptr(stream), ctypes.byref(h)), "milo_compress_rule")
+    return Factors(h)
+
+
+def compress_profiled(K, V, block_size: int, budget: float, events, r_min: int = 4, max_sweeps: int = 0,
+                      keep_intermediates: bool = False, stream=None) -> Factors:
+    """compress() that records five torch.cuda.Event objects: before the Gram, Jacobi, allocation and
+    projection kernels and after the last (milo_compress_profiled)."""
+    if K.shape != V.shape or K.dim() != 3 or K.dtype != V.dtype or len(events) != 5:
+        raise ValueError("K and V must both be [H][T][d] with the same dtype, and five events are needed")
+    H, T, d = K.shape
+    h = ctypes.c_void_p()
+    flags = KEEP_INTERMEDIATES if keep_intermediates else 0
+    evs = (ctypes.c_void_p * 5)(*[e.cuda_event for e in events])
+    _check(load_library().milo_compress_profiled(_dev_ptr(K, "K"), _dev_ptr(V, "V"), _dtype_code(K), H, T, d,
+                                                 block_size, float(budget), r_min, max_sweeps, flags,
+                                                 _stream_ptr(stream), ctypes.byref(h), evs), "milo_compress_profiled")
+    return Factors(h)
+
+
 def _decode_args(q, factors: Factors, K_suf, V_suf, out):
     """Checks the shapes and dtypes of one decode call against the factors (the C ABI takes no q shape or
     dtype beyond batch and heads, so a mismatched tensor would be read or written past its end) and
@@ -225,6 +274,23 @@ def decode_attn(q, factors: Factors, K_suf=None, V_suf=None, scale: float = 0.0,
                                            _dev_ptr(K_suf, "K_suf") if S else None,
                                            _dev_ptr(V_suf, "V_suf") if S else None, S, float(scale),
                                            _dev_ptr(out, "out"), _stream_ptr(stream)), "milo_decode_attn")
+    return out
+
+
+def decode_attn_select(q, factors: Factors, block_mask, K_suf=None, V_suf=None, scale: float = 0.0, out=None,
+                       stream=None):
+    """decode_attn over the blocks block_mask [H][nb] selects (host array, nonzero = attend).
+    See milo_decode_attn_select."""
+    B, Hq, S, out = _decode_args(q, factors, K_suf, V_suf, out)
+    H = factors.shape()[0]
+    nb = factors.describe()["num_blocks"]
+    m = np.ascontiguousarray(np.asarray(block_mask) != 0, dtype=np.uint8)
+    if m.shape != (H, nb):
+        raise ValueError(f"block_mask must be [{H}][{nb}], got {m.shape}")
+    _check(load_library().milo_decode_attn_select(
+        _dev_ptr(q, "q"), B, Hq, factors.handle, _dev_ptr(K_suf, "K_suf") if S else None,
+        _dev_ptr(V_suf, "V_suf") if S else None, S, float(scale), m.ctypes.data_as(ctypes.c_void_p),
+        _dev_ptr(out, "out"), _stream_ptr(stream)), "milo_decode_attn_select")
     return out
 
 

@@ -12,7 +12,7 @@
 //            clamp(lam·w_b, r_min, d) with Σ = R, largest-remainder ranks,
 //            row offsets                                  (one CTA per pool)
 //   project  U_b = X_b · B_b[:, :r_b], stored transposed in 128-token slabs, and B_bᵀ rows
-//                                                         (one CTA per block)
+//            (bf16 blocks: tensor cores, project_tc.cu; fp32: here, one CTA per block)
 #include <math.h>
 
 #include "common.cuh"
@@ -90,7 +90,7 @@ __device__ __forceinline__ void rr_pair(int D, int s, int k, int& p, int& q) {
 template <int D>
 __global__ void __launch_bounds__(kJThreads) jacobi_kernel(const float* __restrict__ gram, int nb, int max_sweeps,
                                                          float* __restrict__ eigvals, float* __restrict__ eigvecs,
-                                                         uint32_t* status) {
+                                                         int32_t* __restrict__ sweeps_out, uint32_t* status) {
   constexpr int E = D / 32;  // elements per lane of one column
   extern __shared__ float smem[];
   float* A = smem;          // column-major: column j at A[j*D]
@@ -107,7 +107,9 @@ __global__ void __launch_bounds__(kJThreads) jacobi_kernel(const float* __restri
   constexpr int NW = kJThreads / 32;
   constexpr int PP = (D / 2) / NW;  // column pairs per warp per round
   bool converged = false;
+  int sweeps_run = 0;
   for (int sweep = 0; sweep < max_sweeps; ++sweep) {
+    ++sweeps_run;
     int rotated = 0;
     for (int s = 0; s < D - 1; ++s) {
       // the warp's PP pairs are handled together so that their loads and reductions overlap
@@ -161,6 +163,7 @@ __global__ void __launch_bounds__(kJThreads) jacobi_kernel(const float* __restri
     }
   }
   if (!converged && threadIdx.x == 0) atomicOr(status, kStatusNoConvergence);
+  if (threadIdx.x == 0) sweeps_out[blk] = sweeps_run;
   // eigenvalue of column j = |G w_j| = norm of A's column j
   for (int j = warp; j < D; j += kJThreads / 32) {
     float ss = 0.f;
@@ -190,64 +193,141 @@ __global__ void __launch_bounds__(kJThreads) jacobi_kernel(const float* __restri
 // ---------------------------------------------------------------- alloc
 __device__ __forceinline__ double clampd(double x, double lo, double hi) { return fmin(fmax(x, lo), hi); }
 
-__global__ void __launch_bounds__(kThreads) alloc_kernel(const float* __restrict__ eigvals, int nb, int D, int R,
-                                                        int r_min, int pool_rows, double* __restrict__ entropy,
-                                                        double* __restrict__ quotas, int32_t* __restrict__ ranks,
-                                                        int64_t* __restrict__ row_offsets) {
+constexpr int kAThreads = 512;
+
+// Sum over the CTA of one value per thread (all threads call it; red holds kAThreads / 32 entries).
+template <typename V>
+__device__ V cta_sum(V v, V* red) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = v;
+  __syncthreads();
+  V t = 0;
+  for (int i = 0; i < kAThreads / 32; ++i) t += red[i];
+  return t;
+}
+
+// Energy share of component i of a block, from its fp32 eigenvalues (negatives count as 0), in fp64.
+__device__ __forceinline__ double share_of(const float* lam, int i, double tot) {
+  return tot > 0.0 ? fmax((double)lam[i], 0.0) / tot : 0.0;
+}
+
+// Candidates of a block for the greedy rule with share >= t (as fp64 bit patterns: non-negative doubles order
+// like their bits): components r_min .. D-1, whose shares do not increase, so a binary search counts them.
+__device__ __forceinline__ int count_at_least(const float* lam, int D, int r_min, double tot, unsigned long long t) {
+  int lo = r_min, hi = D;  // the answer is the first i in [r_min, D] with share(i) < t, minus r_min
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if ((unsigned long long)__double_as_longlong(share_of(lam, mid, tot)) >= t) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo - r_min;
+}
+
+// Rank allocation over one group of N consecutive blocks [g0, g0 + N) of the [2H][nb] block order: a pool
+// (one CTA per pool) or the whole layer (one CTA).  Rules (§4.3 and the §5.3 baselines):
+//   0 entropy  H_b = −Σ p ln p (p = λ/Σλ, fp64), w_b = e^{H_b}, quotas clamp(lam·w_b, r_min, d) with Σ = R,
+//              largest-remainder rounding (ties to the lower index)
+//   1 greedy   every block starts at r_min; the R − N·r_min free units go to the largest next-component
+//              energy shares λ_i/Σλ (ties to the lower block index): the K largest candidates, found by
+//              bisection on their fp64 bit patterns
+//   2 uniform  floor(R / N) each, the remainder to the lowest indices
+//   3 weights  caller weights (the random baseline's draws) with the entropy rule's water-filling
+// Row offsets: pool groups start at p · pool_rows; a layer group's pools follow each other.
+__global__ void __launch_bounds__(kAThreads) alloc_kernel(const float* __restrict__ eigvals, int P, int nb, int D,
+                                                         int R, int r_min, int rule, bool layer, int pool_rows,
+                                                         const double* __restrict__ user_w,
+                                                         double* __restrict__ entropy, double* __restrict__ quotas,
+                                                         int32_t* __restrict__ ranks,
+                                                         int64_t* __restrict__ row_offsets) {
   extern __shared__ double sh[];
-  double* w = sh;             // nb
-  double* q = w + nb;         // nb
-  double* frac = q + nb;      // nb
-  int* fl = (int*)(frac + nb);  // nb
+  const int N = layer ? P * nb : nb;
+  const int g0 = layer ? 0 : blockIdx.x * nb;
+  double* w = sh;             // N: weights (water-filling rules) or Σλ (greedy)
+  double* q = w + N;          // N: quotas
+  int* fl = (int*)(q + N);    // N: integer part of the rank
   __shared__ double s_lam;
   __shared__ int s_rem;
-  const int p = blockIdx.x;
+  __shared__ double red_d[kAThreads / 32];
+  __shared__ long long red_l[kAThreads / 32];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  // entropy and weights
-  for (int b = warp; b < nb; b += kThreads / 32) {
-    const float* lam = eigvals + ((int64_t)p * nb + b) * D;
+  // entropy (always, it is an intermediate) and the rule's per-block weight
+  for (int i = warp; i < N; i += kAThreads / 32) {
+    const float* lam = eigvals + (int64_t)(g0 + i) * D;
     double tot = 0.0;
-    for (int i = lane; i < D; i += 32) tot += fmax((double)lam[i], 0.0);
+    for (int k = lane; k < D; k += 32) tot += fmax((double)lam[k], 0.0);
     tot = warp_sum(tot);
     double h = 0.0;
     if (tot > 0.0) {
-      for (int i = lane; i < D; i += 32) {
-        const double pi = fmax((double)lam[i], 0.0) / tot;
+      for (int k = lane; k < D; k += 32) {
+        const double pi = fmax((double)lam[k], 0.0) / tot;
         if (pi > 0.0) h -= pi * log(pi);
       }
       h = warp_sum(h);
     }
     if (lane == 0) {
-      entropy[(int64_t)p * nb + b] = h;
-      w[b] = exp(h);
+      entropy[g0 + i] = h;
+      w[i] = rule == 0 ? exp(h) : rule == 3 ? user_w[g0 + i] : tot;
     }
   }
   __syncthreads();
-  const bool full = (int64_t)R >= (int64_t)nb * D;
-  if (full) {
-    for (int b = threadIdx.x; b < nb; b += kThreads) {
-      q[b] = D;
-      fl[b] = D;
-      frac[b] = 0.0;
+  const bool full = (int64_t)R >= (int64_t)N * D;
+  const double nan = __longlong_as_double(0x7ff8000000000000LL);
+  if (full || rule == 2) {
+    for (int i = threadIdx.x; i < N; i += kAThreads) {
+      const int r = full ? D : R / N + (i < R % N ? 1 : 0);
+      q[i] = full ? (double)D : nan;
+      fl[i] = r;
     }
-    if (threadIdx.x == 0) s_rem = 0;
+  } else if (rule == 1) {
+    // K-th largest candidate share: the largest bit pattern t with count(share >= t) >= K
+    const long long K = (long long)R - (long long)N * r_min;
+    unsigned long long lo = 0, hi = (unsigned long long)__double_as_longlong(1.0) + 1;  // count(lo) >= K > count(hi)
+    if (K > 0) {
+      while (hi - lo > 1) {
+        const unsigned long long mid = lo + (hi - lo) / 2;
+        long long c = 0;
+        for (int i = threadIdx.x; i < N; i += kAThreads)
+          c += count_at_least(eigvals + (int64_t)(g0 + i) * D, D, r_min, w[i], mid);
+        c = cta_sum<long long>(c, red_l);
+        if (c >= K) lo = mid;
+        else hi = mid;
+      }
+    }
+    // blocks take every candidate above the cut; the units left at exactly the cut value go to the lowest blocks
+    for (int i = threadIdx.x; i < N; i += kAThreads) {
+      const float* lam = eigvals + (int64_t)(g0 + i) * D;
+      const int ge = K > 0 ? count_at_least(lam, D, r_min, w[i], lo) : 0;
+      const int gt = K > 0 ? count_at_least(lam, D, r_min, w[i], lo + 1) : 0;
+      fl[i] = r_min + gt;
+      q[i] = (double)(ge - gt);  // candidates at the cut value (reused below), quota NaN afterwards
+    }
     __syncthreads();
+    if (threadIdx.x == 0) {
+      long long m = K;
+      for (int i = 0; i < N; ++i) m -= fl[i] - r_min;
+      for (int i = 0; i < N; ++i) {
+        const int take = (int)min((long long)q[i], max(m, 0LL));
+        fl[i] += take;
+        m -= take;
+        q[i] = nan;
+      }
+    }
   } else {
     // water level: smallest kink with sum >= R and largest kink with sum < R
     double lo = -1.0, hi = INFINITY;
-    for (int k = threadIdx.x; k < 2 * nb; k += kThreads) {
+    for (int k = threadIdx.x; k < 2 * N; k += kAThreads) {
       const double kink = (k & 1 ? (double)D : (double)r_min) / w[k >> 1];
       double f = 0.0;
-      for (int b = 0; b < nb; ++b) f += clampd(kink * w[b], r_min, D);
+      for (int b = 0; b < N; ++b) f += clampd(kink * w[b], r_min, D);
       if (f >= (double)R) hi = fmin(hi, kink);
       else lo = fmax(lo, kink);
     }
-    // block min / max
     for (int o = 16; o > 0; o >>= 1) {
       hi = fmin(hi, __shfl_xor_sync(0xffffffffu, hi, o));
       lo = fmax(lo, __shfl_xor_sync(0xffffffffu, lo, o));
     }
-    __shared__ double red_lo[kThreads / 32], red_hi[kThreads / 32];
+    __shared__ double red_lo[kAThreads / 32], red_hi[kAThreads / 32];
     if (lane == 0) {
       red_lo[warp] = lo;
       red_hi[warp] = hi;
@@ -255,19 +335,19 @@ __global__ void __launch_bounds__(kThreads) alloc_kernel(const float* __restrict
     __syncthreads();
     if (threadIdx.x == 0) {
       double L = -1.0, Hh = INFINITY;
-      for (int i = 0; i < kThreads / 32; ++i) {
+      for (int i = 0; i < kAThreads / 32; ++i) {
         L = fmax(L, red_lo[i]);
         Hh = fmin(Hh, red_hi[i]);
       }
       double fh = 0.0;
-      for (int b = 0; b < nb; ++b) fh += clampd(Hh * w[b], r_min, D);
+      for (int b = 0; b < N; ++b) fh += clampd(Hh * w[b], r_min, D);
       double lam;
       if (fh == (double)R) {
         lam = Hh;
       } else {
         const double mid = 0.5 * (L + Hh);
         double fixed = 0.0, W = 0.0;
-        for (int b = 0; b < nb; ++b) {
+        for (int b = 0; b < N; ++b) {
           const double x = mid * w[b];
           if (x <= r_min) fixed += r_min;
           else if (x >= D) fixed += D;
@@ -280,43 +360,48 @@ __global__ void __launch_bounds__(kThreads) alloc_kernel(const float* __restrict
     __syncthreads();
     const double lam = s_lam;
     int partial = 0;
-    for (int b = threadIdx.x; b < nb; b += kThreads) {
+    for (int b = threadIdx.x; b < N; b += kAThreads) {
       const double qb = clampd(lam * w[b], r_min, D);
       const double f = floor(qb);
       q[b] = qb;
       fl[b] = (int)f;
-      frac[b] = qb - f;
       partial += (int)f;
     }
-    for (int o = 16; o > 0; o >>= 1) partial += __shfl_xor_sync(0xffffffffu, partial, o);
-    __shared__ int red_i[kThreads / 32];
-    if (lane == 0) red_i[warp] = partial;
+    const int tot = cta_sum<int>(partial, (int*)red_l);
+    if (threadIdx.x == 0) s_rem = R - tot;
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int tot = 0;
-      for (int i = 0; i < kThreads / 32; ++i) tot += red_i[i];
-      s_rem = R - tot;
+    // largest remainder: the s_rem blocks with the largest fractional parts get one more (ties: lower index)
+    const int rem = s_rem;
+    for (int b = threadIdx.x; b < N; b += kAThreads) {
+      int rank = 0;
+      const double fb = q[b] - fl[b];
+      for (int c = 0; c < N; ++c) {
+        const double fc = q[c] - fl[c];
+        rank += (fc > fb) || (fc == fb && c < b);
+      }
+      ranks[g0 + b] = fl[b] + (rank < rem ? 1 : 0);
     }
     __syncthreads();
+    for (int b = threadIdx.x; b < N; b += kAThreads) fl[b] = ranks[g0 + b];
   }
-  const int rem = s_rem;
-  for (int b = threadIdx.x; b < nb; b += kThreads) {
-    int rank = 0;
-    const double fb = frac[b];
-    for (int c = 0; c < nb; ++c) rank += (frac[c] > fb) || (frac[c] == fb && c < b);
-    const int r = fl[b] + (rank < rem ? 1 : 0);
-    ranks[(int64_t)p * nb + b] = r;
-    quotas[(int64_t)p * nb + b] = q[b];
+  __syncthreads();
+  for (int b = threadIdx.x; b < N; b += kAThreads) {
+    ranks[g0 + b] = fl[b];
+    quotas[g0 + b] = q[b];
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    int64_t off = (int64_t)p * pool_rows;
-    int64_t* ro = row_offsets + (int64_t)p * (nb + 1);
-    for (int b = 0; b < nb; ++b) {
-      ro[b] = off;
-      off += ranks[(int64_t)p * nb + b];
+    // row offsets [P][nb + 1]: block b of pool p owns rows [ro[b], ro[b] + r); ro[nb] is the pool's end
+    const int p0 = layer ? 0 : blockIdx.x, p1 = layer ? P : blockIdx.x + 1;
+    int64_t off = layer ? 0 : (int64_t)blockIdx.x * pool_rows;
+    for (int pp = p0; pp < p1; ++pp) {
+      int64_t* ro = row_offsets + (int64_t)pp * (nb + 1);
+      for (int b = 0; b < nb; ++b) {
+        ro[b] = off;
+        off += fl[(pp - p0) * nb + b];
+      }
+      ro[nb] = off;
     }
-    ro[nb] = off;
   }
 }
 
@@ -367,10 +452,14 @@ __global__ void __launch_bounds__(kThreads) project_kernel(const T* __restrict__
 }
 
 template <typename T, int D>
-cudaError_t run(const CompressShape& s, const CompressBuffers& bf, cudaStream_t st) {
+cudaError_t run(const CompressShape& s, const CompressBuffers& bf, cudaStream_t st, const cudaEvent_t* ev) {
   const T* K = static_cast<const T*>(bf.K);
   const T* V = static_cast<const T*>(bf.V);
   dim3 grid(s.nb, 2 * s.H);
+  // ev[k] (optional) is recorded on `st` before kernel k (gram, jacobi, alloc, project) and ev[4] after the last
+  auto mark = [&](int k) -> cudaError_t { return ev && ev[k] ? cudaEventRecord(ev[k], st) : cudaSuccess; };
+  cudaError_t me;
+  if ((me = mark(0)) != cudaSuccess) return me;
   // bf16 blocks: Gram on the tensor cores (gram_tc.cu); fp32 blocks: on the CUDA cores
   const cudaError_t ge = launch_gram_tc(s, K, V, bf.gram, bf.status, st);
   if (ge == cudaErrorNotSupported) {
@@ -382,29 +471,43 @@ cudaError_t run(const CompressShape& s, const CompressBuffers& bf, cudaStream_t 
   const size_t jsm = (2 * D * D + D) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(jacobi_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)jsm);
   if (e != cudaSuccess) return e;
-  jacobi_kernel<D><<<grid, kJThreads, jsm, st>>>(bf.gram, s.nb, s.max_sweeps, bf.eigvals, bf.eigvecs, bf.status);
-  const size_t asm_ = (size_t)s.nb * (3 * sizeof(double) + sizeof(int));
+  if ((e = mark(1)) != cudaSuccess) return e;
+  jacobi_kernel<D><<<grid, kJThreads, jsm, st>>>(bf.gram, s.nb, s.max_sweeps, bf.eigvals, bf.eigvecs, bf.sweeps,
+                                                 bf.status);
+  const int ngroup = s.layer_scope ? 2 * s.H * s.nb : s.nb;
+  const size_t asm_ = (size_t)ngroup * (2 * sizeof(double) + sizeof(int));
   e = cudaFuncSetAttribute(alloc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asm_);
   if (e != cudaSuccess) return e;
-  alloc_kernel<<<2 * s.H, kThreads, asm_, st>>>(bf.eigvals, s.nb, D, s.R, s.r_min, s.pool_rows, bf.entropy,
-                                                 bf.quotas, bf.ranks, bf.row_offsets);
+  if ((e = mark(2)) != cudaSuccess) return e;
+  alloc_kernel<<<s.layer_scope ? 1 : 2 * s.H, kAThreads, asm_, st>>>(
+      bf.eigvals, 2 * s.H, s.nb, D, s.R, s.r_min, s.rule, s.layer_scope, s.pool_rows, bf.weights, bf.entropy,
+      bf.quotas, bf.ranks, bf.row_offsets);
   const size_t psm = (D * D + D * 64) * sizeof(float);
   e = cudaFuncSetAttribute(project_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm);
   if (e != cudaSuccess) return e;
-  project_kernel<T, D><<<grid, kThreads, psm, st>>>(K, V, s.T, s.n, s.nb, bf.eigvecs, bf.ranks, bf.row_offsets,
-                                                    static_cast<T*>(bf.tok), static_cast<T*>(bf.dim), bf.status);
-  return cudaGetLastError();
+  if ((e = mark(3)) != cudaSuccess) return e;
+  // bf16 blocks: projection on the tensor cores (project_tc.cu); fp32 blocks: on the CUDA cores
+  e = launch_project_tc(s, K, V, bf.eigvecs, bf.ranks, bf.row_offsets, bf.tok, bf.dim, bf.status, st);
+  if (e == cudaErrorNotSupported) {
+    cudaGetLastError();
+    project_kernel<T, D><<<grid, kThreads, psm, st>>>(K, V, s.T, s.n, s.nb, bf.eigvecs, bf.ranks, bf.row_offsets,
+                                                      static_cast<T*>(bf.tok), static_cast<T*>(bf.dim), bf.status);
+  } else if (e != cudaSuccess) {
+    return e;
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return mark(4);
 }
 
 }  // namespace
 
-cudaError_t launch_compress(const CompressShape& s, const CompressBuffers& b, cudaStream_t st) {
+cudaError_t launch_compress(const CompressShape& s, const CompressBuffers& b, cudaStream_t st, const cudaEvent_t* ev) {
   if (s.bf16) {
-    if (s.d == 64) return run<__nv_bfloat16, 64>(s, b, st);
-    return run<__nv_bfloat16, 128>(s, b, st);
+    if (s.d == 64) return run<__nv_bfloat16, 64>(s, b, st, ev);
+    return run<__nv_bfloat16, 128>(s, b, st, ev);
   }
-  if (s.d == 64) return run<float, 64>(s, b, st);
-  return run<float, 128>(s, b, st);
+  if (s.d == 64) return run<float, 64>(s, b, st, ev);
+  return run<float, 128>(s, b, st, ev);
 }
 
 }  // namespace milo

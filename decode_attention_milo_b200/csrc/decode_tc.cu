@@ -108,6 +108,7 @@ struct Params {
   const int64_t* row_offsets;
   float* part_acc;  // [pid][128][D]
   float2* part_ml;  // [pid][128]
+  const int* sel;   // [H][nb]: the k-th selected block of each head (block selection), or null for every block
   uint32_t* status;
   int nb, cpb, H, G, ipt, S;
   float c;  // scale · log2(e)
@@ -201,7 +202,10 @@ __device__ __forceinline__ void rescale_tmem(uint32_t taddr, int ncols, float al
 
 __device__ __forceinline__ int pad16(int r) { return (r + 15) & ~15; }
 
-__device__ __forceinline__ bool block_info(const Params& p, int h, int b, int D, BlockInfo& bi) {
+// Block k of head h's walk (the k-th selected block when a selection is given) → its ranks and row offsets.
+__device__ __forceinline__ bool block_info(const Params& p, int h, int k, int D, BlockInfo& bi) {
+  const int b = p.sel ? p.sel[(int64_t)h * p.nb + k] : k;
+  if ((unsigned)b >= (unsigned)p.nb) return false;
   bi.rk = p.ranks[(int64_t)(2 * h) * p.nb + b];
   bi.rv = p.ranks[(int64_t)(2 * h + 1) * p.nb + b];
   bi.rowk = p.row_offsets[(int64_t)(2 * h) * (p.nb + 1) + b];
@@ -1185,6 +1189,8 @@ bool make_call_maps(Maps* M, const DecodeShape& s, const TcInputs& in, int ipt) 
 
 struct TcPlan {
   int Bq = 0, Hq = 0, S = 0;
+  std::vector<uint8_t> mask;  // the block selection this plan was built for (empty: every block)
+  int off_sel = -1;
   int grid = 0, nsegs = 0, ipt = 0, nrt = 0;
   int* d_work = nullptr;  // seg_first | segs | pre_range | suf_range
   int off_segs = 0, off_pre = 0, off_suf = 0;
@@ -1233,20 +1239,27 @@ inline double suffix_atom_ns(int c, int d) {
 // slots [first, end) of one output row group).  Returns the number of words used, or -1 if `cap` is too small
 // or a row would have more than kMaxParts partials.
 int build_worklist_fixed(const DecodeShape& s, const int32_t* host_ranks, int grid, int* w, int cap, int& nsegs,
-                         int& off_segs, int& off_pre, int& off_suf, int& ipt_out, int& nrt_out) {
+                         int& off_segs, int& off_pre, int& off_suf, int& ipt_out, int& nrt_out,
+                         const uint8_t* mask, int* off_sel) {
   const int H = s.H, nb = s.nb, D = s.d, G = s.Hq / s.H, Bq = s.Bq, S = s.S;
   const int cpb = s.n / kChunk;
   const int ipt = std::min(Bq, 128 / G);
   const int nrt = (Bq + ipt - 1) / ipt;
   const int nsc = (S + kChunk - 1) / kChunk;
   const int seg_words = (int)(sizeof(Seg) / sizeof(int));
+  // prefix chunks are numbered along each head's walk: the k-th walked block (the k-th selected one under a
+  // selection) holds chunks [k·cpb, k·cpb + cpb)
   auto for_each_atom = [&](auto&& fn) {
     for (int h = 0; h < H; ++h)
-      for (int rt = 0; rt < nrt; ++rt)
+      for (int rt = 0; rt < nrt; ++rt) {
+        int k = 0;
         for (int b = 0; b < nb; ++b) {
+          if (mask && !mask[(size_t)h * nb + b]) continue;
           const int rk = host_ranks[(size_t)(2 * h) * nb + b], rv = host_ranks[(size_t)(2 * h + 1) * nb + b];
-          for (int cc = 0; cc < cpb; ++cc) fn(0, h, rt, b * cpb + cc, prefix_atom_ns(rk, rv, cc, D));
+          for (int cc = 0; cc < cpb; ++cc) fn(0, h, rt, k * cpb + cc, prefix_atom_ns(rk, rv, cc, D));
+          ++k;
         }
+      }
     for (int i = 0; i < Bq; ++i)
       for (int h = 0; h < H; ++h)
         for (int c = 0; c < nsc; ++c)
@@ -1294,8 +1307,18 @@ int build_worklist_fixed(const DecodeShape& s, const int32_t* host_ranks, int gr
   for (int k = cta + 1; k <= grid; ++k) seg_first[k] = n;
   off_pre = off_segs + n * seg_words;
   off_suf = off_pre + 2 * H * nrt;
-  const int nwords = off_suf + 2 * Bq * H;
+  const int nwords = off_suf + 2 * Bq * H + (mask ? H * nb : 0);
   if (nwords > cap) return -1;
+  if (off_sel) *off_sel = mask ? off_suf + 2 * Bq * H : -1;
+  if (mask) {  // the selected blocks of each head in order (entries past a head's count are unused)
+    int* sel = w + off_suf + 2 * Bq * H;
+    for (int h = 0; h < H; ++h) {
+      int k = 0;
+      for (int b = 0; b < nb; ++b)
+        if (mask[(size_t)h * nb + b]) sel[(size_t)h * nb + k++] = b;
+      for (; k < nb; ++k) sel[(size_t)h * nb + k] = 0;
+    }
+  }
   int* pre = w + off_pre;
   int* suf = w + off_suf;
   for (int i = 0; i < 2 * H * nrt; ++i) pre[i] = -1;
@@ -1322,35 +1345,42 @@ int build_worklist_fixed(const DecodeShape& s, const int32_t* host_ranks, int gr
   return nwords;
 }
 
-// CTAs of the decode kernel: one per SM, fewer when there are fewer atoms.
-int plan_grid(const DecodeShape& s, int sms) {
-  const int cpb = s.n / kChunk, nsc = (s.S + kChunk - 1) / kChunk;
-  const int ipt = std::min(s.Bq, 128 / (s.Hq / s.H));
-  const int64_t natoms =
-      (int64_t)s.H * ((s.Bq + ipt - 1) / ipt) * s.nb * cpb + (int64_t)s.Bq * s.H * nsc;
-  return (int)std::max<int64_t>(1, std::min<int64_t>(sms, natoms));
-}
-// Words a work list can need at most (every atom its own segment).
-int64_t worklist_cap(const DecodeShape& s, int grid) {
+// Work atoms of a decode shape (128-token chunks of every (KV head, row tile) walk and of every suffix).
+int64_t count_atoms(const DecodeShape& s, const uint8_t* mask) {
   const int cpb = s.n / kChunk, nsc = (s.S + kChunk - 1) / kChunk;
   const int ipt = std::min(s.Bq, 128 / (s.Hq / s.H)), nrt = (s.Bq + ipt - 1) / ipt;
-  const int64_t natoms = (int64_t)s.H * nrt * s.nb * cpb + (int64_t)s.Bq * s.H * nsc;
-  return grid + 1 + natoms * (int64_t)(sizeof(Seg) / sizeof(int)) + 2LL * s.H * nrt + 2LL * s.Bq * s.H;
+  int64_t blocks = (int64_t)s.H * s.nb;
+  if (mask) {
+    blocks = 0;
+    for (int64_t i = 0; i < (int64_t)s.H * s.nb; ++i) blocks += mask[i] ? 1 : 0;
+  }
+  return blocks * nrt * cpb + (int64_t)s.Bq * s.H * nsc;
+}
+// CTAs of the decode kernel: one per SM, fewer when there are fewer atoms.
+int plan_grid(const DecodeShape& s, int sms, const uint8_t* mask = nullptr) {
+  return (int)std::max<int64_t>(1, std::min<int64_t>(sms, count_atoms(s, mask)));
+}
+// Words a work list can need at most (every atom its own segment).
+int64_t worklist_cap(const DecodeShape& s, int grid, const uint8_t* mask = nullptr) {
+  const int ipt = std::min(s.Bq, 128 / (s.Hq / s.H)), nrt = (s.Bq + ipt - 1) / ipt;
+  return grid + 1 + count_atoms(s, mask) * (int64_t)(sizeof(Seg) / sizeof(int)) + 2LL * s.H * nrt +
+         2LL * s.Bq * s.H + (mask ? (int64_t)s.H * s.nb : 0);
 }
 
-static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& in) {
+static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& in, const uint8_t* mask) {
   const int D = s.d;
   const int cpb = s.n / kChunk;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = plan_grid(s, sms);
-  const int64_t cap = worklist_cap(s, grid);
+  const int grid = plan_grid(s, sms, mask);
+  const int64_t cap = worklist_cap(s, grid, mask);
   if (cap > (int64_t)1 << 30) return cudaErrorInvalidValue;
   std::vector<int> host((size_t)cap);
   int nsegs = 0, off_segs = 0, off_pre = 0, off_suf = 0, ipt = 0, nrt = 0;
   const int nwords = build_worklist_fixed(s, in.host_ranks, grid, host.data(), (int)cap, nsegs, off_segs, off_pre,
-                                          off_suf, ipt, nrt);
+                                          off_suf, ipt, nrt, mask, &pl->off_sel);
+  if (mask) pl->mask.assign(mask, mask + (size_t)s.H * s.nb);
   if (nwords < 0) return cudaErrorInvalidValue;
   pl->off_segs = off_segs;
   pl->off_pre = off_pre;
@@ -1371,7 +1401,7 @@ static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& 
   pl->nrt = nrt;
   // factor maps: the token factor as a [rows · n/128][128] array of 128-token slab rows, the dim factor
   // as [rows][d]
-  const uint64_t rows = (uint64_t)2 * s.H * in.pool_rows;
+  const uint64_t rows = (uint64_t)in.total_rows;
   if (!make_row_maps(&pl->map_tok, in.tok, kChunk, rows * cpb)) return cudaErrorInvalidValue;
   if (!make_row_maps(&pl->map_dim, in.dim, D, rows)) return cudaErrorInvalidValue;
   if (!make_pacc_map(&pl->map_pacc, pl->part_acc, pl->nsegs, D)) return cudaErrorInvalidValue;
@@ -1381,13 +1411,16 @@ static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& 
 }
 
 cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, void* out, cudaStream_t st,
-                      cudaEvent_t ev0, cudaEvent_t ev1) {
+                      cudaEvent_t ev0, cudaEvent_t ev1, const uint8_t* mask) {
   TcPlan* pl = *plan;
-  if (!pl || pl->Bq != s.Bq || pl->Hq != s.Hq || pl->S != s.S || pl->tok != in.tok) {
+  const bool same_mask = pl && (mask ? pl->mask.size() == (size_t)s.H * s.nb &&
+                                           std::memcmp(pl->mask.data(), mask, pl->mask.size()) == 0
+                                     : pl->mask.empty());
+  if (!pl || pl->Bq != s.Bq || pl->Hq != s.Hq || pl->S != s.S || pl->tok != in.tok || !same_mask) {
     tc_plan_destroy(pl);
     *plan = nullptr;
     pl = new TcPlan();
-    cudaError_t e = build_plan(pl, s, in);
+    cudaError_t e = build_plan(pl, s, in, mask);
     if (e != cudaSuccess) {
       tc_plan_destroy(pl);
       return e;
@@ -1407,6 +1440,7 @@ cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, v
   p.row_offsets = in.row_offsets;
   p.part_acc = pl->part_acc;
   p.part_ml = pl->part_ml;
+  p.sel = pl->off_sel >= 0 ? pl->d_work + pl->off_sel : nullptr;
   p.status = in.status;
   p.nb = s.nb;
   p.cpb = s.n / kChunk;
@@ -1459,8 +1493,8 @@ int tc_worklist(const DecodeShape& s, const int32_t* host_ranks, int sms, int* w
   if (cap > INT32_MAX) cap = INT32_MAX;
   const int grid = plan_grid(s, sms);
   int nsegs = 0, off_segs = 0, off_pre = 0, off_suf = 0, ipt = 0, nrt = 0;
-  const int nwords =
-      build_worklist_fixed(s, host_ranks, grid, w, (int)cap, nsegs, off_segs, off_pre, off_suf, ipt, nrt);
+  const int nwords = build_worklist_fixed(s, host_ranks, grid, w, (int)cap, nsegs, off_segs, off_pre, off_suf, ipt,
+                                          nrt, nullptr, nullptr);
   if (nwords < 0) return -1;
   const int64_t v[8] = {nwords, nsegs, grid, off_segs, off_pre, off_suf, ipt, nrt};
   for (int i = 0; i < 8; ++i) info[i] = v[i];
@@ -1494,7 +1528,7 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
   const int grid = plan_grid(s, sms);
   int nsegs = 0, off_segs = 0, off_pre = 0, off_suf = 0, ipt = 0, nrt = 0;
   const int nwords = build_worklist_fixed(s, in.host_ranks, grid, g_noalloc_host_words, kNoAllocMaxWords, nsegs,
-                                          off_segs, off_pre, off_suf, ipt, nrt);
+                                          off_segs, off_pre, off_suf, ipt, nrt, nullptr, nullptr);
   const size_t words_bytes = ((size_t)std::max(nwords, 0) * sizeof(int) + 255) & ~(size_t)255;
   const size_t ml_bytes = ((size_t)nsegs * 128 * sizeof(float2) + 255) & ~(size_t)255;
   const size_t acc_bytes = (size_t)nsegs * 128 * s.d * sizeof(float);
@@ -1511,7 +1545,7 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
     return e;
   const int D = s.d, G = s.Hq / s.H;
   Maps maps;
-  const uint64_t rows = (uint64_t)2 * s.H * in.pool_rows;
+  const uint64_t rows = (uint64_t)in.total_rows;
   if (!make_row_maps(&maps.tok, in.tok, kChunk, rows * cpb)) return cudaErrorInvalidValue;
   if (!make_row_maps(&maps.dim, in.dim, D, rows)) return cudaErrorInvalidValue;
   if (!make_pacc_map(&maps.pacc, part_acc, nsegs, D)) return cudaErrorInvalidValue;
@@ -1523,6 +1557,7 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
   p.row_offsets = in.row_offsets;
   p.part_acc = part_acc;
   p.part_ml = part_ml;
+  p.sel = nullptr;
   p.status = in.status;
   p.nb = s.nb;
   p.cpb = cpb;

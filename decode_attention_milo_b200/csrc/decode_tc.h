@@ -19,7 +19,7 @@ struct TcInputs {
   const int32_t* ranks;        // device [2H][nb]
   const int64_t* row_offsets;  // device [2H][nb+1]
   uint32_t* status;
-  int pool_rows;
+  int64_t total_rows;  // rows of the factor arrays (Σ of every block's rank)
   const int32_t* host_ranks;  // [2H][nb]
 };
 
@@ -28,8 +28,9 @@ bool tc_shape_ok(const DecodeShape& s);
 bool tc_supported(const DecodeShape& s);
 int tc_launches(const DecodeShape& s);
 // ev0 / ev1 (optional) are recorded on `st` right before and right after the main decode kernel.
+// mask (optional, host [H][nb], nonzero = attended): block selection; the plan is rebuilt when it changes.
 cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, void* out, cudaStream_t st,
-                      cudaEvent_t ev0 = nullptr, cudaEvent_t ev1 = nullptr);
+                      cudaEvent_t ev0 = nullptr, cudaEvent_t ev1 = nullptr, const uint8_t* mask = nullptr);
 void tc_plan_destroy(TcPlan* plan);
 
 // The same decode with its scratch in a fixed device array (no allocation).  *too_large is set when

@@ -12,11 +12,13 @@ struct CompressShape {
   int d;       // head dim
   int n;       // block size
   int nb;      // blocks per pool
-  int R;       // total rank per pool (before capping at nb*d)
-  int pool_rows;  // min(R, nb*d)
+  int R;       // total rank of one allocation group: a pool, or with layer_scope all 2H pools (before capping)
+  int pool_rows;  // rows per pool, min(R, nb*d) (pool scope only)
   int r_min;
   int max_sweeps;
   bool bf16;
+  int rule = 0;             // 0 entropy, 1 greedy, 2 uniform, 3 caller weights
+  bool layer_scope = false; // one budget over all pools of the layer
 };
 
 struct CompressBuffers {
@@ -24,9 +26,11 @@ struct CompressBuffers {
   const void* V;
   float* gram;        // [2H][nb][d][d]
   float* eigvals;     // [2H][nb][d]
+  int32_t* sweeps;    // [2H][nb] Jacobi sweeps run per block (the last one found no pair to rotate)
   float* eigvecs;     // [2H][nb][d][d]
   double* entropy;    // [2H][nb]
   double* quotas;     // [2H][nb]
+  const double* weights;  // [2H][nb] device, rule 3 only
   int32_t* ranks;     // [2H][nb]
   int64_t* row_offsets;  // [2H][nb+1]
   void* tok;          // [2H*pool_rows][n]
@@ -34,11 +38,19 @@ struct CompressBuffers {
   uint32_t* status;
 };
 
-cudaError_t launch_compress(const CompressShape& s, const CompressBuffers& b, cudaStream_t st);
+// ev (optional, 5 events): recorded before the Gram, Jacobi, allocation and projection kernels and after the last.
+cudaError_t launch_compress(const CompressShape& s, const CompressBuffers& b, cudaStream_t st,
+                            const cudaEvent_t* ev = nullptr);
 // Tensor-core Gram of bf16 blocks (d in {64, 128}, n % 128 == 0); cudaErrorNotSupported otherwise.
 bool gram_tc_supported(const CompressShape& s);
 cudaError_t launch_gram_tc(const CompressShape& s, const void* K, const void* V, float* gram, uint32_t* status,
                            cudaStream_t st);
+
+// Tensor-core projection of bf16 blocks (d in {64, 128}, n % 128 == 0); cudaErrorNotSupported otherwise.
+bool project_tc_supported(const CompressShape& s);
+cudaError_t launch_project_tc(const CompressShape& s, const void* K, const void* V, const float* eigvecs,
+                              const int32_t* ranks, const int64_t* row_offsets, void* tok, void* dim,
+                              uint32_t* status, cudaStream_t st);
 
 // Rank-space decode on CUDA cores (any dtype; the fp32 path and a cross-check for bf16).
 struct DecodeShape {

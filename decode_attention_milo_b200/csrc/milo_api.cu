@@ -18,6 +18,8 @@ struct milo_factors {
   int H = 0;
   int64_t T = 0;
   int d = 0, n = 0, nb = 0, r_min = 0, R = 0, pool_rows = 0;
+  int64_t total_rows = 0;       // rows of the factor arrays: Σ of every block's rank
+  int rule = 0, scope = 0;      // allocation rule and budget scope (milo_alloc_rule, milo_pool_scope)
   int dtype = 0;
   uint32_t flags = 0;
   int32_t* ranks = nullptr;
@@ -26,6 +28,7 @@ struct milo_factors {
   void* dim = nullptr;
   uint32_t* status = nullptr;
   float* eigvals = nullptr;
+  int32_t* sweeps = nullptr;
   float* eigvecs = nullptr;
   double* entropy = nullptr;
   double* quotas = nullptr;
@@ -65,6 +68,7 @@ void free_all(milo_factors* f) {
   cudaFree(f->dim);
   cudaFree(f->status);
   cudaFree(f->eigvals);
+  cudaFree(f->sweeps);
   if (f->eigvecs) cudaFreeAsync(f->eigvecs, 0);
   cudaFree(f->entropy);
   cudaFree(f->quotas);
@@ -107,9 +111,11 @@ const char* milo_status_string(int32_t s) {
   }
 }
 
-milo_status milo_compress(const void* K, const void* V, int32_t dtype, int32_t num_kv_heads, int64_t context,
-                          int32_t head_dim, int32_t block_size, double budget, int32_t r_min,
-                          int32_t max_sweeps, uint32_t flags, void* stream, milo_factors** out) {
+static milo_status compress_impl(const void* K, const void* V, int32_t dtype, int32_t num_kv_heads,
+                                 int64_t context, int32_t head_dim, int32_t block_size, double budget,
+                                 int32_t r_min, int32_t max_sweeps, uint32_t flags, int32_t rule, int32_t scope,
+                                 const double* host_weights, void* stream, milo_factors** out,
+                                 const cudaEvent_t* ev) {
   if (!out) return MILO_ERR_INVALID_ARGUMENT;
   *out = nullptr;
   if (!K || !V) return MILO_ERR_INVALID_ARGUMENT;
@@ -117,9 +123,16 @@ milo_status milo_compress(const void* K, const void* V, int32_t dtype, int32_t n
   if (st != MILO_OK) return st;
   if (!(budget > 0.0) || !isfinite(budget) || max_sweeps < 0 || (flags & ~MILO_KEEP_INTERMEDIATES))
     return MILO_ERR_INVALID_ARGUMENT;
+  if (rule < MILO_ALLOC_ENTROPY || rule > MILO_ALLOC_WEIGHTS || (scope != MILO_POOL_HEAD && scope != MILO_POOL_LAYER))
+    return MILO_ERR_INVALID_ARGUMENT;
+  if ((rule == MILO_ALLOC_WEIGHTS) != (host_weights != nullptr)) return MILO_ERR_INVALID_ARGUMENT;
   const int nb = (int)(context / block_size);
-  // the allocation kernel keeps 28 bytes per block of a pool in shared memory
-  if (nb > kMaxAllocBlocks) return MILO_ERR_UNSUPPORTED;
+  const int P = 2 * num_kv_heads;
+  // the allocation kernel keeps 20 bytes per block of its group (a pool, or the layer) in shared memory
+  if ((scope == MILO_POOL_LAYER ? (int64_t)P * nb : nb) > kMaxAllocBlocks) return MILO_ERR_UNSUPPORTED;
+  if (host_weights)
+    for (int64_t i = 0; i < (int64_t)P * nb; ++i)
+      if (!(host_weights[i] > 0.0) || !isfinite(host_weights[i])) return MILO_ERR_INVALID_ARGUMENT;
   const double Rd = floor(budget * (double)(context * head_dim) / (double)(block_size + head_dim));
   if (Rd < (double)nb * r_min) return MILO_ERR_BUDGET;
   const int64_t full = (int64_t)nb * head_dim;
@@ -135,12 +148,15 @@ milo_status milo_compress(const void* K, const void* V, int32_t dtype, int32_t n
   f->nb = nb;
   f->r_min = r_min;
   f->R = R;
-  f->pool_rows = R;
+  f->pool_rows = scope == MILO_POOL_HEAD ? R : 0;
+  // with one budget over the layer the pools' rank sums differ, but they still total P·R (R is capped at nb·d)
+  f->total_rows = (int64_t)P * R;
+  f->rule = rule;
+  f->scope = scope;
   f->dtype = dtype;
   f->flags = flags;
-  const int P = 2 * num_kv_heads;
   f->host_ranks.assign((size_t)P * nb, 0);
-  const size_t rows = (size_t)P * f->pool_rows;
+  const size_t rows = (size_t)f->total_rows;
   const size_t nblk = (size_t)P * nb;
   const size_t dd = (size_t)head_dim * head_dim;
   float* gram = nullptr;
@@ -164,20 +180,36 @@ milo_status milo_compress(const void* K, const void* V, int32_t dtype, int32_t n
   ALLOC(f->dim, rows * head_dim * esize(dtype) + 256);
   ALLOC(f->status, sizeof(uint32_t));
   ALLOC(f->eigvals, nblk * head_dim * sizeof(float));
+  ALLOC(f->sweeps, nblk * sizeof(int32_t));
   if ((e = cudaMallocAsync((void**)&f->eigvecs, nblk * dd * sizeof(float), s)) != cudaSuccess) return fail(e);
   ALLOC(f->entropy, nblk * sizeof(double));
   ALLOC(f->quotas, nblk * sizeof(double));
   if ((e = cudaMallocAsync((void**)&gram, nblk * dd * sizeof(float), s)) != cudaSuccess) return fail(e);
+  double* d_weights = nullptr;
+  if (host_weights) {
+    if ((e = cudaMallocAsync((void**)&d_weights, nblk * sizeof(double), s)) != cudaSuccess) return fail(e);
+    // pageable source: the copy is staged before the call returns, so the caller may reuse host_weights
+    if ((e = cudaMemcpyAsync(d_weights, host_weights, nblk * sizeof(double), cudaMemcpyHostToDevice, s)) !=
+        cudaSuccess) {
+      cudaFreeAsync(d_weights, s);
+      return fail(e);
+    }
+  }
 #undef ALLOC
   if ((e = cudaMemsetAsync(f->status, 0, sizeof(uint32_t), s)) != cudaSuccess) return fail(e);
   if ((e = cudaMemsetAsync(f->tok, 0, rows * block_size * esize(dtype) + 256, s)) != cudaSuccess) return fail(e);
   if ((e = cudaMemsetAsync(f->dim, 0, rows * head_dim * esize(dtype) + 256, s)) != cudaSuccess) return fail(e);
 
-  milo::CompressShape cs{num_kv_heads, context, head_dim, block_size, nb, R, f->pool_rows, r_min,
-                         max_sweeps ? max_sweeps : 30, dtype == MILO_BF16};
-  milo::CompressBuffers cb{K, V, gram, f->eigvals, f->eigvecs, f->entropy, f->quotas, f->ranks,
-                           f->row_offsets, f->tok, f->dim, f->status};
-  if ((e = milo::launch_compress(cs, cb, s)) != cudaSuccess) return fail(e);
+  milo::CompressShape cs{num_kv_heads, context, head_dim, block_size, nb,
+                         scope == MILO_POOL_LAYER ? P * R : R, R, r_min, max_sweeps ? max_sweeps : 30,
+                         dtype == MILO_BF16, rule, scope == MILO_POOL_LAYER};
+  milo::CompressBuffers cb{K, V, gram, f->eigvals, f->sweeps, f->eigvecs, f->entropy, f->quotas, d_weights,
+                           f->ranks, f->row_offsets, f->tok, f->dim, f->status};
+  if ((e = milo::launch_compress(cs, cb, s, ev)) != cudaSuccess) {
+    if (d_weights) cudaFreeAsync(d_weights, s);
+    return fail(e);
+  }
+  if (d_weights) cudaFreeAsync(d_weights, s);
   if ((e = cudaEventCreateWithFlags(&f->ready, cudaEventDisableTiming)) != cudaSuccess) return fail(e);
   if ((e = cudaEventRecord(f->ready, s)) != cudaSuccess) return fail(e);
   // The Gram scratch (and, unless kept, the eigenpairs) are released once the stream has used them.
@@ -191,6 +223,32 @@ milo_status milo_compress(const void* K, const void* V, int32_t dtype, int32_t n
   return MILO_OK;
 }
 
+milo_status milo_compress(const void* K, const void* V, int32_t dtype, int32_t num_kv_heads, int64_t context,
+                          int32_t head_dim, int32_t block_size, double budget, int32_t r_min,
+                          int32_t max_sweeps, uint32_t flags, void* stream, milo_factors** out) {
+  return compress_impl(K, V, dtype, num_kv_heads, context, head_dim, block_size, budget, r_min, max_sweeps, flags,
+                       MILO_ALLOC_ENTROPY, MILO_POOL_HEAD, nullptr, stream, out, nullptr);
+}
+
+milo_status milo_compress_rule(const void* K, const void* V, int32_t dtype, int32_t num_kv_heads, int64_t context,
+                               int32_t head_dim, int32_t block_size, double budget, int32_t r_min,
+                               int32_t max_sweeps, uint32_t flags, int32_t rule, int32_t scope,
+                               const double* host_weights, void* stream, milo_factors** out) {
+  return compress_impl(K, V, dtype, num_kv_heads, context, head_dim, block_size, budget, r_min, max_sweeps, flags,
+                       rule, scope, host_weights, stream, out, nullptr);
+}
+
+milo_status milo_compress_profiled(const void* K, const void* V, int32_t dtype, int32_t num_kv_heads,
+                                   int64_t context, int32_t head_dim, int32_t block_size, double budget,
+                                   int32_t r_min, int32_t max_sweeps, uint32_t flags, void* stream,
+                                   milo_factors** out, void* const* events) {
+  cudaEvent_t ev[5] = {};
+  if (events)
+    for (int k = 0; k < 5; ++k) ev[k] = static_cast<cudaEvent_t>(events[k]);
+  return compress_impl(K, V, dtype, num_kv_heads, context, head_dim, block_size, budget, r_min, max_sweeps, flags,
+                       MILO_ALLOC_ENTROPY, MILO_POOL_HEAD, nullptr, stream, out, ev);
+}
+
 milo_status milo_factors_import(int32_t dtype, int32_t num_kv_heads, int64_t context, int32_t head_dim,
                                 int32_t block_size, int32_t r_min, const int32_t* host_ranks,
                                 const void* host_tok, const void* host_dim, void* stream, milo_factors** out) {
@@ -201,7 +259,8 @@ milo_status milo_factors_import(int32_t dtype, int32_t num_kv_heads, int64_t con
   if (st != MILO_OK) return st;
   const int nb = (int)(context / block_size);
   const int P = 2 * num_kv_heads;
-  int pool_rows = -1;
+  int64_t total = 0;
+  int pool_rows = -1;  // the common rank sum of the pools, or 0 when they differ
   for (int p = 0; p < P; ++p) {
     int64_t sum = 0;
     for (int b = 0; b < nb; ++b) {
@@ -209,8 +268,9 @@ milo_status milo_factors_import(int32_t dtype, int32_t num_kv_heads, int64_t con
       if (r < 1 || r > head_dim) return MILO_ERR_INVALID_ARGUMENT;
       sum += r;
     }
+    total += sum;
     if (pool_rows < 0) pool_rows = (int)sum;
-    if (sum != pool_rows) return MILO_ERR_INVALID_ARGUMENT;
+    else if (sum != pool_rows) pool_rows = 0;
   }
   milo_factors* f = new (std::nothrow) milo_factors();
   if (!f) return MILO_ERR_OUT_OF_MEMORY;
@@ -223,11 +283,13 @@ milo_status milo_factors_import(int32_t dtype, int32_t num_kv_heads, int64_t con
   f->r_min = r_min;
   f->R = pool_rows;
   f->pool_rows = pool_rows;
+  f->total_rows = total;
+  f->scope = pool_rows ? MILO_POOL_HEAD : MILO_POOL_LAYER;
   f->dtype = dtype;
-  const size_t rows = (size_t)P * pool_rows;
+  const size_t rows = (size_t)total;
   std::vector<int64_t> offs((size_t)P * (nb + 1));
+  int64_t o = 0;
   for (int p = 0; p < P; ++p) {
-    int64_t o = (int64_t)p * pool_rows;
     for (int b = 0; b < nb; ++b) {
       offs[(size_t)p * (nb + 1) + b] = o;
       o += host_ranks[(size_t)p * nb + b];
@@ -285,12 +347,16 @@ milo_status milo_factors_describe(const milo_factors* f, milo_factors_desc* d) {
   d->r_min = f->r_min;
   d->pool_rows = f->pool_rows;
   d->dtype = f->dtype;
+  d->alloc_rule = f->rule;
+  d->pool_scope = f->scope;
+  d->total_rows = f->total_rows;
   d->ranks = f->ranks;
   d->row_offsets = f->row_offsets;
   d->tok = f->tok;
   d->dim = f->dim;
   const bool keep = f->flags & MILO_KEEP_INTERMEDIATES;
   d->eigvals = keep ? f->eigvals : nullptr;
+  d->sweeps = f->sweeps;
   d->eigvecs = keep ? f->eigvecs : nullptr;
   d->entropy = keep ? f->entropy : nullptr;
   d->quotas = keep ? f->quotas : nullptr;
@@ -341,13 +407,21 @@ int32_t milo_decode_launches(const milo_factors* f, int32_t batch, int32_t num_q
 
 static milo_status decode_impl(const void* q, int32_t batch, int32_t num_q_heads, const milo_factors* fc,
                                const void* K_suffix, const void* V_suffix, int32_t suffix_len, float scale,
-                               void* out, void* stream, cudaEvent_t ev0, cudaEvent_t ev1) {
+                               void* out, void* stream, cudaEvent_t ev0, cudaEvent_t ev1,
+                               const uint8_t* mask = nullptr) {
   if (!fc || !q || !out || batch <= 0 || num_q_heads <= 0 || suffix_len < 0) return MILO_ERR_INVALID_ARGUMENT;
   milo_factors* f = const_cast<milo_factors*>(fc);
   if (num_q_heads % f->H != 0) return MILO_ERR_INVALID_ARGUMENT;
   if (suffix_len > 0 && (!K_suffix || !V_suffix)) return MILO_ERR_INVALID_ARGUMENT;
   if (!(scale == scale) || isinf(scale)) return MILO_ERR_INVALID_ARGUMENT;
   if (batch > 65535 || num_q_heads > 4096 || suffix_len > (1 << 20)) return MILO_ERR_INVALID_ARGUMENT;
+  if (mask && suffix_len == 0) {  // a head with no selected block and no suffix has nothing to attend
+    for (int h = 0; h < f->H; ++h) {
+      bool any = false;
+      for (int b = 0; b < f->nb && !any; ++b) any = mask[(size_t)h * f->nb + b] != 0;
+      if (!any) return MILO_ERR_INVALID_ARGUMENT;
+    }
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)f->d);
   std::lock_guard<std::mutex> lock(f->mu);
@@ -366,9 +440,10 @@ static milo_status decode_impl(const void* q, int32_t batch, int32_t num_q_heads
       f->host_ranks_valid = true;
     }
     milo::TcInputs in{q,        K_suffix, V_suffix,     f->tok,       f->dim,
-                      f->ranks, f->row_offsets, f->status, f->pool_rows, f->host_ranks.data()};
-    return cuda_status(milo::tc_decode(&f->tc_plan, ds, in, out, s, ev0, ev1));
+                      f->ranks, f->row_offsets, f->status, f->total_rows, f->host_ranks.data()};
+    return cuda_status(milo::tc_decode(&f->tc_plan, ds, in, out, s, ev0, ev1, mask));
   }
+  if (mask) return MILO_ERR_UNSUPPORTED;  // block selection runs on the bf16 tensor-core decode
   const size_t need = milo::simt_decode_partials_floats(ds);
   if (need > f->partials_floats) {
     MILO_CUDA(cudaStreamSynchronize(s));
@@ -414,11 +489,19 @@ milo_status milo_decode_attn_noalloc(const void* q, int32_t batch, int32_t num_q
   MILO_CUDA(cudaStreamIsCapturing(s, &cap));
   if (cap == cudaStreamCaptureStatusNone) MILO_CUDA(cudaStreamWaitEvent(s, f->ready, 0));
   milo::TcInputs in{q,        K_suffix, V_suffix,     f->tok,       f->dim,
-                    f->ranks, f->row_offsets, f->status, f->pool_rows, f->host_ranks.data()};
+                    f->ranks, f->row_offsets, f->status, f->total_rows, f->host_ranks.data()};
   bool too_large = false;
   const cudaError_t e = milo::tc_decode_noalloc(ds, in, out, s, &too_large);
   if (too_large) return MILO_ERR_UNSUPPORTED;
   return cuda_status(e);
+}
+
+milo_status milo_decode_attn_select(const void* q, int32_t batch, int32_t num_q_heads, const milo_factors* f,
+                                    const void* K_suffix, const void* V_suffix, int32_t suffix_len, float scale,
+                                    const uint8_t* host_block_mask, void* out, void* stream) {
+  if (!host_block_mask) return MILO_ERR_INVALID_ARGUMENT;
+  return decode_impl(q, batch, num_q_heads, f, K_suffix, V_suffix, suffix_len, scale, out, stream, nullptr,
+                     nullptr, host_block_mask);
 }
 
 milo_status milo_decode_attn_profiled(const void* q, int32_t batch, int32_t num_q_heads, const milo_factors* f,

@@ -36,9 +36,10 @@
  *          U_b = X_b·B_b (X_b the n×d block) transposed and cut into
  *          128-token slabs, element (j, t) at
  *          row0·n + (t / 128)·(r·128) + j·128 + (t % 128)
- *   so that X_b ≈ U_b · B_bᵀ.  The blocks of a pool are consecutive and pool p
- *   starts at row p * pool_rows.  Factor elements have the dtype of the
- *   compressed cache.
+ *   so that X_b ≈ U_b · B_bᵀ.  The blocks of a pool are consecutive and the
+ *   pools follow each other (pool p starts at row p * pool_rows when every pool
+ *   has the same rank sum).  Factor elements have the dtype of the compressed
+ *   cache.
  */
 #ifndef MILO_H_
 #define MILO_H_
@@ -49,7 +50,7 @@
 extern "C" {
 #endif
 
-#define MILO_ABI_VERSION 1
+#define MILO_ABI_VERSION 2
 
 typedef enum {
   MILO_OK = 0,
@@ -69,6 +70,19 @@ typedef enum { MILO_F32 = 0, MILO_BF16 = 1 } milo_dtype;
 
 typedef struct milo_factors milo_factors; /* opaque, device-resident, library-owned */
 
+/* Allocation rules (milo_compress_rule): the entropy rule of §4.3, the greedy marginal-gain
+ * form §4.3 describes in words, and the uniform and random baselines of §5.3 (random: the
+ * caller draws the weights and passes them in). */
+typedef enum {
+  MILO_ALLOC_ENTROPY = 0, /* ranks ∝ exp(H_b), water-filling, largest remainder (milo_compress) */
+  MILO_ALLOC_GREEDY = 1,  /* from r_min, each unit to the largest next-component energy share */
+  MILO_ALLOC_UNIFORM = 2, /* floor(R / blocks) each, the remainder to the lowest block indices */
+  MILO_ALLOC_WEIGHTS = 3  /* ranks ∝ caller weights, with the entropy rule's water-filling */
+} milo_alloc_rule;
+/* Budget scope: R = floor(budget*T*d/(n+d)) rank units per pool (one KV head's keys or values),
+ * or P·R units shared by all P = 2H pools of the layer (blocks ordered pool p = 2h + t, then block). */
+typedef enum { MILO_POOL_HEAD = 0, MILO_POOL_LAYER = 1 } milo_pool_scope;
+
 typedef struct {
   int32_t num_kv_heads;  /* H */
   int32_t num_blocks;    /* nb = context / block_size */
@@ -76,9 +90,12 @@ typedef struct {
   int32_t head_dim;      /* d */
   int64_t context;       /* T */
   int32_t r_min;
-  int32_t pool_rows;     /* rows per pool = min(R, nb*d), R = floor(budget*T*d/(n+d)) */
+  int32_t pool_rows;     /* rows per pool = min(R, nb*d), R = floor(budget*T*d/(n+d)); 0 if pools differ */
   int32_t dtype;         /* milo_dtype */
+  int32_t alloc_rule;    /* milo_alloc_rule */
+  int32_t pool_scope;    /* milo_pool_scope */
   int32_t reserved;
+  int64_t total_rows;    /* rows of tok (in units of n) and dim: Σ of every block's rank */
   const int32_t* ranks;       /* device [2H][nb]                         */
   const int64_t* row_offsets; /* device [2H][nb+1]                       */
   const void* tok;            /* device, 2H*pool_rows*n elements (slabs)  */
@@ -88,6 +105,9 @@ typedef struct {
   const float* eigvecs;       /* device [2H][nb][d][d], row i = eigenvector of λ_i      */
   const double* entropy;      /* device [2H][nb], H_b                                  */
   const double* quotas;       /* device [2H][nb], real quotas before rounding          */
+  /* present for objects made by milo_compress (NULL for imported ones): */
+  const int32_t* sweeps;      /* device [2H][nb], Jacobi sweeps run per block (the last  */
+                              /* one rotated no pair; max_sweeps means no convergence)    */
 } milo_factors_desc;
 
 /*
@@ -119,6 +139,41 @@ milo_status milo_compress(const void* K, const void* V, int32_t dtype, int32_t n
                           milo_factors** out);
 
 /*
+ * milo_compress_rule — milo_compress with a chosen allocation rule and budget
+ * scope (§4.3's greedy form, §5.3's uniform and random baselines, and a
+ * layer-wide budget; see milo_alloc_rule and milo_pool_scope).  The Gram,
+ * eigen-decomposition and projection steps are those of milo_compress.
+ *   rule          milo_alloc_rule.
+ *   scope         milo_pool_scope; MILO_POOL_LAYER allocates one budget of
+ *                 2H·R units over all 2H·nb blocks (at most 8192 blocks).
+ *   host_weights  host [2H][nb], finite and > 0, for MILO_ALLOC_WEIGHTS only
+ *                 (NULL otherwise); copied before the call returns.
+ * The greedy rule takes its decisions on the fp32 eigenvalues in fp64 (shares
+ * λ_i/Σλ); the quotas intermediate is NaN for the greedy and uniform rules.
+ * Other arguments, results and errors as milo_compress.
+ */
+milo_status milo_compress_rule(const void* K, const void* V, int32_t dtype, int32_t num_kv_heads,
+                               int64_t context, int32_t head_dim, int32_t block_size, double budget,
+                               int32_t r_min, int32_t max_sweeps, uint32_t flags, int32_t rule,
+                               int32_t scope, const double* host_weights, void* stream,
+                               milo_factors** out);
+
+/*
+ * milo_compress_profiled — milo_compress that also records caller-created CUDA
+ * events (cudaEvent_t passed as void*) on `stream` between its kernels:
+ * events[0] before the Gram kernel, events[1] before the Jacobi eigensolver,
+ * events[2] before the entropy and rank allocation kernel, events[3] before the
+ * projection kernel and events[4] after it, so cudaEventElapsedTime between
+ * neighbours gives each step's duration.  `events` is host memory, 5 entries,
+ * any of them NULL (not recorded); events itself may be NULL.  Same arguments,
+ * results and errors as milo_compress otherwise.
+ */
+milo_status milo_compress_profiled(const void* K, const void* V, int32_t dtype, int32_t num_kv_heads,
+                                   int64_t context, int32_t head_dim, int32_t block_size, double budget,
+                                   int32_t r_min, int32_t max_sweeps, uint32_t flags, void* stream,
+                                   milo_factors** out, void* const* events);
+
+/*
  * milo_decode_attn — one decode step of softmax attention over the compressed
  * prefix and each query's uncompressed suffix.
  * Source: §4.4 (inference attends over the stored low-rank caches).  Every
@@ -142,6 +197,25 @@ milo_status milo_compress(const void* K, const void* V, int32_t dtype, int32_t n
 milo_status milo_decode_attn(const void* q, int32_t batch, int32_t num_q_heads,
                              const milo_factors* f, const void* K_suffix, const void* V_suffix,
                              int32_t suffix_len, float scale, void* out, void* stream);
+
+/*
+ * milo_decode_attn_select — milo_decode_attn over a selection of the
+ * compressed blocks.  Source: §4.4 (decoding retrieves the selected blocks and
+ * attends over them sparsely).  The blocks of KV head h that the mask leaves
+ * out take no part in the softmax of any query of that head; the suffix is
+ * always attended.
+ *   host_block_mask  host [H][nb], nonzero = attend; read during the call only.
+ * The selection is applied through the work list: a call whose mask differs
+ * from the previous call's on this factor object rebuilds it (one host-to-
+ * device copy, and scratch allocation when it grows), so a fixed selection
+ * costs nothing extra.  bf16 factors only (MILO_ERR_UNSUPPORTED for fp32).
+ * MILO_ERR_INVALID_ARGUMENT when suffix_len == 0 and some head selects no
+ * block.  Other arguments, results and errors as milo_decode_attn.
+ */
+milo_status milo_decode_attn_select(const void* q, int32_t batch, int32_t num_q_heads,
+                                    const milo_factors* f, const void* K_suffix, const void* V_suffix,
+                                    int32_t suffix_len, float scale, const uint8_t* host_block_mask,
+                                    void* out, void* stream);
 
 /*
  * milo_decode_attn_profiled — milo_decode_attn that also records two caller-created
@@ -234,9 +308,9 @@ milo_status milo_factors_status(const milo_factors* f, uint32_t* host_bits);
 
 /*
  * Builds a factor object from host arrays in the layout above (a copy), e.g.
- * factors computed elsewhere or saved earlier.  host_ranks [2H][nb];
- * host_tok [2H*pool_rows][n] and host_dim [2H*pool_rows][d] in `dtype`, with
- * pool_rows = Σ of each pool's ranks (all pools must have the same sum);
+ * factors computed elsewhere or saved earlier.  host_ranks [2H][nb], each in
+ * [1, d]; host_tok [rows][n] and host_dim [rows][d] in `dtype`, rows = Σ of all
+ * ranks, pools in order (their sums may differ, as with a layer-wide budget);
  * host_tok holds each block's 128-token slabs as described above.
  * Synchronises `stream`.
  */
