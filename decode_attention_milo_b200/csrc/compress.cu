@@ -190,6 +190,185 @@ __global__ void __launch_bounds__(kJThreads) jacobi_kernel(const float* __restri
   }
 }
 
+// Eigen-decomposition of G_b by one-sided Jacobi preconditioned with a pivoted Cholesky factor
+// (the preconditioning of Demmel–Veselić and Drmač for Jacobi SVD): G = L̃ L̃ᵀ with L̃ the Cholesky
+// factor under diagonal pivoting, its rows kept in the original index order; then one-sided Jacobi
+// orthogonalises the columns of L̃, L̃·U = B·Σ, so that G = (L̃U)(L̃U)ᵀ = B Σ² Bᵀ: the eigenvalues are the
+// squared column norms and the eigenvectors the normalised columns, already in the original order.
+// The rows of the pivoted factor are graded and nearly orthogonal, so the sweeps are few, and no
+// accumulated rotation matrix is needed (the columns themselves become the eigenvectors).  Pivots below a
+// floor far under fp32 resolution (1e-9 of the mean diagonal) are raised to it, so that a rank-deficient
+// block still yields an orthonormal basis.
+constexpr int kEThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kEThreads, 3) eig_kernel(const float* __restrict__ gram, int nb, int max_sweeps,
+                                                       float* __restrict__ eigvals, float* __restrict__ eigvecs,
+                                                       int32_t* __restrict__ sweeps_out, uint32_t* status) {
+  constexpr int E = D / 32;           // elements per lane of one column
+  constexpr int NW = kEThreads / 32;  // warps
+  constexpr int PP = (D / 2) / NW;    // column pairs per warp per round
+  constexpr int PG = PP < 4 ? PP : 4; // pairs handled together (their loads and reductions overlap)
+  extern __shared__ float smem[];
+  float* A = smem;              // column-major [D][D]: the Schur complement, then the columns of L̃
+  float* nrm = A + D * D;       // [D] squared column norms during the sweeps
+  int* done = reinterpret_cast<int*>(nrm + D);  // [D] index already pivoted
+  __shared__ float s_floor;
+  __shared__ int s_piv;
+  const int bidx = blockIdx.x + blockIdx.y * nb;
+  const float* Gg = gram + (int64_t)bidx * D * D;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int e = threadIdx.x; e < D * D; e += kEThreads) A[e] = Gg[e];
+  for (int i = threadIdx.x; i < D; i += kEThreads) done[i] = 0;
+  __syncthreads();
+  if (warp == 0) {
+    float tr = 0.f;
+    for (int i = lane; i < D; i += 32) tr += fmaxf(A[i * D + i], 0.f);
+    tr = warp_sum(tr);
+    if (lane == 0) s_floor = fmaxf(1e-9f * tr / D, 1e-30f);
+  }
+  // ---- pivoted Cholesky, in place
+  for (int k = 0; k < D; ++k) {
+    if (warp == 0) {
+      float best = -INFINITY;
+      int bi = 0;
+      for (int i = lane; i < D; i += 32) {
+        const float v = done[i] ? -INFINITY : A[i * D + i];
+        if (v > best) {
+          best = v;
+          bi = i;
+        }
+      }
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ob > best || (ob == best && oi < bi)) {
+          best = ob;
+          bi = oi;
+        }
+      }
+      if (lane == 0) s_piv = bi;
+    }
+    __syncthreads();
+    const int p = s_piv;
+    const float piv = fmaxf(A[p * D + p], s_floor);
+    const float l = sqrtf(piv), il = 1.f / l;
+    __syncthreads();  // every thread has read the pivot before column p changes
+    // column p becomes column k of L̃: remaining rows scaled, the pivot row l, eliminated rows 0
+    for (int i = threadIdx.x; i < D; i += kEThreads) {
+      float* a = &A[p * D + i];
+      *a = i == p ? l : (done[i] ? 0.f : *a * il);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) done[p] = 1;
+    // Schur complement of the remaining indices: A[i][j] -= L̃[i][k] L̃[j][k]
+    for (int e = threadIdx.x; e < D * D; e += kEThreads) {
+      const int j = e / D, i = e % D;
+      if (j == p || i == p) continue;
+      const float li = A[p * D + i], lj = A[p * D + j];
+      if (li != 0.f && lj != 0.f) A[e] = fmaf(-li, lj, A[e]);
+    }
+    __syncthreads();
+  }
+  // every column has now been pivoted: the columns of A are the columns of L̃ (in pivot order)
+  // ---- one-sided Jacobi on the columns of L̃ (round-robin pairs), norms carried along
+  for (int j = warp; j < D; j += NW) {
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) ss = fmaf(A[j * D + lane + 32 * e], A[j * D + lane + 32 * e], ss);
+    ss = warp_sum(ss);
+    if (lane == 0) nrm[j] = ss;
+  }
+  __syncthreads();
+  bool converged = false;
+  int sweeps_run = 0;
+  for (int sweep = 0; sweep < max_sweeps; ++sweep) {
+    ++sweeps_run;
+    int rotated = 0;
+    for (int s = 0; s < D - 1; ++s) {
+#pragma unroll 1
+      for (int g0 = 0; g0 < PP; g0 += PG) {
+        float ap[PG][E], aq[PG][E], ga[PG];
+        int pj[PG], qj[PG];
+#pragma unroll
+        for (int t = 0; t < PG; ++t) {
+          // round-robin pair k of round s without a division: (s, D-1) for k = 0, else (s+k, s-k) mod D-1
+          const int k = warp + (g0 + t) * NW, m = D - 1;
+          int pp = s + k, qq = s - k;
+          if (pp >= m) pp -= m;
+          if (qq < 0) qq += m;
+          pj[t] = k == 0 ? s : pp;
+          qj[t] = k == 0 ? m : qq;
+          ga[t] = 0.f;
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            ap[t][e] = A[pj[t] * D + lane + 32 * e];
+            aq[t][e] = A[qj[t] * D + lane + 32 * e];
+            ga[t] = fmaf(ap[t][e], aq[t][e], ga[t]);
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+          for (int t = 0; t < PG; ++t) ga[t] += __shfl_xor_sync(0xffffffffu, ga[t], o);
+#pragma unroll
+        for (int t = 0; t < PG; ++t) {
+          const int p = pj[t], q = qj[t];
+          const float al = nrm[p], be = nrm[q];
+          if (ga[t] != 0.f && fabsf(ga[t]) > kJacobiTol * sqrtf(al) * sqrtf(be)) {
+            const float zeta = (be - al) / (2.f * ga[t]);
+            const float tn = (zeta >= 0.f ? 1.f : -1.f) / (fabsf(zeta) + sqrtf(1.f + zeta * zeta));
+            const float c = 1.f / sqrtf(1.f + tn * tn);
+            const float sn = c * tn, tau = sn / (1.f + c);
+            // the rotation written as a correction of each column (a_p − s(a_q + τa_p), a_q + s(a_p − τa_q),
+            // τ = s / (1 + c)): its rounding scales with the correction, not with the column, so that the many
+            // small late rotations do not drift the column norms (the eigenvalues)
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+              A[p * D + lane + 32 * e] = ap[t][e] - sn * fmaf(tau, ap[t][e], aq[t][e]);
+              A[q * D + lane + 32 * e] = aq[t][e] + sn * fmaf(-tau, aq[t][e], ap[t][e]);
+            }
+            __syncwarp();
+            if (lane == 0) {
+              nrm[p] = al - tn * ga[t];
+              nrm[q] = be + tn * ga[t];
+            }
+            rotated = 1;
+          }
+        }
+      }
+      __syncthreads();
+    }
+    // exact norms again (the carried ones drift by rounding)
+    for (int j = warp; j < D; j += NW) {
+      float ss = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) ss = fmaf(A[j * D + lane + 32 * e], A[j * D + lane + 32 * e], ss);
+      ss = warp_sum(ss);
+      if (lane == 0) nrm[j] = ss;
+    }
+    if (!__syncthreads_or(rotated)) {
+      converged = true;
+      break;
+    }
+  }
+  if (!converged && threadIdx.x == 0) atomicOr(status, kStatusNoConvergence);
+  if (threadIdx.x == 0) sweeps_out[bidx] = sweeps_run;
+  // eigenvalue λ_j = |column j|², eigenvector = column j / |column j|; sorted descending (ties: lower column)
+  for (int j = warp; j < D; j += NW) {
+    const float lj = nrm[j];
+    int rank = 0;
+    for (int i = lane; i < D; i += 32) rank += (nrm[i] > lj) || (nrm[i] == lj && i < j);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+    if (lane == 0) eigvals[(int64_t)bidx * D + rank] = lj;
+    const float inv = lj > 0.f ? rsqrtf(lj) : 0.f;
+    float* dst = eigvecs + ((int64_t)bidx * D + rank) * D;
+#pragma unroll
+    for (int e = 0; e < E; ++e) dst[lane + 32 * e] = A[j * D + lane + 32 * e] * inv;
+  }
+}
+
 // ---------------------------------------------------------------- alloc
 __device__ __forceinline__ double clampd(double x, double lo, double hi) { return fmin(fmax(x, lo), hi); }
 
@@ -468,12 +647,12 @@ cudaError_t run(const CompressShape& s, const CompressBuffers& bf, cudaStream_t 
   } else if (ge != cudaSuccess) {
     return ge;
   }
-  const size_t jsm = (2 * D * D + D) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(jacobi_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)jsm);
+  const size_t jsm = (size_t)D * D * sizeof(float) + D * (sizeof(float) + sizeof(int));
+  cudaError_t e = cudaFuncSetAttribute(eig_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)jsm);
   if (e != cudaSuccess) return e;
   if ((e = mark(1)) != cudaSuccess) return e;
-  jacobi_kernel<D><<<grid, kJThreads, jsm, st>>>(bf.gram, s.nb, s.max_sweeps, bf.eigvals, bf.eigvecs, bf.sweeps,
-                                                 bf.status);
+  eig_kernel<D><<<grid, kEThreads, jsm, st>>>(bf.gram, s.nb, s.max_sweeps, bf.eigvals, bf.eigvecs, bf.sweeps,
+                                              bf.status);
   const int ngroup = s.layer_scope ? 2 * s.H * s.nb : s.nb;
   const size_t asm_ = (size_t)ngroup * (2 * sizeof(double) + sizeof(int));
   e = cudaFuncSetAttribute(alloc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asm_);

@@ -58,6 +58,7 @@ constexpr int kRingBytes = 122880;  // TMA ring: variable-size items, each one c
 constexpr int kItemSlots = 16;       // items in flight at most (one FULL/EMPTY barrier pair each)
 constexpr int kChunk = 128;          // tokens per score chunk
 constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr uint32_t kSleepNs = 2000;  // suspend-time hint of one try_wait in a wait loop
 
 // shared-memory map (bytes from a 1024-aligned base)
 constexpr int kOffQ = 0;          // [cb][128 rows][128 B]  query rows, K-major over d
@@ -77,6 +78,7 @@ constexpr uint32_t kTmAcc = 0, kTmS0 = 128, kTmA = 384;
 // TMEM column, relative to its region, of k-step t (16 bf16) of an A operand that the two softmax
 // warpgroups packed in place: warpgroup w holds K indices [64w, 64w + 64) in columns [64w, 64w + 32).
 __device__ __forceinline__ uint32_t ta_col(int t) { return (uint32_t)(64 * (t >> 2) + 8 * (t & 3)); }
+
 
 enum Bar {
   B_FULL = 0,
@@ -101,9 +103,10 @@ struct Seg {
   int pad;
 };
 
+struct CtaRec;
 struct Params {
   const Seg* segs;
-  const int* seg_first;  // [grid + 1]
+  const CtaRec* recs;    // [grid]
   const int32_t* ranks;
   const int64_t* row_offsets;
   float* part_acc;  // [pid][128][D]
@@ -119,13 +122,12 @@ struct BlockInfo {
   int64_t rowk, rowv;
 };
 
-// Tensor maps of one row-major bf16 operand array (rows of 64 or 128 columns): 2D maps with boxes of
-// 16, 32, 64 and 128 rows × 64 columns, and for 128-column arrays 3D maps (x: 64 columns, y: rows,
-// z: the two 64-column blocks) whose box of h rows × both column blocks lands in shared memory as
-// [column block][h][128 B], one instruction for a whole item.
+// Tensor maps of one row-major bf16 operand array (rows of 64 or 128 columns), one per item height
+// h = 16, 32, ..., 128 rows, so that every item is a single TMA instruction: for 128-column arrays 3D maps
+// (x: 64 columns, y: rows, z: the two 64-column blocks) whose box of h rows × both column blocks lands in
+// shared memory as [column block][h][128 B]; for 64-column arrays 2D boxes of h rows × 64 columns.
 struct RowMaps {
-  CUtensorMap m2[4];
-  CUtensorMap m3[4];
+  CUtensorMap m[8];
 };
 struct Maps {
   RowMaps tok, dim, ksuf, vsuf;  // the suffix maps use the 128-row boxes only
@@ -133,27 +135,46 @@ struct Maps {
   CUtensorMap pacc;  // partial accumulators [segments · 128][d] fp32, boxes of 128 rows × 32 columns
 };
 
-__device__ __forceinline__ const CUtensorMap* map_of(const RowMaps& m, bool three_d, int hi) {
+__device__ __forceinline__ const CUtensorMap* map_of(const RowMaps& m, int k) {
   // constant indices: the result stays an address in the kernel-parameter space
-  if (three_d) return hi == 0 ? &m.m3[0] : hi == 1 ? &m.m3[1] : hi == 2 ? &m.m3[2] : &m.m3[3];
-  return hi == 0 ? &m.m2[0] : hi == 1 ? &m.m2[1] : hi == 2 ? &m.m2[2] : &m.m2[3];
+  switch (k) {
+    case 0: return &m.m[0];
+    case 1: return &m.m[1];
+    case 2: return &m.m[2];
+    case 3: return &m.m[3];
+    case 4: return &m.m[4];
+    case 5: return &m.m[5];
+    case 6: return &m.m[6];
+    default: return &m.m[7];
+  }
 }
 
-// Per-CTA state in shared memory: the CTA's segments and the rank / row offset of every block they
-// touch, staged once at start so that no role reads them from global memory inside the pipeline.
+// One CTA's work, built on the host: its segments and the rank / row offset of every block they touch, in
+// the order the roles walk them.  The CTA copies it to shared memory with one coalesced load at start, so
+// that no role reads a table from global memory inside the pipeline.
+struct CtaRec {
+  int nseg;        // segments staged (0 when they did not fit: the roles read the global tables)
+  int nblk;        // blocks staged
+  int s_begin, s_end;          // the CTA's range in the global segment list
+  int blk0[kMaxSegsSmem + 1];  // first block entry of each segment
+  int pad[3];
+  Seg segs[kMaxSegsSmem];
+  BlockInfo blocks[kMaxBlocksSmem];
+};
+static_assert(sizeof(CtaRec) % 16 == 0, "records are copied in 16-byte words");
+
+// Per-CTA state in shared memory.
 struct Shared {
   uint32_t tmem_base;
   int abort_flag;
-  int nseg;        // segments of this CTA staged (0 when they did not fit: roles read global memory)
-  int nblk;        // blocks staged
-  int blk0[kMaxSegsSmem + 1];  // first table entry of each segment
-  Seg segs[kMaxSegsSmem];
-  BlockInfo blocks[kMaxBlocksSmem];
+  int pad[2];
+  CtaRec rec;
   uint32_t pos_log[kItemSlots], len_log[kItemSlots];  // producer's record of the items in flight
   float mx_x[2][2][128];  // row maxima exchanged by the two softmax warpgroups (double-buffered)
   float l_x[128];         // warpgroup 1's row sums at a segment's end
 };
-static_assert(8 * B_COUNT + 64 + sizeof(Shared) <= kBarRegion, "barrier region too small");
+constexpr int kSharedOff = (8 * B_COUNT + 64 + 15) & ~15;  // 16-byte aligned for the record copy
+static_assert(kSharedOff + sizeof(Shared) <= kBarRegion, "barrier region too small");
 
 // Warp-collective bounded wait on an mbarrier phase (all 32 lanes call it together; the result is uniform).
 // Gives up after kWaitNs, records kStatusDecodeTimeout and raises the CTA's abort flag, or returns false at
@@ -164,7 +185,9 @@ __device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, Shared
   uint64_t t0 = 0;
   if ((threadIdx.x & 31) == 0) t0 = ptx::globaltimer();
   for (uint32_t i = 1;; ++i) {
-    if (__all_sync(0xffffffffu, ptx::mbar_try_wait(bar, parity))) return true;
+    // sleep in the wait (woken when the phase completes) rather than spin: the waiting roles share the
+    // SM sub-partitions with the TMA and MMA-issuing warps, whose issue slots the spinning would take
+    if (__all_sync(0xffffffffu, ptx::mbar_try_wait_sleep(bar, parity, kSleepNs))) return true;
     if ((i & 63) == 0) {
       int outcome = 0;  // 0 keep waiting, 1 aborted elsewhere, 2 timed out
       if ((threadIdx.x & 31) == 0) {
@@ -216,14 +239,14 @@ __device__ __forceinline__ bool block_info(const Params& p, int h, int k, int D,
 // Block `k` (0-based, in walk order) of segment `si` of this CTA: from the smem table when staged.
 __device__ __forceinline__ bool seg_block(const Params& p, const Shared* sh, int si_local, int k, int h, int b, int D,
                                           BlockInfo& bi) {
-  if (sh->nseg > 0) {
-    bi = sh->blocks[sh->blk0[si_local] + k];
+  if (sh->rec.nseg > 0) {
+    bi = sh->rec.blocks[sh->rec.blk0[si_local] + k];
     return bi.rk >= 1 && bi.rk <= D && bi.rv >= 1 && bi.rv <= D;
   }
   return block_info(p, h, b, D, bi);
 }
 __device__ __forceinline__ Seg get_seg(const Params& p, const Shared* sh, int s_begin, int si) {
-  return sh->nseg > 0 ? sh->segs[si - s_begin] : p.segs[si];
+  return sh->rec.nseg > 0 ? sh->rec.segs[si - s_begin] : p.segs[si];
 }
 
 // Placement of items in the TMA ring.  Producer and consumer call place() with the same sizes in the same
@@ -296,20 +319,9 @@ struct Producer {
     const uint32_t fb = bar(B_FULL + i % kItemSlots);
     if ((threadIdx.x & 31) == 0) {
       ptx::mbar_arrive_expect_tx(fb, bytes);
-      const int k16 = rows >> 4;
-      if (ncb == 2 && (k16 & (k16 - 1)) == 0) {
-        const int hi = k16 == 1 ? 0 : k16 == 2 ? 1 : k16 == 4 ? 2 : 3;
-        ptx::tma_load_3d(dst, map_of(m, true, hi), fb, 0, (int)y0, 0);
-      } else {
-        int r0 = 0;
-        for (int hi = 3; hi >= 0; --hi) {
-          const int h = 16 << hi;
-          if (rows - r0 < h) continue;
-          for (int cb = 0; cb < ncb; ++cb)
-            ptx::tma_load_2d(dst + cb * rows * 128 + r0 * 128, map_of(m, false, hi), fb, 64 * cb, (int)(y0 + r0));
-          r0 += h;
-        }
-      }
+      const CUtensorMap* tm = map_of(m, (rows >> 4) - 1);
+      if (ncb == 2) ptx::tma_load_3d(dst, tm, fb, 0, (int)y0, 0);
+      else ptx::tma_load_2d(dst, tm, fb, 0, (int)y0);
     }
     __syncwarp();
     return true;
@@ -354,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t base = ptx::smem_u32(smem);
-  Shared* sh = reinterpret_cast<Shared*>(smem + kOffBar + 8 * B_COUNT + 64);
+  Shared* sh = reinterpret_cast<Shared*>(smem + kOffBar + kSharedOff);
   auto bar = [&](int i) { return base + kOffBar + 8 * i; };
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -385,38 +397,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tmem_alloc(ptx::smem_u32(&sh->tmem_base), 512);
     ptx::tmem_relinquish();
   }
-  const int s_begin = p.seg_first[blockIdx.x], s_end = p.seg_first[blockIdx.x + 1];
-  // stage this CTA's segments and the rank / row offsets of their blocks in shared memory
-  const int nseg_here = s_end - s_begin;
-  const bool stage_tables = nseg_here <= kMaxSegsSmem;
-  if (stage_tables && (int)threadIdx.x < nseg_here) sh->segs[threadIdx.x] = p.segs[s_begin + threadIdx.x];
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int nblk = 0;
-    for (int i = 0; i < (stage_tables ? nseg_here : 0); ++i) {
-      sh->blk0[i] = nblk;
-      const Seg& sg = sh->segs[i];
-      if (sg.type == 0) nblk += (sg.c1 - 1) / p.cpb - sg.c0 / p.cpb + 1;
-    }
-    sh->blk0[stage_tables ? nseg_here : 0] = nblk;
-    const bool fits = stage_tables && nblk <= kMaxBlocksSmem;
-    sh->nblk = fits ? nblk : 0;
-    sh->nseg = fits ? nseg_here : 0;
+  // this CTA's work record (segments and block tables) into shared memory: one coalesced load
+  {
+    const int4* src = reinterpret_cast<const int4*>(p.recs + blockIdx.x);
+    int4* dst = reinterpret_cast<int4*>(&sh->rec);
+    for (int i = threadIdx.x; i < (int)(sizeof(CtaRec) / 16); i += kThreads) dst[i] = src[i];
   }
   __syncthreads();
-  for (int t = threadIdx.x; t < sh->nblk; t += kThreads) {
-    int i = 0;
-    while (sh->blk0[i + 1] <= t) ++i;
-    const Seg& sg = sh->segs[i];
-    BlockInfo bi;
-    block_info(p, sg.h, sg.c0 / p.cpb + (t - sh->blk0[i]), D, bi);
-    sh->blocks[t] = bi;
-  }
+  const int s_begin = sh->rec.s_begin, s_end = sh->rec.s_end;
   ptx::fence_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
+  // the combine kernel that follows may launch now (it waits for this grid before reading the partials)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp < kSoftWarp0) {
   // the register decrease dominates the producer's and the MMA issuer's code
@@ -1049,6 +1044,9 @@ __global__ void __launch_bounds__(D) combine_tc_kernel(const float* __restrict__
   const int hq = blockIdx.x, i = blockIdx.y, c = threadIdx.x;
   const int G = Hq / H, h = hq / G, g = hq % G;
   const int rt = i / ipt, prow = (i % ipt) * G + g;
+  // launched as a programmatic dependent of the decode kernel: its launch overlaps the decode's last CTAs, and
+  // this waits until the decode grid has completed and its partials are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int p0 = pre_range[2 * (h * nrt + rt)], p1 = pre_range[2 * (h * nrt + rt) + 1];
   const int s0 = suf_range[2 * (i * H + h)], s1 = suf_range[2 * (i * H + h) + 1];
   const int npre = p1 - p0, nall = npre + (s1 - s0);
@@ -1099,6 +1097,26 @@ __global__ void __launch_bounds__(D) combine_tc_kernel(const float* __restrict__
 }
 
 // ------------------------------------------------------------------------------------------------ host
+// The combine kernel for one decode call, launched with programmatic stream serialization so that its launch
+// overlaps the tail of the decode kernel before it (it waits for that grid with griddepcontrol.wait).
+cudaError_t launch_combine(const DecodeShape& s, const float* part_acc, const float2* part_ml, const int* pre,
+                           const int* suf, int ipt, int nrt, void* out, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(s.Hq, s.Bq);
+  cfg.blockDim = dim3(s.d);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+  if (s.d == 64)
+    return cudaLaunchKernelEx(&cfg, combine_tc_kernel<64>, part_acc, part_ml, pre, suf, s.H, s.Hq, ipt, nrt, o);
+  return cudaLaunchKernelEx(&cfg, combine_tc_kernel<128>, part_acc, part_ml, pre, suf, s.H, s.Hq, ipt, nrt, o);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -1138,18 +1156,20 @@ cudaError_t prepare_kernel(int d) {
   return cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
 }
 
-// The 2D and (for 128-column arrays) 3D maps of a [rows][width] bf16 array, boxes of 16/32/64/128 rows.
+// The maps of a [rows][width] bf16 array, one per box height 16, 32, ..., 128 rows: 3D for 128 columns (two
+// 64-column blocks), 2D for 64 columns.
 bool make_row_maps(RowMaps* rm, const void* ptr, uint64_t width, uint64_t rows) {
   std::memset(rm, 0, sizeof(RowMaps));
-  for (int hi = 0; hi < 4; ++hi) {
-    const uint32_t h = 16u << hi;
-    const uint64_t d2[2] = {width, rows}, s2[1] = {width * 2};
-    const uint32_t b2[2] = {64, h};
-    if (!make_map(&rm->m2[hi], ptr, 2, d2, s2, b2)) return false;
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t h = 16u * (k + 1);
     if (width == 128) {
       const uint64_t d3[3] = {64, rows, 2}, s3[2] = {width * 2, 128};
       const uint32_t b3[3] = {64, h, 2};
-      if (!make_map(&rm->m3[hi], ptr, 3, d3, s3, b3)) return false;
+      if (!make_map(&rm->m[k], ptr, 3, d3, s3, b3)) return false;
+    } else {
+      const uint64_t d2[2] = {width, rows}, s2[1] = {width * 2};
+      const uint32_t b2[2] = {64, h};
+      if (!make_map(&rm->m[k], ptr, 2, d2, s2, b2)) return false;
     }
   }
   return true;
@@ -1191,6 +1211,7 @@ struct TcPlan {
   int Bq = 0, Hq = 0, S = 0;
   std::vector<uint8_t> mask;  // the block selection this plan was built for (empty: every block)
   int off_sel = -1;
+  int off_rec = 0;            // per-CTA records (CtaRec) in d_work
   int grid = 0, nsegs = 0, ipt = 0, nrt = 0;
   int* d_work = nullptr;  // seg_first | segs | pre_range | suf_range
   int off_segs = 0, off_pre = 0, off_suf = 0;
@@ -1356,6 +1377,60 @@ int64_t count_atoms(const DecodeShape& s, const uint8_t* mask) {
   }
   return blocks * nrt * cpb + (int64_t)s.Bq * s.H * nsc;
 }
+// The per-CTA work records for a work list `w` (build_worklist_fixed's layout): each CTA's segments with the
+// rank and row offset of every block they walk (the k-th selected block of a head under a selection), the row
+// offsets taken as the running sum of the ranks over pools and blocks in order (the factor layout).  A CTA
+// whose work does not fit its record gets nseg = 0 and reads the global tables instead.
+void build_records(const DecodeShape& s, const int32_t* host_ranks, const int* w, int grid, int off_segs,
+                   int off_sel, CtaRec* recs) {
+  const int nb = s.nb, cpb = s.n / kChunk;
+  std::vector<int64_t> row0((size_t)2 * s.H * nb);
+  int64_t acc = 0;
+  for (size_t i = 0; i < row0.size(); ++i) {
+    row0[i] = acc;
+    acc += host_ranks[i];
+  }
+  const Seg* segs = reinterpret_cast<const Seg*>(w + off_segs);
+  const int* sel = off_sel >= 0 ? w + off_sel : nullptr;
+  for (int k = 0; k < grid; ++k) {
+    CtaRec& r = recs[k];
+    std::memset(&r, 0, sizeof(CtaRec));
+    r.s_begin = w[k];
+    r.s_end = w[k + 1];
+    const int nseg = r.s_end - r.s_begin;
+    int nblk = 0;
+    bool fits = nseg <= kMaxSegsSmem;
+    for (int i = 0; i < nseg && fits; ++i) {
+      const Seg& sg = segs[r.s_begin + i];
+      r.segs[i] = sg;
+      r.blk0[i] = nblk;
+      if (sg.type != 0) continue;
+      for (int vb = sg.c0 / cpb; vb <= (sg.c1 - 1) / cpb; ++vb) {
+        if (nblk >= kMaxBlocksSmem) {
+          fits = false;
+          break;
+        }
+        const int b = sel ? sel[(size_t)sg.h * nb + vb] : vb;
+        BlockInfo& bi = r.blocks[nblk++];
+        bi.rk = host_ranks[(size_t)(2 * sg.h) * nb + b];
+        bi.rv = host_ranks[(size_t)(2 * sg.h + 1) * nb + b];
+        bi.rowk = row0[(size_t)(2 * sg.h) * nb + b];
+        bi.rowv = row0[(size_t)(2 * sg.h + 1) * nb + b];
+      }
+    }
+    if (fits) {
+      r.blk0[nseg] = nblk;
+      r.nseg = nseg;
+      r.nblk = nblk;
+    } else {
+      std::memset(r.blk0, 0, sizeof(r.blk0));
+      r.nseg = 0;
+      r.nblk = 0;
+    }
+  }
+}
+constexpr int kRecWords = (int)(sizeof(CtaRec) / sizeof(int));
+
 // CTAs of the decode kernel: one per SM, fewer when there are fewer atoms.
 int plan_grid(const DecodeShape& s, int sms, const uint8_t* mask = nullptr) {
   return (int)std::max<int64_t>(1, std::min<int64_t>(sms, count_atoms(s, mask)));
@@ -1376,18 +1451,24 @@ static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& 
   const int grid = plan_grid(s, sms, mask);
   const int64_t cap = worklist_cap(s, grid, mask);
   if (cap > (int64_t)1 << 30) return cudaErrorInvalidValue;
-  std::vector<int> host((size_t)cap);
+  std::vector<int> host((size_t)cap + 4 + (size_t)grid * kRecWords);
   int nsegs = 0, off_segs = 0, off_pre = 0, off_suf = 0, ipt = 0, nrt = 0;
   const int nwords = build_worklist_fixed(s, in.host_ranks, grid, host.data(), (int)cap, nsegs, off_segs, off_pre,
                                           off_suf, ipt, nrt, mask, &pl->off_sel);
   if (mask) pl->mask.assign(mask, mask + (size_t)s.H * s.nb);
   if (nwords < 0) return cudaErrorInvalidValue;
+  // per-CTA records after the work list, 16-byte aligned
+  pl->off_rec = (nwords + 3) & ~3;
+  build_records(s, in.host_ranks, host.data(), grid, off_segs, pl->off_sel,
+                reinterpret_cast<CtaRec*>(host.data() + pl->off_rec));
+  const int nwords_all = pl->off_rec + grid * kRecWords;
   pl->off_segs = off_segs;
   pl->off_pre = off_pre;
   pl->off_suf = off_suf;
   cudaError_t e;
-  if ((e = cudaMalloc((void**)&pl->d_work, nwords * sizeof(int))) != cudaSuccess) return e;
-  if ((e = cudaMemcpy(pl->d_work, host.data(), nwords * sizeof(int), cudaMemcpyHostToDevice)) != cudaSuccess)
+  if ((e = cudaMalloc((void**)&pl->d_work, (size_t)nwords_all * sizeof(int))) != cudaSuccess) return e;
+  if ((e = cudaMemcpy(pl->d_work, host.data(), (size_t)nwords_all * sizeof(int), cudaMemcpyHostToDevice)) !=
+      cudaSuccess)
     return e;
   const size_t np = std::max<size_t>(1, (size_t)nsegs);
   if ((e = cudaMalloc((void**)&pl->part_acc, np * 128 * D * sizeof(float))) != cudaSuccess) return e;
@@ -1434,7 +1515,7 @@ cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, v
   maps.pacc = pl->map_pacc;
   if (!make_call_maps(&maps, s, in, pl->ipt)) return cudaErrorInvalidValue;
   Params p;
-  p.seg_first = pl->d_work;
+  p.recs = reinterpret_cast<const CtaRec*>(pl->d_work + pl->off_rec);
   p.segs = reinterpret_cast<const Seg*>(pl->d_work + pl->off_segs);
   p.ranks = in.ranks;
   p.row_offsets = in.row_offsets;
@@ -1460,13 +1541,7 @@ cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, v
   if (ev1 && (e = cudaEventRecord(ev1, st)) != cudaSuccess) return e;
   const int* pre = pl->d_work + pl->off_pre;
   const int* suf = pl->d_work + pl->off_suf;
-  if (D == 64)
-    combine_tc_kernel<64><<<dim3(s.Hq, s.Bq), 64, 0, st>>>(pl->part_acc, pl->part_ml, pre, suf, s.H, s.Hq, pl->ipt,
-                                                          pl->nrt, static_cast<__nv_bfloat16*>(out));
-  else
-    combine_tc_kernel<128><<<dim3(s.Hq, s.Bq), 128, 0, st>>>(pl->part_acc, pl->part_ml, pre, suf, s.H, s.Hq,
-                                                            pl->ipt, pl->nrt, static_cast<__nv_bfloat16*>(out));
-  return cudaGetLastError();
+  return launch_combine(s, pl->part_acc, pl->part_ml, pre, suf, pl->ipt, pl->nrt, out, st);
 }
 
 
@@ -1485,7 +1560,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 std::mutex g_noalloc_mu;
 void* g_noalloc_dev_ptr[kNoAllocMaxDevices];  // device address of g_noalloc_scratch, per device
 bool g_noalloc_ready[kNoAllocMaxDevices][2];  // decode kernel prepared on the device, per head dim (64, 128)
-int g_noalloc_host_words[kNoAllocMaxWords];   // work list staging, guarded by g_noalloc_mu
+alignas(16) int g_noalloc_host_words[kNoAllocMaxWords];  // work list and records staging, guarded by g_noalloc_mu
 
 }  // namespace
 
@@ -1527,8 +1602,17 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
   const int cpb = s.n / kChunk;
   const int grid = plan_grid(s, sms);
   int nsegs = 0, off_segs = 0, off_pre = 0, off_suf = 0, ipt = 0, nrt = 0;
-  const int nwords = build_worklist_fixed(s, in.host_ranks, grid, g_noalloc_host_words, kNoAllocMaxWords, nsegs,
-                                          off_segs, off_pre, off_suf, ipt, nrt, nullptr, nullptr);
+  // the work list, then the per-CTA records (16-byte aligned) in the same staging buffer
+  const int rec_words = grid * kRecWords;
+  int nwords = build_worklist_fixed(s, in.host_ranks, grid, g_noalloc_host_words, kNoAllocMaxWords - rec_words - 4,
+                                    nsegs, off_segs, off_pre, off_suf, ipt, nrt, nullptr, nullptr);
+  int off_rec = 0;
+  if (nwords >= 0) {
+    off_rec = (nwords + 3) & ~3;
+    build_records(s, in.host_ranks, g_noalloc_host_words, grid, off_segs, -1,
+                  reinterpret_cast<CtaRec*>(g_noalloc_host_words + off_rec));
+    nwords = off_rec + rec_words;
+  }
   const size_t words_bytes = ((size_t)std::max(nwords, 0) * sizeof(int) + 255) & ~(size_t)255;
   const size_t ml_bytes = ((size_t)nsegs * 128 * sizeof(float2) + 255) & ~(size_t)255;
   const size_t acc_bytes = (size_t)nsegs * 128 * s.d * sizeof(float);
@@ -1551,7 +1635,7 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
   if (!make_pacc_map(&maps.pacc, part_acc, nsegs, D)) return cudaErrorInvalidValue;
   if (!make_call_maps(&maps, s, in, ipt)) return cudaErrorInvalidValue;
   Params p;
-  p.seg_first = d_work;
+  p.recs = reinterpret_cast<const CtaRec*>(d_work + off_rec);
   p.segs = reinterpret_cast<const Seg*>(d_work + off_segs);
   p.ranks = in.ranks;
   p.row_offsets = in.row_offsets;
@@ -1571,13 +1655,7 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
   else
     decode_tc_kernel<128><<<grid, kThreads, kSmemBytes, st>>>(maps, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (D == 64)
-    combine_tc_kernel<64><<<dim3(s.Hq, s.Bq), 64, 0, st>>>(part_acc, part_ml, d_work + off_pre, d_work + off_suf,
-                                                          s.H, s.Hq, ipt, nrt, static_cast<__nv_bfloat16*>(out));
-  else
-    combine_tc_kernel<128><<<dim3(s.Hq, s.Bq), 128, 0, st>>>(part_acc, part_ml, d_work + off_pre, d_work + off_suf,
-                                                            s.H, s.Hq, ipt, nrt, static_cast<__nv_bfloat16*>(out));
-  return cudaGetLastError();
+  return launch_combine(s, part_acc, part_ml, d_work + off_pre, d_work + off_suf, ipt, nrt, out, st);
 }
 
 }  // namespace milo

@@ -160,3 +160,11 @@ def test_decode_32b_stack_sharp_softmax():
     wl, dt, lay, f, q, Ks, Vs = _setup("qwen2.5-32b-stack", beta=0.5, q_scale=60.0)
     out, want = _run(wl, dt, lay, f, q, Ks, Vs, sample=_tile_sample(wl, wl.batch))
     assert_close(out, want, TOL[dt], "32b stack layer q x 60")
+
+
+def test_decode_large_batch_7b():
+    """A batch of 300 queries with 256-token suffixes: 17 row tiles per KV head and some 1200 suffix segments,
+    more segments than a CTA's staged work record holds, so that CTAs also read the global segment tables."""
+    wl, dt, lay, f, q, Ks, Vs = _setup("qwen2.5-7b-layer", batch=300)
+    out, want = _run(wl, dt, lay, f, q, Ks, Vs, sample=[0, 17, 18, 151, 287, 288, 299])
+    assert_close(out, want, TOL[dt], "batch 300")
