@@ -103,10 +103,26 @@ struct Seg {
   int pad;
 };
 
+// One TMA load of the producer's walk, built on the host in the order the issuing warp consumes the data.
+// Ring items (kinds 0 and 1) land at byte `a` of the ring; a query tile (kind 2) lands in the query buffer
+// at coordinates (y, z = a).  Before a ring item is issued the producer retires the `retire` oldest ring
+// items in flight (waits until the MMAs that read them have completed), which frees its bytes and slot.
+struct Item {
+  uint32_t a;      // ring byte offset (kinds 0, 1) or z coordinate (kind 2)
+  int32_t y;       // row coordinate
+  uint32_t bytes;  // bytes the load delivers
+  uint32_t meta;   // map index (bits 0-7) | kind (bits 8-9: 0 2D box, 1 3D box, 2 query tile) | retire (16-23)
+};
+static_assert(sizeof(Item) == 16, "items are loaded as 16-byte words");
+constexpr uint32_t kItem2D = 0, kItem3D = 1, kItemQ = 2;
+
 struct CtaRec;
+struct PlanMaps;
 struct Params {
   const Seg* segs;
   const CtaRec* recs;    // [grid]
+  const Item* items;     // every CTA's items, CTA k's at [recs[k].item0, + recs[k].nitems)
+  const PlanMaps* gmaps;
   const int32_t* ranks;
   const int64_t* row_offsets;
   float* part_acc;  // [pid][128][D]
@@ -129,25 +145,20 @@ struct BlockInfo {
 struct RowMaps {
   CUtensorMap m[8];
 };
+// The maps of one call's arrays, passed as the kernel parameter (kept small: a launch copies its parameters).
 struct Maps {
-  RowMaps tok, dim, ksuf, vsuf;  // the suffix maps use the 128-row boxes only
-  CUtensorMap qpre, qsuf;
+  CUtensorMap ksuf, vsuf;  // suffix keys and values, boxes of 128 rows
+  CUtensorMap qpre, qsuf;  // query rows of a prefix row tile / of one query
+};
+// The maps of a plan's factors and partials, in device memory (128-byte aligned), written once per plan.
+struct PlanMaps {
+  RowMaps tok, dim;
   CUtensorMap pacc;  // partial accumulators [segments · 128][d] fp32, boxes of 128 rows × 32 columns
 };
-
-__device__ __forceinline__ const CUtensorMap* map_of(const RowMaps& m, int k) {
-  // constant indices: the result stays an address in the kernel-parameter space
-  switch (k) {
-    case 0: return &m.m[0];
-    case 1: return &m.m[1];
-    case 2: return &m.m[2];
-    case 3: return &m.m[3];
-    case 4: return &m.m[4];
-    case 5: return &m.m[5];
-    case 6: return &m.m[6];
-    default: return &m.m[7];
-  }
-}
+// An item's map index: [0, 16) counts CUtensorMaps from the start of PlanMaps, [16, 20) from the start of Maps.
+constexpr int kMapTok = 0, kMapDim = 8, kMapKsuf = 16, kMapVsuf = 17, kMapQpre = 18, kMapQsuf = 19;
+static_assert(sizeof(RowMaps) == 8 * sizeof(CUtensorMap), "row maps hold 8 boxes");
+static_assert(sizeof(Maps) == 4 * sizeof(CUtensorMap), "call maps in the order of the item map index");
 
 // One CTA's work, built on the host: its segments and the rank / row offset of every block they touch, in
 // the order the roles walk them.  The CTA copies it to shared memory with one coalesced load at start, so
@@ -157,7 +168,8 @@ struct CtaRec {
   int nblk;        // blocks staged
   int s_begin, s_end;          // the CTA's range in the global segment list
   int blk0[kMaxSegsSmem + 1];  // first block entry of each segment
-  int pad[3];
+  int item0, nitems;           // the CTA's producer items in Params::items
+  int pad;
   Seg segs[kMaxSegsSmem];
   BlockInfo blocks[kMaxBlocksSmem];
 };
@@ -169,7 +181,6 @@ struct Shared {
   int abort_flag;
   int pad[2];
   CtaRec rec;
-  uint32_t pos_log[kItemSlots], len_log[kItemSlots];  // producer's record of the items in flight
   float mx_x[2][2][128];  // row maxima exchanged by the two softmax warpgroups (double-buffered)
   float l_x[128];         // warpgroup 1's row sums at a segment's end
 };
@@ -273,70 +284,6 @@ struct BlockWalk {
   __device__ void next() { c += chunks(); }
 };
 
-// -------------------------------------------------------------------------------------------- producer
-template <int D>
-struct Producer {
-  static constexpr int NCB = D / 64;
-  uint32_t base;
-  RingPlace ring;
-  uint32_t oldest = 0;  // first item not yet known to be released
-  uint32_t q_uses = 0;
-  Shared* sh;
-  uint32_t* status;
-  uint32_t* pos_log;  // [kItemSlots] offsets of the items in flight (smem, producer only)
-  uint32_t* len_log;  // [kItemSlots] their sizes
-
-  __device__ uint32_t bar(int i) const { return base + kOffBar + 8 * i; }
-
-  // Waits until the oldest item in flight has been consumed and forgets it.
-  __device__ bool retire_oldest() {
-    const uint32_t j = oldest;
-    if (!wait_bar(bar(B_EMPTY + j % kItemSlots), (j / kItemSlots) & 1, sh, status)) return false;
-    ++oldest;
-    return true;
-  }
-
-  // `rows` (multiple of 16, <= 128) rows × `ncb` 64-column blocks at row y0 → one item, laid out
-  // [cb][rows][128 B].  A power-of-two height over two column blocks is one 3D load; other heights are
-  // 2D loads of 128/64/32/16 rows per column block.
-  __device__ __noinline__ bool item(const RowMaps& m, int64_t y0, int rows, int ncb) {
-    const uint32_t bytes = (uint32_t)rows * 128u * ncb;
-    const uint32_t i = ring.n;
-    const uint32_t head = ring.head;  // end of the newest item in flight
-    const uint32_t pos = ring.place(bytes);
-    // Free the space: the items in flight occupy the cyclic byte range [start of the oldest, head) (with any
-    // gap skipped at a wrap counted as occupied); retire the oldest until [pos, pos + bytes) lies outside it
-    // and fewer than kItemSlots items are in flight.
-    while (oldest < i) {
-      const uint32_t tail = pos_log[oldest % kItemSlots];
-      const bool room = tail < head ? (pos + bytes <= tail || pos >= head) : (pos + bytes <= tail && pos >= head);
-      if (room && i - oldest < (uint32_t)kItemSlots) break;
-      if (!retire_oldest()) return false;
-    }
-    pos_log[i % kItemSlots] = pos;
-    len_log[i % kItemSlots] = bytes;
-    const uint32_t dst = base + kOffRing + pos;
-    const uint32_t fb = bar(B_FULL + i % kItemSlots);
-    if ((threadIdx.x & 31) == 0) {
-      ptx::mbar_arrive_expect_tx(fb, bytes);
-      const CUtensorMap* tm = map_of(m, (rows >> 4) - 1);
-      if (ncb == 2) ptx::tma_load_3d(dst, tm, fb, 0, (int)y0, 0);
-      else ptx::tma_load_2d(dst, tm, fb, 0, (int)y0);
-    }
-    __syncwarp();
-    return true;
-  }
-  __device__ bool q_tile(const CUtensorMap* m, int y, int z, int box_rows) {
-    if (!wait_bar(bar(B_QEMPTY), (q_uses & 1) ^ 1, sh, status)) return false;
-    if ((threadIdx.x & 31) == 0) {
-      ptx::mbar_arrive_expect_tx(bar(B_QFULL), box_rows * 128 * NCB);
-      for (int cb = 0; cb < NCB; ++cb) ptx::tma_load_3d(base + kOffQ + cb * kTileCb, m, bar(B_QFULL), 64 * cb, y, z);
-    }
-    ++q_uses;
-    return true;
-  }
-};
-
 // K-major SW128 descriptor of k-step k (16 bf16) of a tile whose 64-column blocks are `cbs` bytes apart.
 __device__ __forceinline__ uint64_t kdesc(uint32_t tile, int k, uint32_t cbs) {
   return ptx::sw128_desc(tile + (uint32_t)(k >> 2) * cbs + (uint32_t)(k & 3) * 32, 16, 1024);
@@ -418,74 +365,58 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (kRegSplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
   if (warp == 0) {
     // ==================================================================== TMA producer
-    // Loads items in exactly the order the issuing warp consumes them (see the softmax section).
-    Producer<D> pr;
-    pr.base = base;
-    pr.sh = sh;
-    pr.status = p.status;
-    pr.pos_log = sh->pos_log;
-    pr.len_log = sh->len_log;
+    // Walks the CTA's item list: the host has fixed every load's map, coordinates, ring offset and how many
+    // older items must be released before it, so that each item costs a few instructions here.  Lane l holds
+    // item i0 + l of the current batch of 32; the batch after it is loaded while this one is issued.
+    const Item* items = p.items + sh->rec.item0;
+    const int nitems = sh->rec.nitems;
+    const CUtensorMap* gmap0 = reinterpret_cast<const CUtensorMap*>(p.gmaps);
+    const CUtensorMap* pmap0 = reinterpret_cast<const CUtensorMap*>(&maps);
+    auto load_item = [&](int i) -> uint4 {
+      return i < nitems ? __ldg(reinterpret_cast<const uint4*>(items + i)) : make_uint4(0, 0, 0, 0);
+    };
+    uint32_t oldest = 0, ring_n = 0, q_uses = 0;
     bool ok = true;
-    auto bad_block = [&]() {
-      atomicOr(p.status, kStatusDecodeBounds);
-      sh->abort_flag = 1;
-      return false;
-    };
-    // token-factor slab of chunk cc (index inside the block) of a block: rows [row0·cpb + cc·r, +r)
-    auto tok_item = [&](int64_t row0, int r, int cc) {
-      return pr.item(maps.tok, row0 * p.cpb + (int64_t)cc * r, pad16(r), 2);
-    };
-    auto dim_item = [&](int64_t row0, int r) { return pr.item(maps.dim, row0, pad16(r), NCB); };
-    for (int si = s_begin; si < s_end && ok; ++si) {
-      const Seg sg = get_seg(p, sh, s_begin, si);
-      if (sg.type == 0) {
-        ok = pr.q_tile(&maps.qpre, sg.h * p.G, sg.tile * p.ipt, p.G * p.ipt);
-        BlockWalk w{sg.c0, sg.c1, p.cpb};
-        BlockInfo bi, bn, prev;
-        bool have_prev = false;
-        int kb = 0;
-        if (ok && !seg_block(p, sh, si - s_begin, kb, sg.h, w.block(), D, bi)) ok = bad_block();
-        if (ok) ok = dim_item(bi.rowk, bi.rk);  // B_K of the first block
-        while (ok) {
-          const int n = w.chunks(), cc0 = w.first_cc();
-          const bool next = w.has_next();
-          if (next && !seg_block(p, sh, si - s_begin, kb + 1, sg.h, w.block() + 1, D, bn)) ok = bad_block();
-          if (ok) ok = tok_item(bi.rowk, bi.rk, cc0);                       // U(0)
-          if (ok && n >= 2) ok = tok_item(bi.rowk, bi.rk, cc0 + 1);         // U(1)
-          else if (ok && next) ok = dim_item(bn.rowk, bn.rk);               // B_K(next)
-          if (ok && have_prev) ok = dim_item(prev.rowv, prev.rv);           // Q_V(previous block)
-          for (int j = 0; j < n && ok; ++j) {
-            ok = tok_item(bi.rowv, bi.rv, cc0 + j);                         // P(j)
-            if (ok && j + 2 < n) ok = tok_item(bi.rowk, bi.rk, cc0 + j + 2);  // U(j+2)
-            else if (ok && j + 2 == n && next) ok = dim_item(bn.rowk, bn.rk);  // B_K(next)
+    uint4 cur = load_item(lane);
+    for (int i0 = 0; i0 < nitems && ok; i0 += 32) {
+      const uint4 nxt = load_item(i0 + 32 + lane);
+      const int nb = min(32, nitems - i0);
+      for (int k = 0; k < nb && ok; ++k) {
+        const uint32_t a = __shfl_sync(0xffffffffu, cur.x, k);
+        const int y = (int)__shfl_sync(0xffffffffu, cur.y, k);
+        const uint32_t bytes = __shfl_sync(0xffffffffu, cur.z, k);
+        const uint32_t meta = __shfl_sync(0xffffffffu, cur.w, k);
+        const uint32_t mi = meta & 255u;
+        const CUtensorMap* tm = mi < (uint32_t)kMapKsuf ? gmap0 + mi : pmap0 + (mi - kMapKsuf);
+        const uint32_t kind = (meta >> 8) & 3u;
+        if (kind == kItemQ) {
+          ok = wait_bar(bar(B_QEMPTY), (q_uses & 1) ^ 1, sh, p.status);
+          if (ok && lane == 0) {
+            ptx::mbar_arrive_expect_tx(bar(B_QFULL), bytes);
+            for (int cb = 0; cb < NCB; ++cb)
+              ptx::tma_load_3d(base + kOffQ + cb * kTileCb, tm, bar(B_QFULL), 64 * cb, y, (int)a);
           }
-          if (!ok || !next) break;
-          prev = bi;
-          have_prev = true;
-          w.next();
-          bi = bn;
-          ++kb;
+          ++q_uses;
+          continue;
         }
-        if (ok) ok = dim_item(bi.rowv, bi.rv);  // Q_V of the last block
-      } else {
-        ok = pr.q_tile(&maps.qsuf, sg.h * p.G, sg.tile, p.G);
-        const int64_t row0 = ((int64_t)sg.tile * p.H + sg.h) * p.S;
-        const int n = sg.c1 - sg.c0;
-        auto kv = [&](const RowMaps& m, int j) {
-          return pr.item(m, row0 + (int64_t)(sg.c0 + j) * kChunk, kChunk, NCB);
-        };
-        if (ok) ok = kv(maps.ksuf, 0);
-        if (ok && n >= 2) ok = kv(maps.ksuf, 1);
-        for (int j = 0; j < n && ok; ++j) {
-          ok = kv(maps.vsuf, j);
-          if (ok && j + 2 < n) ok = kv(maps.ksuf, j + 2);
+        for (uint32_t r = (meta >> 16) & 255u; r > 0 && ok; --r, ++oldest)
+          ok = wait_bar(bar(B_EMPTY + oldest % kItemSlots), (oldest / kItemSlots) & 1, sh, p.status);
+        if (!ok) break;
+        const uint32_t fb = bar(B_FULL + ring_n % kItemSlots);
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(fb, bytes);
+          if (kind == kItem3D) ptx::tma_load_3d(base + kOffRing + a, tm, fb, 0, y, 0);
+          else ptx::tma_load_2d(base + kOffRing + a, tm, fb, 0, y);
         }
+        __syncwarp();
+        ++ring_n;
       }
+      cur = nxt;
     }
     // drain: every copy this warp issued must have landed before the CTA exits
-    for (uint32_t j = pr.oldest; j < pr.ring.n; ++j)
+    for (uint32_t j = oldest; j < ring_n; ++j)
       wait_bar(bar(B_FULL + j % kItemSlots), (j / kItemSlots) & 1, sh, p.status, true);
-    if (pr.q_uses) wait_bar(bar(B_QFULL), (pr.q_uses - 1) & 1, sh, p.status, true);
+    if (q_uses) wait_bar(bar(B_QFULL), (q_uses - 1) & 1, sh, p.status, true);
   } else if (warp == 1) {
     // ==================================================================== MMA issuer (warp 1)
     // Issues the tensor-core MMAs when the softmax warps signal (named barriers) that what they produce is
@@ -942,7 +873,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::fence_async_smem();
       soft_sync();
       if (storer) {
-        for (int cb = 0; cb < D / 32; ++cb) ptx::tma_store_2d(&maps.pacc, base + kOffQtHi + 16384u * cb, 32 * cb, sg.pid * 128);
+        for (int cb = 0; cb < D / 32; ++cb) ptx::tma_store_2d(&p.gmaps->pacc, base + kOffQtHi + 16384u * cb, 32 * cb, sg.pid * 128);
         ptx::bulk_commit();
         store_pending = true;
       }
@@ -1156,22 +1087,23 @@ cudaError_t prepare_kernel(int d) {
   return cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
 }
 
-// The maps of a [rows][width] bf16 array, one per box height 16, 32, ..., 128 rows: 3D for 128 columns (two
-// 64-column blocks), 2D for 64 columns.
+// The map of a [rows][width] bf16 array with boxes of h rows: 3D for 128 columns (x: 64 columns, y: rows,
+// z: the two 64-column blocks), 2D for 64 columns.
+bool make_rows_map(CUtensorMap* m, const void* ptr, uint64_t width, uint64_t rows, uint32_t h) {
+  if (width == 128) {
+    const uint64_t d3[3] = {64, rows, 2}, s3[2] = {width * 2, 128};
+    const uint32_t b3[3] = {64, h, 2};
+    return make_map(m, ptr, 3, d3, s3, b3);
+  }
+  const uint64_t d2[2] = {width, rows}, s2[1] = {width * 2};
+  const uint32_t b2[2] = {64, h};
+  return make_map(m, ptr, 2, d2, s2, b2);
+}
+// The maps of a [rows][width] bf16 array, one per box height 16, 32, ..., 128 rows.
 bool make_row_maps(RowMaps* rm, const void* ptr, uint64_t width, uint64_t rows) {
   std::memset(rm, 0, sizeof(RowMaps));
-  for (int k = 0; k < 8; ++k) {
-    const uint32_t h = 16u * (k + 1);
-    if (width == 128) {
-      const uint64_t d3[3] = {64, rows, 2}, s3[2] = {width * 2, 128};
-      const uint32_t b3[3] = {64, h, 2};
-      if (!make_map(&rm->m[k], ptr, 3, d3, s3, b3)) return false;
-    } else {
-      const uint64_t d2[2] = {width, rows}, s2[1] = {width * 2};
-      const uint32_t b2[2] = {64, h};
-      if (!make_map(&rm->m[k], ptr, 2, d2, s2, b2)) return false;
-    }
-  }
+  for (int k = 0; k < 8; ++k)
+    if (!make_rows_map(&rm->m[k], ptr, width, rows, 16u * (k + 1))) return false;
   return true;
 }
 
@@ -1197,10 +1129,11 @@ bool make_call_maps(Maps* M, const DecodeShape& s, const TcInputs& in, int ipt) 
   if (!make_map(&M->qsuf, in.q, 3, dims, strd, box_suf)) return false;
   if (s.S > 0) {
     const uint64_t rows = (uint64_t)s.Bq * s.H * s.S;
-    if (!make_row_maps(&M->ksuf, in.K_suf, D, rows) || !make_row_maps(&M->vsuf, in.V_suf, D, rows)) return false;
+    if (!make_rows_map(&M->ksuf, in.K_suf, D, rows, kChunk) || !make_rows_map(&M->vsuf, in.V_suf, D, rows, kChunk))
+      return false;
   } else {
-    M->ksuf = M->tok;  // never read
-    M->vsuf = M->tok;
+    M->ksuf = M->qpre;  // never read
+    M->vsuf = M->qpre;
   }
   return true;
 }
@@ -1212,6 +1145,7 @@ struct TcPlan {
   std::vector<uint8_t> mask;  // the block selection this plan was built for (empty: every block)
   int off_sel = -1;
   int off_rec = 0;            // per-CTA records (CtaRec) in d_work
+  int off_items = 0;          // producer items (Item) in d_work
   int grid = 0, nsegs = 0, ipt = 0, nrt = 0;
   int* d_work = nullptr;  // seg_first | segs | pre_range | suf_range
   int off_segs = 0, off_pre = 0, off_suf = 0;
@@ -1219,8 +1153,7 @@ struct TcPlan {
   float2* part_ml = nullptr;
   const void* tok = nullptr;
   const void* dim = nullptr;
-  RowMaps map_tok, map_dim;
-  CUtensorMap map_pacc;
+  PlanMaps* d_maps = nullptr;  // the factor and partial maps in device memory
 };
 
 bool tc_shape_ok(const DecodeShape& s) {
@@ -1237,6 +1170,7 @@ void tc_plan_destroy(TcPlan* plan) {
   cudaFree(plan->d_work);
   cudaFree(plan->part_acc);
   cudaFree(plan->part_ml);
+  cudaFree(plan->d_maps);
   delete plan;
 }
 
@@ -1431,6 +1365,126 @@ void build_records(const DecodeShape& s, const int32_t* host_ranks, const int* w
 }
 constexpr int kRecWords = (int)(sizeof(CtaRec) / sizeof(int));
 
+// The producer's item list of every CTA, in the order the MMA warp consumes the data: per prefix segment the
+// query tile, B_K of the first block, then per block U(0), U(1) (or B_K of the next block when the block has
+// one chunk here), Q_V of the previous block, and per chunk j P(j) followed by U(j + 2) (or B_K of the next
+// block in place of the first missing U), and finally Q_V of the last block; per suffix segment the query
+// tile, K(0), K(1), then per chunk V(j) followed by K(j + 2).  Ring offsets follow the MMA warp's placement
+// (an item that does not fit before the end of the ring starts at offset 0), and each ring item retires the
+// oldest items in flight until its bytes are free and fewer than kItemSlots items are outstanding.  Writes
+// at most `cap` items to `out` and sets every record's item range; returns the item count, or -1 when `cap` is
+// too small, a coordinate does not fit the TMA's 32 bits or a rank lies outside [1, d].
+int64_t build_items(const DecodeShape& s, const int32_t* host_ranks, const int* w, int grid, int off_segs,
+                    int off_sel, CtaRec* recs, Item* out, int64_t cap) {
+  const int nb = s.nb, cpb = s.n / kChunk, G = s.Hq / s.H, ncb = s.d / 64;
+  const int ipt = std::min(s.Bq, 128 / G);
+  std::vector<int64_t> row0((size_t)2 * s.H * nb);
+  int64_t acc = 0;
+  for (size_t i = 0; i < row0.size(); ++i) {
+    row0[i] = acc;
+    acc += host_ranks[i];
+  }
+  const Seg* segs = reinterpret_cast<const Seg*>(w + off_segs);
+  const int* sel = off_sel >= 0 ? w + off_sel : nullptr;
+  auto pad = [](int r) { return (r + 15) & ~15; };
+  bool fits = true;
+  int64_t cnt = 0;
+  auto push = [&](const Item& it) {
+    if (cnt < cap) out[cnt] = it;
+    else fits = false;
+    ++cnt;
+  };
+  for (int k = 0; k < grid && fits; ++k) {
+    recs[k].item0 = (int)cnt;
+    uint32_t head = 0, n = 0, oldest = 0;  // the ring as the MMA warp places it
+    uint32_t pos_of[kItemSlots];          // offsets of the items in flight (at most kItemSlots)
+    auto ring = [&](int map, int64_t y, int rows, int nc) {  // `map`: the item's final map index
+      if (y > INT32_MAX || rows < 16 || rows > 128) fits = false;
+      const uint32_t bytes = (uint32_t)rows * 128u * nc;
+      const uint32_t pos = head + bytes <= (uint32_t)kRingBytes ? head : 0u;
+      uint32_t retire = 0;
+      while (oldest < n) {
+        const uint32_t tail = pos_of[oldest % kItemSlots];
+        const bool room = tail < head ? (pos + bytes <= tail || pos >= head) : (pos + bytes <= tail && pos >= head);
+        if (room && n - oldest < (uint32_t)kItemSlots) break;
+        ++oldest;
+        ++retire;
+      }
+      head = pos + bytes;
+      pos_of[n % kItemSlots] = pos;
+      ++n;
+      const uint32_t kind = nc == 2 ? kItem3D : kItem2D;
+      push(Item{pos, (int32_t)y, bytes, (uint32_t)map | kind << 8 | retire << 16});
+    };
+    auto qtile = [&](int map, int y, int z, int box_rows) {
+      push(Item{(uint32_t)z, y, (uint32_t)box_rows * 128u * ncb, (uint32_t)map | kItemQ << 8});
+    };
+    struct BI {
+      int rk, rv;
+      int64_t rowk, rowv;
+    };
+    for (int si = w[k]; si < w[k + 1]; ++si) {
+      const Seg& sg = segs[si];
+      if (sg.type != 0) {
+        qtile(kMapQsuf, sg.h * G, sg.tile, G);
+        const int64_t r0 = ((int64_t)sg.tile * s.H + sg.h) * s.S;
+        const int nc = sg.c1 - sg.c0;
+        auto kv = [&](int map, int j) { ring(map, r0 + (int64_t)(sg.c0 + j) * kChunk, kChunk, ncb); };
+        kv(kMapKsuf, 0);
+        if (nc >= 2) kv(kMapKsuf, 1);
+        for (int j = 0; j < nc; ++j) {
+          kv(kMapVsuf, j);
+          if (j + 2 < nc) kv(kMapKsuf, j + 2);
+        }
+        continue;
+      }
+      qtile(kMapQpre, sg.h * G, sg.tile * ipt, G * ipt);
+      auto info = [&](int vb) {
+        const int b = sel ? sel[(size_t)sg.h * nb + vb] : vb;
+        const size_t ik = (size_t)(2 * sg.h) * nb + b, iv = (size_t)(2 * sg.h + 1) * nb + b;
+        const BI r{host_ranks[ik], host_ranks[iv], row0[ik], row0[iv]};
+        if (r.rk < 1 || r.rk > s.d || r.rv < 1 || r.rv > s.d) fits = false;
+        return r;
+      };
+      auto dim_item = [&](int64_t r0, int r) { ring(kMapDim + pad(r) / 16 - 1, r0, pad(r), ncb); };
+      auto tok_item = [&](int64_t r0, int r, int cc) {
+        ring(kMapTok + pad(r) / 16 - 1, r0 * cpb + (int64_t)cc * r, pad(r), 2);
+      };
+      int c = sg.c0;
+      BI bi = info(c / cpb), prev{};
+      bool have_prev = false;
+      dim_item(bi.rowk, bi.rk);
+      while (true) {
+        const int blk = c / cpb, cc0 = c - blk * cpb;
+        const int nch = std::min(sg.c1, (blk + 1) * cpb) - c;
+        const bool next = c + nch < sg.c1;
+        const BI bn = next ? info(blk + 1) : BI{};
+        tok_item(bi.rowk, bi.rk, cc0);
+        if (nch >= 2) tok_item(bi.rowk, bi.rk, cc0 + 1);
+        else if (next) dim_item(bn.rowk, bn.rk);
+        if (have_prev) dim_item(prev.rowv, prev.rv);
+        for (int j = 0; j < nch; ++j) {
+          tok_item(bi.rowv, bi.rv, cc0 + j);
+          if (j + 2 < nch) tok_item(bi.rowk, bi.rk, cc0 + j + 2);
+          else if (j + 2 == nch && next) dim_item(bn.rowk, bn.rk);
+        }
+        if (!next) break;
+        prev = bi;
+        have_prev = true;
+        c += nch;
+        bi = bn;
+      }
+      dim_item(bi.rowv, bi.rv);
+    }
+    recs[k].nitems = (int)(cnt - recs[k].item0);
+  }
+  return fits && cnt <= INT32_MAX ? cnt : -1;
+}
+constexpr int kItemWords = (int)(sizeof(Item) / sizeof(int));
+// Items of a work list at most: per atom (a 128-token chunk) its two ring items, and per segment (at most one
+// per atom) a query tile and per block visit (at most one per atom) two dim-factor items.
+int64_t items_cap(const DecodeShape& s, const uint8_t* mask = nullptr) { return 5 * count_atoms(s, mask); }
+
 // CTAs of the decode kernel: one per SM, fewer when there are fewer atoms.
 int plan_grid(const DecodeShape& s, int sms, const uint8_t* mask = nullptr) {
   return (int)std::max<int64_t>(1, std::min<int64_t>(sms, count_atoms(s, mask)));
@@ -1457,11 +1511,19 @@ static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& 
                                           off_suf, ipt, nrt, mask, &pl->off_sel);
   if (mask) pl->mask.assign(mask, mask + (size_t)s.H * s.nb);
   if (nwords < 0) return cudaErrorInvalidValue;
-  // per-CTA records after the work list, 16-byte aligned
+  // per-CTA records after the work list, then the producer items, each 16-byte aligned
   pl->off_rec = (nwords + 3) & ~3;
-  build_records(s, in.host_ranks, host.data(), grid, off_segs, pl->off_sel,
-                reinterpret_cast<CtaRec*>(host.data() + pl->off_rec));
-  const int nwords_all = pl->off_rec + grid * kRecWords;
+  CtaRec* recs = reinterpret_cast<CtaRec*>(host.data() + pl->off_rec);
+  build_records(s, in.host_ranks, host.data(), grid, off_segs, pl->off_sel, recs);
+  const int off_items = pl->off_rec + grid * kRecWords;
+  const int64_t icap = items_cap(s, mask);
+  host.resize((size_t)off_items + (size_t)icap * kItemWords);
+  recs = reinterpret_cast<CtaRec*>(host.data() + pl->off_rec);
+  const int64_t nitems = build_items(s, in.host_ranks, host.data(), grid, off_segs, pl->off_sel, recs,
+                                     reinterpret_cast<Item*>(host.data() + off_items), icap);
+  if (nitems < 0 || off_items + nitems * kItemWords > INT32_MAX) return cudaErrorInvalidValue;
+  pl->off_items = off_items;
+  const int nwords_all = (int)(off_items + nitems * kItemWords);
   pl->off_segs = off_segs;
   pl->off_pre = off_pre;
   pl->off_suf = off_suf;
@@ -1483,9 +1545,12 @@ static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& 
   // factor maps: the token factor as a [rows · n/128][128] array of 128-token slab rows, the dim factor
   // as [rows][d]
   const uint64_t rows = (uint64_t)in.total_rows;
-  if (!make_row_maps(&pl->map_tok, in.tok, kChunk, rows * cpb)) return cudaErrorInvalidValue;
-  if (!make_row_maps(&pl->map_dim, in.dim, D, rows)) return cudaErrorInvalidValue;
-  if (!make_pacc_map(&pl->map_pacc, pl->part_acc, pl->nsegs, D)) return cudaErrorInvalidValue;
+  PlanMaps pm;
+  if (!make_row_maps(&pm.tok, in.tok, kChunk, rows * cpb)) return cudaErrorInvalidValue;
+  if (!make_row_maps(&pm.dim, in.dim, D, rows)) return cudaErrorInvalidValue;
+  if (!make_pacc_map(&pm.pacc, pl->part_acc, pl->nsegs, D)) return cudaErrorInvalidValue;
+  if ((e = cudaMalloc((void**)&pl->d_maps, sizeof(PlanMaps))) != cudaSuccess) return e;
+  if ((e = cudaMemcpy(pl->d_maps, &pm, sizeof(PlanMaps), cudaMemcpyHostToDevice)) != cudaSuccess) return e;
   pl->tok = in.tok;
   pl->dim = in.dim;
   return prepare_kernel(D);
@@ -1510,12 +1575,11 @@ cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, v
   }
   const int D = s.d, G = s.Hq / s.H;
   Maps maps;
-  maps.tok = pl->map_tok;
-  maps.dim = pl->map_dim;
-  maps.pacc = pl->map_pacc;
   if (!make_call_maps(&maps, s, in, pl->ipt)) return cudaErrorInvalidValue;
   Params p;
   p.recs = reinterpret_cast<const CtaRec*>(pl->d_work + pl->off_rec);
+  p.items = reinterpret_cast<const Item*>(pl->d_work + pl->off_items);
+  p.gmaps = pl->d_maps;
   p.segs = reinterpret_cast<const Seg*>(pl->d_work + pl->off_segs);
   p.ranks = in.ranks;
   p.row_offsets = in.row_offsets;
@@ -1606,13 +1670,22 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
   const int rec_words = grid * kRecWords;
   int nwords = build_worklist_fixed(s, in.host_ranks, grid, g_noalloc_host_words, kNoAllocMaxWords - rec_words - 4,
                                     nsegs, off_segs, off_pre, off_suf, ipt, nrt, nullptr, nullptr);
-  int off_rec = 0;
+  int off_rec = 0, off_items = 0;
   if (nwords >= 0) {
     off_rec = (nwords + 3) & ~3;
-    build_records(s, in.host_ranks, g_noalloc_host_words, grid, off_segs, -1,
-                  reinterpret_cast<CtaRec*>(g_noalloc_host_words + off_rec));
-    nwords = off_rec + rec_words;
+    CtaRec* recs = reinterpret_cast<CtaRec*>(g_noalloc_host_words + off_rec);
+    build_records(s, in.host_ranks, g_noalloc_host_words, grid, off_segs, -1, recs);
+    off_items = off_rec + rec_words;
+    const int64_t room = ((int64_t)kNoAllocMaxWords - off_items) / kItemWords;
+    const int64_t nitems = room > 0 ? build_items(s, in.host_ranks, g_noalloc_host_words, grid, off_segs, -1, recs,
+                                                  reinterpret_cast<Item*>(g_noalloc_host_words + off_items), room)
+                                    : -1;
+    nwords = nitems < 0 ? -1 : (int)(off_items + nitems * kItemWords);
   }
+  // the plan's maps after the items, 128-byte aligned
+  constexpr int kMapWords = (int)(sizeof(PlanMaps) / sizeof(int));
+  const int off_maps = (std::max(nwords, 0) + 31) & ~31;
+  if (nwords >= 0) nwords = off_maps + kMapWords <= kNoAllocMaxWords ? off_maps + kMapWords : -1;
   const size_t words_bytes = ((size_t)std::max(nwords, 0) * sizeof(int) + 255) & ~(size_t)255;
   const size_t ml_bytes = ((size_t)nsegs * 128 * sizeof(float2) + 255) & ~(size_t)255;
   const size_t acc_bytes = (size_t)nsegs * 128 * s.d * sizeof(float);
@@ -1623,19 +1696,23 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
   int* d_work = reinterpret_cast<int*>(scratch);
   float2* part_ml = reinterpret_cast<float2*>(scratch + words_bytes);
   float* part_acc = reinterpret_cast<float*>(scratch + words_bytes + ml_bytes);
+  const int D = s.d, G = s.Hq / s.H;
+  PlanMaps pm;
+  const uint64_t rows = (uint64_t)in.total_rows;
+  if (!make_row_maps(&pm.tok, in.tok, kChunk, rows * cpb)) return cudaErrorInvalidValue;
+  if (!make_row_maps(&pm.dim, in.dim, D, rows)) return cudaErrorInvalidValue;
+  if (!make_pacc_map(&pm.pacc, part_acc, nsegs, D)) return cudaErrorInvalidValue;
+  std::memcpy(g_noalloc_host_words + off_maps, &pm, sizeof(PlanMaps));
   // pageable source: the call returns once the words are staged, so the host buffer can be reused
   if ((e = cudaMemcpyAsync(d_work, g_noalloc_host_words, (size_t)nwords * sizeof(int), cudaMemcpyHostToDevice, st)) !=
       cudaSuccess)
     return e;
-  const int D = s.d, G = s.Hq / s.H;
   Maps maps;
-  const uint64_t rows = (uint64_t)in.total_rows;
-  if (!make_row_maps(&maps.tok, in.tok, kChunk, rows * cpb)) return cudaErrorInvalidValue;
-  if (!make_row_maps(&maps.dim, in.dim, D, rows)) return cudaErrorInvalidValue;
-  if (!make_pacc_map(&maps.pacc, part_acc, nsegs, D)) return cudaErrorInvalidValue;
   if (!make_call_maps(&maps, s, in, ipt)) return cudaErrorInvalidValue;
   Params p;
   p.recs = reinterpret_cast<const CtaRec*>(d_work + off_rec);
+  p.items = reinterpret_cast<const Item*>(d_work + off_items);
+  p.gmaps = reinterpret_cast<const PlanMaps*>(d_work + off_maps);
   p.segs = reinterpret_cast<const Seg*>(d_work + off_segs);
   p.ranks = in.ranks;
   p.row_offsets = in.row_offsets;
