@@ -9,7 +9,8 @@ Sources (page "MILO: Efficient Many-shot In-Context Learning with Block-wise
 Low-rank Compression", a section summary of the paper):
   §4.2  block-wise low-rank compression of keys and values, block by block;
   §4.3  entropy-driven rank allocation under a fixed total budget;
-  §4.4  workflow: encode (partition, entropy, low-rank store), then decode.
+  §4.4  workflow: encode (partition, entropy, low-rank store), then decode;
+  §5.3  composition with asymmetric INT8 quantisation (oracle/quant.py).
 
 Every function states the passage it follows and the reading taken where the
 page is silent.
@@ -35,4 +36,5 @@ from .milo import (  # noqa: F401
     stored_factors,
 )
 from .hestenes import hestenes_svd  # noqa: F401
+from .quant import dequantize_channel, quantize_block, quantize_channel, quantize_layer, quantize_pool  # noqa: F401
 from .tiefree import cut_gap, greedy_cut_gap, tiefree_taus  # noqa: F401
