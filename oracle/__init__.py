@@ -36,5 +36,6 @@ from .milo import (  # noqa: F401
     stored_factors,
 )
 from .hestenes import hestenes_svd  # noqa: F401
-from .quant import dequantize_channel, quantize_block, quantize_channel, quantize_layer, quantize_pool  # noqa: F401
+from .quant import (dequantize_channel, quantize_block, quantize_channel, quantize_channel_symmetric,  # noqa: F401
+                    quantize_layer, quantize_pool)
 from .tiefree import cut_gap, greedy_cut_gap, tiefree_taus  # noqa: F401

@@ -27,6 +27,10 @@ scheme beyond those names.  Readings taken here:
       B̂[:, r] = Σ_j (lo_j + 128·a_j)·B[:, j]
   so that codes_aug · B̂ᵀ = Σ_j x̂_j B_jᵀ exactly, and the decode of
   decode_attention runs unchanged on (codes_aug, B̂) at rank r + 1.
+* Blocks stored at full rank r = d, where one more component would exceed the
+  head dimension, use the symmetric form instead (zero point 0, no extra
+  component): a = max_t |x_t| / 127, c_t = round(x_t / a) in [−127, 127], x̂_t =
+  a·c_t (a = 0 gives c_t = 0), and B̂[:, j] = a_j·B[:, j] at rank d.
 """
 from __future__ import annotations
 
@@ -54,17 +58,36 @@ def dequantize_channel(codes, a, lo) -> np.ndarray:
     return float(a) * (np.asarray(codes, dtype=np.float64) + 128.0) + float(lo)
 
 
-def quantize_block(u, b) -> dict:
-    """One block's pair (U n×r, B d×r, stored values) → the 8-bit form at rank r + 1.
+def quantize_channel_symmetric(x) -> tuple[np.ndarray, np.float32]:
+    """One channel in the symmetric form (full-rank blocks) → (int8 codes in [−127, 127], scale a), fp32 decisions."""
+    x = np.asarray(x, dtype=np.float32)
+    a = np.float32(np.abs(x).max() / np.float32(127.0))
+    if a > 0:
+        c = np.clip(np.rint(x / a), -127, 127).astype(np.int32)
+    else:
+        c = np.zeros(x.shape, dtype=np.int32)
+    return c.astype(np.int8), a
 
-    Returns codes (n×r int8), scale and lo (r each, fp32), the dequantized
-    token factor u_hat (n×r), and the augmented pair U_aug (n×(r+1): the codes
-    as numbers, last column 1) and B_aug (d×(r+1), fp64) with
-    U_aug·B_augᵀ = u_hat·Bᵀ.
+
+def quantize_block(u, b) -> dict:
+    """One block's pair (U n×r, B d×r, stored values) → the 8-bit form at rank r + 1 (r < d) or r (r = d).
+
+    Returns codes (n×r int8), scale and lo (r each, fp32; lo = 0 in the
+    symmetric form), the dequantized token factor u_hat (n×r), and the stored
+    pair U_aug (the codes as numbers, plus a last column of 1 when r < d) and
+    B_aug (fp64) with U_aug·B_augᵀ = u_hat·Bᵀ.
     """
     u = np.asarray(u, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
     n, r = u.shape
+    if r >= b.shape[0]:  # full rank: symmetric, no extra component
+        codes = np.empty((n, r), dtype=np.int8)
+        scale = np.empty(r, dtype=np.float32)
+        for j in range(r):
+            codes[:, j], scale[j] = quantize_channel_symmetric(u[:, j])
+        u_hat = codes.astype(np.float64) * scale.astype(np.float64)[None, :]
+        return dict(codes=codes, scale=scale, lo=np.zeros(r, dtype=np.float32), u_hat=u_hat,
+                    U_aug=codes.astype(np.float64), B_aug=b * scale.astype(np.float64)[None, :])
     codes = np.empty((n, r), dtype=np.int8)
     scale = np.empty(r, dtype=np.float32)
     lo = np.empty(r, dtype=np.float32)
@@ -79,10 +102,11 @@ def quantize_block(u, b) -> dict:
 
 
 def quantize_pool(pool: dict) -> dict:
-    """A pool (compress_pool output, factors in stored values) → the same pool in 8-bit form at ranks r_b + 1.
+    """A pool (compress_pool output, factors in stored values) → the same pool in 8-bit form at ranks r_b + 1
+    (r_b at full rank).
 
-    The returned pool has U = the augmented codes, B = the augmented
-    dimension factors and ranks = r_b + 1, so decode_attention and
+    The returned pool has U = the stored codes, B = the folded dimension
+    factors and ranks = r_b + 1 (r_b at full rank), so decode_attention and
     reconstruct_pool take it as they are; it also keeps codes, scales,
     minima and the dequantized token factors per block.
     """
@@ -90,7 +114,7 @@ def quantize_pool(pool: dict) -> dict:
     out = dict(pool)
     out["U"] = [q["U_aug"] for q in blocks]
     out["B"] = [q["B_aug"] for q in blocks]
-    out["ranks"] = np.asarray(pool["ranks"]) + 1
+    out["ranks"] = np.array([q["U_aug"].shape[1] for q in blocks])
     out["codes"] = [q["codes"] for q in blocks]
     out["scale"] = [q["scale"] for q in blocks]
     out["lo"] = [q["lo"] for q in blocks]

@@ -63,29 +63,65 @@ def test_folded_scales_reproduce_the_dequantized_block():
     assert np.all(np.abs(q["u_hat"] - u) <= 0.5 * q["scale"].astype(np.float64) * (1 + 1e-5) + 1e-5)
 
 
-def _quantized_tiny():
+def _quantized_tiny(beta=None):
     wl = WORKLOADS["tiny"]
     L = gen_layer(wl)
     K, V = from_storage(L["K"], wl.dtype), from_storage(L["V"], wl.dtype)
-    lay = stored_layer(oracle.compress_layer(K, V, wl.block_size, wl.budgets[0], wl.r_min), "bf16")
+    beta = wl.budgets[0] if beta is None else beta
+    lay = stored_layer(oracle.compress_layer(K, V, wl.block_size, beta, wl.r_min), "bf16")
     return wl, L, lay, oracle.quantize_layer(lay)
+
+
+def test_symmetric_codes_hand_example():
+    # max |x| = 2: a = 2/127; 1/a = 63.5 rounds to 64 (half to even), 0.5/a = 31.75 rounds to 32
+    c, a = oracle.quantize_channel_symmetric([-2.0, 1.0, 0.5, 2.0])
+    assert list(c) == [-127, 64, 32, 127]
+    assert a == np.float32(2.0) / np.float32(127.0)
+    c, a = oracle.quantize_channel_symmetric(np.zeros(5))
+    assert a == 0.0 and np.all(c == 0)
+
+
+def test_full_rank_block_takes_the_symmetric_form():
+    rng = np.random.default_rng(4)
+    n, d = 256, 16
+    u = rng.standard_normal((n, d)) * rng.uniform(0.1, 10, d)
+    b = np.linalg.qr(rng.standard_normal((d, d)))[0]
+    q = oracle.quantize_block(u, b)
+    assert q["U_aug"].shape == (n, d) and q["B_aug"].shape == (d, d)  # no extra component at rank d
+    assert np.all(np.abs(q["codes"].astype(int)) <= 127)
+    assert np.allclose(q["U_aug"] @ q["B_aug"].T, q["u_hat"] @ b.T, rtol=0, atol=1e-12 * np.abs(u).max())
+    assert np.all(np.abs(q["u_hat"] - u) <= 0.5 * q["scale"].astype(np.float64) * (1 + 1e-5) + 1e-5)
+    for j in range(d):  # the largest magnitude of each channel maps to ±127
+        t = np.argmax(np.abs(u[:, j]))
+        assert abs(int(q["codes"][t, j])) == 127
 
 
 def test_quantized_layer_ranks_and_shapes():
     _, _, lay, ql = _quantized_tiny()
     for t in ("K", "V"):
         for p, qp in zip(lay[t], ql[t]):
-            assert np.array_equal(qp["ranks"], np.asarray(p["ranks"]) + 1)
+            d = p["B"][0].shape[0]
+            want = np.where(np.asarray(p["ranks"]) < d, np.asarray(p["ranks"]) + 1, np.asarray(p["ranks"]))
+            assert np.array_equal(qp["ranks"], want)
             for u, qu, qb in zip(p["U"], qp["U"], qp["B"]):
-                assert qu.shape == (u.shape[0], u.shape[1] + 1) and qb.shape[1] == u.shape[1] + 1
-                assert np.all((qu[:, :-1] >= -128) & (qu[:, :-1] <= 127)) and np.all(qu[:, -1] == 1)
+                r = u.shape[1]
+                extra = 1 if r < d else 0
+                assert qu.shape == (u.shape[0], r + extra) and qb.shape[1] == r + extra
+                assert np.all((qu[:, :r] >= -128) & (qu[:, :r] <= 127))
+                if extra:
+                    assert np.all(qu[:, -1] == 1)
 
 
-def test_decode_over_8bit_factors_is_attention_over_dequantized_cache():
+@pytest.mark.parametrize("beta", [None, 0.75, 1.25])
+def test_decode_over_8bit_factors_is_attention_over_dequantized_cache(beta):
     """Rank-space decode on (codes, folded B) equals plain softmax attention over the dense keys and values
     rebuilt from the dequantized token factors: a dropped zero-point column, a wrong sign of the offset or a
-    scale on the wrong side changes the keys and fails this."""
-    wl, L, lay, ql = _quantized_tiny()
+    scale on the wrong side changes the keys and fails this.  Budgets: every block below full rank
+    (asymmetric), some blocks at full rank (both forms), every block at full rank (symmetric)."""
+    wl, L, lay, ql = _quantized_tiny(beta)
+    d = wl.head_dim
+    full = sum(int(np.sum(np.asarray(p["ranks"]) == d)) for t in ("K", "V") for p in lay[t])
+    print(f"budget {beta}: {full} blocks at full rank")
     q = from_storage(L["q"], wl.dtype)
     Ks, Vs = from_storage(L["K_suf"], wl.dtype), from_storage(L["V_suf"], wl.dtype)
     got = oracle.decode_attention(q, ql, Ks, Vs)
