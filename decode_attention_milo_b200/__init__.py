@@ -12,10 +12,10 @@ import os
 
 import numpy as np
 
-__all__ = ["F32", "BF16", "MiloError", "Factors", "compress", "decode_attn", "import_factors", "lib_path",
-           "load_library"]
+__all__ = ["F32", "BF16", "I8", "MiloError", "Factors", "compress", "decode_attn", "import_factors", "lib_path",
+           "load_library", "quantize"]
 
-F32, BF16 = 0, 1
+F32, BF16, I8 = 0, 1, 2  # I8: factor objects only (int8 token factors, bf16 dimension factors)
 KEEP_INTERMEDIATES = 1
 ALLOC_RULES = {"entropy": 0, "greedy": 1, "uniform": 2, "weights": 3}
 POOL_SCOPES = {"pool": 0, "layer": 1}
@@ -89,9 +89,11 @@ def load_library(path: str | None = None):
     L.milo_factors_status.argtypes = [vp, ctypes.POINTER(u32)]
     L.milo_factors_import.restype = i32
     L.milo_factors_import.argtypes = [i32, i32, i64, i32, i32, i32, vp, vp, vp, vp, ctypes.POINTER(vp)]
+    L.milo_factors_quantize.restype = i32
+    L.milo_factors_quantize.argtypes = [vp, vp, ctypes.POINTER(vp)]
     L.milo_factors_destroy.restype = None
     L.milo_factors_destroy.argtypes = [vp]
-    if L.milo_abi_version() != 2:
+    if L.milo_abi_version() != 3:
         raise RuntimeError("libmilo.so ABI version mismatch")
     _lib = L
     return L
@@ -243,7 +245,7 @@ def _decode_args(q, factors: Factors, K_suf, V_suf, out):
     returns (batch, q heads, suffix length, out)."""
     import torch
     H, d, dt = factors.shape()
-    want = torch.bfloat16 if dt == BF16 else torch.float32
+    want = torch.bfloat16 if dt in (BF16, I8) else torch.float32
     if q.dim() != 3 or q.shape[2] != d or q.shape[1] % H != 0 or q.shape[0] < 1:
         raise ValueError(f"q must be [batch][q_heads][{d}] with q_heads a multiple of {H}, got {tuple(q.shape)}")
     if q.dtype != want:
@@ -318,16 +320,30 @@ def decode_attn_noalloc(q, factors: Factors, K_suf=None, V_suf=None, scale: floa
 
 def import_factors(dtype: int, num_kv_heads: int, context: int, head_dim: int, block_size: int, r_min: int,
                    ranks: np.ndarray, tok: np.ndarray, dim: np.ndarray, stream=None) -> Factors:
-    """Builds a factor object from host arrays in the library's layout (tok [rows][n], dim [rows][d])."""
+    """Builds a factor object from host arrays in the library's layout (tok [rows][n], dim [rows][d]); with
+    dtype I8, tok holds int8 codes and dim bf16 bit patterns (2-byte elements)."""
     ranks = np.ascontiguousarray(ranks, dtype=np.int32)
     tok = np.ascontiguousarray(tok)
     dim = np.ascontiguousarray(dim)
+    rows = int(ranks.sum())
+    tok_bytes, dim_bytes = {F32: (4, 4), BF16: (2, 2), I8: (1, 2)}.get(dtype, (0, 0))
+    if tok.nbytes != rows * block_size * tok_bytes or dim.nbytes != rows * head_dim * dim_bytes:
+        raise ValueError(f"tok must hold {rows}x{block_size} and dim {rows}x{head_dim} elements of dtype code {dtype}")
     h = ctypes.c_void_p()
     _check(load_library().milo_factors_import(dtype, num_kv_heads, context, head_dim, block_size, r_min,
                                               ranks.ctypes.data_as(ctypes.c_void_p),
                                               tok.ctypes.data_as(ctypes.c_void_p),
                                               dim.ctypes.data_as(ctypes.c_void_p), _stream_ptr(stream),
                                               ctypes.byref(h)), "milo_factors_import")
+    return Factors(h)
+
+
+def quantize(factors: Factors, stream=None) -> Factors:
+    """8-bit copy of a bf16 factor object (int8 token factors per rank channel, scales folded into the bf16
+    dimension factors at rank r + 1). See milo_factors_quantize."""
+    h = ctypes.c_void_p()
+    _check(load_library().milo_factors_quantize(factors.handle, _stream_ptr(stream), ctypes.byref(h)),
+           "milo_factors_quantize")
     return Factors(h)
 
 

@@ -43,6 +43,10 @@ namespace {
 // warps 2 and 3 are idle and warpgroup 0 holds only the producer and the issuer).
 constexpr int kSoftWarp0 = 2;
 constexpr int kThreads = 32 * (kSoftWarp0 + 8);
+// 8-bit mode: two more warps (kConvWarp0, kConvWarp0 + 1) convert the int8 token-factor tiles to bf16
+constexpr int kConvWarp0 = kSoftWarp0 + 8;
+template <bool Q8>
+constexpr int threads_of() { return Q8 ? kThreads + 64 : kThreads; }
 // Register split (setmaxnreg, needs kSoftWarp0 = 4): warpgroup 0 gives registers to the two softmax
 // warpgroups.  The split must fit in what the launch allocates (kThreads × kLaunchRegs), or the increase
 // would wait forever: the host refuses a build whose kernel was allocated fewer registers.
@@ -53,8 +57,7 @@ static_assert(!kRegSplit || (kSoftWarp0 == 4 && 128 * kRegsLow + 256 * kRegsHigh
 constexpr int kSigThreads = 288;  // softmax warps + MMA warp on a signal barrier
 // named barriers (0 is __syncthreads): softmax warps → MMA warp (P alternates by S slot), one per TMEM
 // lane quarter for its two softmax warps, and one for all softmax warps
-constexpr int kSigQt = 1, kSigAt = 2, kSigP0 = 3, kPairBar0 = 5, kSoftBar = 9;
-constexpr int kRingBytes = 122880;  // TMA ring: variable-size items, each one contiguous tile
+constexpr int kSigQt = 1, kSigAt = 2, kSigP0 = 3, kPairBar0 = 5, kSoftBar = 9, kConvBar = 10;
 constexpr int kItemSlots = 16;       // items in flight at most (one FULL/EMPTY barrier pair each)
 constexpr int kChunk = 128;          // tokens per score chunk
 constexpr uint64_t kWaitNs = 1000000000ull;
@@ -64,15 +67,25 @@ constexpr uint32_t kSleepNs = 2000;  // suspend-time hint of one try_wait in a w
 constexpr int kOffQ = 0;          // [cb][128 rows][128 B]  query rows, K-major over d
 constexpr int kOffQtHi = 32768;   // [cb][128][128 B]  q̃ high part, K-major over rank
 constexpr int kOffQtLo = 65536;   // [cb][128][128 B]  q̃ low part
-constexpr int kOffRing = 98304;   // kRingBytes of items laid out [64-column block][rows][128 B]
-constexpr int kOffBar = kOffRing + kRingBytes;             // 221184: barriers, then the Shared block
+constexpr int kOffStage = 98304;  // 8-bit mode: [2][kStageBytes] bf16 token-factor tiles converted from the ring
+constexpr int kStageBytes = 32768;
 constexpr int kBarRegion = 8192;
-constexpr int kSmemBytes = kOffBar + kBarRegion + 1024;     // + alignment slack (230400)
+// The TMA ring (variable-size items, each one contiguous tile laid out [64-column block][rows][128 B]), then the
+// barriers and the Shared block.  The 8-bit mode gives part of the ring to the two staging tiles.
+template <bool Q8>
+struct Smem {
+  static constexpr int kOffRing = Q8 ? kOffStage + 2 * kStageBytes : 98304;
+  static constexpr int kRingBytes = Q8 ? 59392 : 122880;
+  static constexpr int kOffBar = kOffRing + kRingBytes;
+  static constexpr int kBytes = kOffBar + kBarRegion + 1024;  // + alignment slack
+};
+static_assert(Smem<false>::kBytes <= 232448 && Smem<true>::kBytes <= 232448, "227 KB of shared memory per CTA");
 constexpr uint32_t kTileCb = 16384;  // column-block stride of a 128-row tile
 constexpr int kMaxSegsSmem = 16, kMaxBlocksSmem = 64;  // per-CTA work tables staged in smem
 
 // TMEM columns: acc [0,128), two S slots [128,256) and [256,384) (q̃ of a block also passes through
-// an S slot; p is packed over the scores it came from), ã [384,512) (packed in place for G4)
+// an S slot; p is packed over the scores it came from), ã [384,512) (packed in place for G4 as bf16 high
+// and low parts)
 constexpr uint32_t kTmAcc = 0, kTmS0 = 128, kTmA = 384;
 
 // TMEM column, relative to its region, of k-step t (16 bf16) of an A operand that the two softmax
@@ -90,7 +103,9 @@ enum Bar {
   B_ATFULL = B_SFREE + 2, // ã of a block complete
   B_ACCDONE,              // acc written (G4, or a suffix segment's last G3')
   B_FINAL,
-  B_COUNT
+  B_STAGED,               // [2] 8-bit mode: bf16 staging tile k written by the converter warps
+  B_STFREE = B_STAGED + 2,  // [2] 8-bit mode: staging tile k read by the MMAs
+  B_COUNT = B_STFREE + 2
 };
 
 struct Seg {
@@ -263,11 +278,12 @@ __device__ __forceinline__ Seg get_seg(const Params& p, const Shared* sh, int s_
 // Placement of items in the TMA ring.  Producer and consumer call place() with the same sizes in the same
 // order, so they agree on every item's offset without exchanging it; an item that does not fit before the
 // end of the ring starts at offset 0.
+template <int kRing>
 struct RingPlace {
   uint32_t head = 0;  // next free byte offset
   uint32_t n = 0;     // items placed so far
   __device__ uint32_t place(uint32_t bytes) {
-    const uint32_t pos = head + bytes <= (uint32_t)kRingBytes ? head : 0u;
+    const uint32_t pos = head + bytes <= (uint32_t)kRing ? head : 0u;
     head = pos + bytes;
     ++n;
     return pos;
@@ -305,20 +321,22 @@ __device__ __forceinline__ void st_tile8(uint32_t tile, int row, int col, uint32
   ptx::st_shared_v4(addr, a, b, c, d);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, bool Q8>
+__global__ void __launch_bounds__(threads_of<Q8>(), 1)
     decode_tc_kernel(const __grid_constant__ Maps maps,
                      const Params p) {
   constexpr int NCB = D / 64;
+  using L = Smem<Q8>;
+  constexpr int kNThreads = threads_of<Q8>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t base = ptx::smem_u32(smem);
-  Shared* sh = reinterpret_cast<Shared*>(smem + kOffBar + kSharedOff);
-  auto bar = [&](int i) { return base + kOffBar + 8 * i; };
+  Shared* sh = reinterpret_cast<Shared*>(smem + L::kOffBar + kSharedOff);
+  auto bar = [&](int i) { return base + L::kOffBar + 8 * i; };
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   // ---- setup: zero the query tile (rows no TMA box writes stay finite), barriers, TMEM
-  for (int i = threadIdx.x; i < 32768 / 16; i += kThreads) ptx::st_shared_v4(base + kOffQ + 16 * i, 0, 0, 0, 0);
+  for (int i = threadIdx.x; i < 32768 / 16; i += kNThreads) ptx::st_shared_v4(base + kOffQ + 16 * i, 0, 0, 0, 0);
   if (threadIdx.x == 0) {
     for (int i = 0; i < kItemSlots; ++i) {
       ptx::mbar_init(bar(B_FULL + i), 1);
@@ -333,6 +351,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(bar(B_ATFULL), 1);
     ptx::mbar_init(bar(B_ACCDONE), 1);
     ptx::mbar_init(bar(B_FINAL), 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(bar(B_STAGED + i), 1);
+      ptx::mbar_init(bar(B_STFREE + i), 1);
+    }
     sh->abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -348,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   {
     const int4* src = reinterpret_cast<const int4*>(p.recs + blockIdx.x);
     int4* dst = reinterpret_cast<int4*>(&sh->rec);
-    for (int i = threadIdx.x; i < (int)(sizeof(CtaRec) / 16); i += kThreads) dst[i] = src[i];
+    for (int i = threadIdx.x; i < (int)(sizeof(CtaRec) / 16); i += kNThreads) dst[i] = src[i];
   }
   __syncthreads();
   const int s_begin = sh->rec.s_begin, s_end = sh->rec.s_end;
@@ -405,8 +427,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t fb = bar(B_FULL + ring_n % kItemSlots);
         if (lane == 0) {
           ptx::mbar_arrive_expect_tx(fb, bytes);
-          if (kind == kItem3D) ptx::tma_load_3d(base + kOffRing + a, tm, fb, 0, y, 0);
-          else ptx::tma_load_2d(base + kOffRing + a, tm, fb, 0, y);
+          if (kind == kItem3D) ptx::tma_load_3d(base + L::kOffRing + a, tm, fb, 0, y, 0);
+          else ptx::tma_load_2d(base + L::kOffRing + a, tm, fb, 0, y);
         }
         __syncwarp();
         ++ring_n;
@@ -428,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kSigThreads) : "memory");
       ptx::tc_fence_after();
     };
-    RingPlace ring;                      // consumer view of the TMA ring
+    RingPlace<L::kRingBytes> ring;       // consumer view of the TMA ring
     uint32_t cur = 0;                    // item being consumed
     uint32_t use_i = 0, use_c = 0;       // S-slot uses issued / consumed (signalled)
     uint32_t q_uses = 0;
@@ -438,11 +460,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t pos = ring.place((uint32_t)rows * 128u * ncb);
       if (!wait_bar(bar(B_FULL + cur % kItemSlots), (cur / kItemSlots) & 1, sh, p.status)) return false;
       ptx::tc_fence_after();
-      addr = base + kOffRing + pos;
+      addr = base + L::kOffRing + pos;
       return true;
     };
     auto release = [&]() {  // the item's space is free once the MMAs issued so far have read it
       if (leader) ptx::umma_commit(bar(B_EMPTY + cur % kItemSlots));
+    };
+    // Token-factor tiles (U, P).  In the 8-bit mode the converter warps turn the ring's int8 tile into a bf16
+    // staging tile and release the ring item themselves; the MMAs read the staging tile, which is free again
+    // once they complete.
+    uint32_t staged = 0, stage_k = 0;  // staging tiles consumed; the tile of the current item
+    auto take_tok = [&](int rows, uint32_t& addr) -> bool {
+      if (!Q8) return take(rows, 2, addr);
+      cur = ring.n;
+      ring.place((uint32_t)rows * 128u);  // one byte per token: the ring holds the codes
+      stage_k = staged & 1;
+      const bool got = wait_bar(bar(B_STAGED + stage_k), (staged >> 1) & 1, sh, p.status);
+      ++staged;
+      if (!got) return false;
+      ptx::tc_fence_after();
+      addr = base + kOffStage + stage_k * kStageBytes;
+      return true;
+    };
+    auto release_tok = [&]() {
+      if (!Q8) release();
+      else if (leader) ptx::umma_commit(bar(B_STFREE + stage_k));
     };
     auto commit = [&](int b) {
       if (leader) ptx::umma_commit(bar(b));
@@ -481,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto g2 = [&](int rk) -> bool {
       const int rp = pad16(rk);
       uint32_t it;
-      if (!slot_free(use_i & 1) || !take(rp, 2, it)) return false;
+      if (!slot_free(use_i & 1) || !take_tok(rp, it)) return false;
       if (leader) {
         const uint32_t d = tmem + kTmS0 + 128 * (use_i & 1);
         const uint64_t db = mndesc(it, 0, (uint32_t)rp * 128u);
@@ -492,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::umma_bf16(d, dl + kstep(t, kTileCb), bd, idS, 1);
         }
       }
-      release();
+      release_tok();
       s_commit();
       return true;
     };
@@ -500,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto g3 = [&](int rv, bool fresh, uint32_t s) -> bool {
       const int rp = pad16(rv);
       uint32_t it;
-      if (!take(rp, 2, it)) return false;
+      if (!take_tok(rp, it)) return false;
       if (leader) {
         const uint64_t db = kdesc(it, 0, 0);
         const uint32_t cbs = (uint32_t)rp * 128u, id = ptx::idesc_bf16(128, rp, false, false);
@@ -509,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < kChunk / 16; ++t)
           ptx::umma_bf16_ta(tmem + kTmA, a + ta_col(t), db + kstep(t, cbs), id, (t > 0 || !fresh) ? 1u : 0u);
       }
-      release();
+      release_tok();
       p_commit(s);
       return true;
     };
@@ -520,9 +562,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!take(rp, NCB, it)) return false;
       if (leader) {
         const uint64_t db = mndesc(it, 0, (uint32_t)rp * 128u);
-        for (int t = 0; t < rp / 16; ++t)
-          ptx::umma_bf16_ta(tmem + kTmAcc, tmem + kTmA + ta_col(t), db + (uint64_t)(t * 128), idD,
-                            (t > 0 || !fresh) ? 1u : 0u);
+        for (int t = 0; t < rp / 16; ++t) {  // ã's high part, then its low part (32 columns further)
+          const uint64_t bd = db + (uint64_t)(t * 128);
+          ptx::umma_bf16_ta(tmem + kTmAcc, tmem + kTmA + ta_col(t), bd, idD, (t > 0 || !fresh) ? 1u : 0u);
+          ptx::umma_bf16_ta(tmem + kTmAcc, tmem + kTmA + ta_col(t) + 32, bd, idD, 1u);
+        }
       }
       release();
       commit(B_ACCDONE);
@@ -659,6 +703,62 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     wait_bar(bar(B_FINAL), 0, sh, p.status, true);
   }
+  } else if (Q8 && warp >= kConvWarp0) {
+    // ==================================================================== 8-bit converter (two warps)
+    // Follows the producer's item list and turns every int8 token-factor tile of the ring into the bf16 tile
+    // that the MMAs read, in one of two staging tiles: the codes c in [-128, 127] are exact in bf16.  The ring
+    // item is released as soon as it has been read; the staging tile when the MMAs that read it complete.
+    const int ct = threadIdx.x - 32 * kConvWarp0;  // 0..63
+    const Item* items = p.items + sh->rec.item0;
+    const int nitems = sh->rec.nitems;
+    uint32_t ring_n = 0, staged = 0;
+    // The loop depends only on the item list: after a failed wait both warps still take the same barriers.
+    for (int i = 0; i < nitems; ++i) {
+      const uint4 it = __ldg(reinterpret_cast<const uint4*>(items + i));
+      const uint32_t kind = (it.w >> 8) & 3u, mi = it.w & 255u;
+      if (kind == kItemQ) continue;
+      const uint32_t ri = ring_n++;
+      if (mi >= (uint32_t)kMapTok + 8) continue;  // not a token-factor tile
+      const uint32_t k = staged & 1;
+      bool got = wait_bar(bar(B_FULL + ri % kItemSlots), (ri / kItemSlots) & 1, sh, p.status);
+      if (got) got = wait_bar(bar(B_STFREE + k), ((staged >> 1) & 1) ^ 1, sh, p.status);
+      ++staged;
+      got = ptx::bar_and(kConvBar, 64, got);
+      if (got) {
+        ptx::tc_fence_after();
+        const int rows = (int)(it.z >> 7);  // one byte per token, 128 tokens per row
+        const uint32_t src = base + L::kOffRing + it.x;
+        const uint32_t dst = base + kOffStage + k * kStageBytes;
+        // unit (row j, 16-byte chunk c): the 16 codes of tokens 16c .. 16c + 15, read from the TMA's 128-byte
+        // swizzled row and written as two 16-byte bf16 chunks of the [64-token block][rows][128 B] tile
+        for (int u = ct; u < rows * 8; u += 64) {
+          const int j = u >> 3, c = u & 7;
+          const uint4 w = ptx::ld_shared_v4(src + (uint32_t)j * 128u + ((uint32_t)(c ^ (j & 7)) << 4));
+          const uint32_t wd[4] = {w.x ^ 0x80808080u, w.y ^ 0x80808080u, w.z ^ 0x80808080u, w.w ^ 0x80808080u};
+          uint32_t o[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            // byte b = c + 128 as the low mantissa bits of 2^23: (2^23 + b) − (2^23 + 128) = c exactly
+            float f[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              f[e] = __uint_as_float(__byte_perm(wd[q], 0x4B000000u, 0x7540u | e)) - 8388736.0f;
+            o[2 * q] = __byte_perm(__float_as_uint(f[0]), __float_as_uint(f[1]), 0x7632u);
+            o[2 * q + 1] = __byte_perm(__float_as_uint(f[2]), __float_as_uint(f[3]), 0x7632u);
+          }
+          const uint32_t row = dst + (uint32_t)(c >> 2) * (uint32_t)rows * 128u + (uint32_t)j * 128u;
+          const int ch = 2 * (c & 3);
+          ptx::st_shared_v4(row + ((uint32_t)(ch ^ (j & 7)) << 4), o[0], o[1], o[2], o[3]);
+          ptx::st_shared_v4(row + ((uint32_t)((ch + 1) ^ (j & 7)) << 4), o[4], o[5], o[6], o[7]);
+        }
+        ptx::fence_async_smem();
+      }
+      asm volatile("bar.sync %0, 64;" ::"r"(kConvBar) : "memory");
+      if (got && ct == 0) {
+        ptx::mbar_arrive(bar(B_EMPTY + ri % kItemSlots));  // the codes have been read
+        ptx::mbar_arrive(bar(B_STAGED + k));
+      }
+    }
   } else {
   if (kRegSplit) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
   {
@@ -716,7 +816,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       signal(kSigQt);
       return got;
     };
-    // ã (fp32, TMEM) → packed bf16 in place (warpgroup wg: columns [64wg, 64wg + 32)), ranks >= r zeroed
+    // ã (fp32, TMEM) → bf16 high and low parts packed in place (warpgroup wg: ranks [64wg, 64wg + 64), high
+    // part in columns [64wg, 64wg + 32), low part in [64wg + 32, 64wg + 64)), ranks >= r zeroed.  G4 takes both,
+    // so that ã keeps about 16 bits: with 8-bit factors its entries are sums of codes whose large terms cancel
+    // against the zero-point component, and one bf16 rounding of them would be visible in the output.
     auto convert_at = [&](bool active, int rv) -> bool {
       const bool got = wait_bar(bar(B_ATFULL), at_uses & 1, sh, p.status);
       ++at_uses;
@@ -724,20 +827,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (got) {
         ptx::tc_fence_after();
         if (active && 64 * wg < pad16(rv)) {
-          // 32 columns at a time: packed half h lands on columns [16h, 16h + 16), which half 0 has read
-#pragma unroll 1
-          for (int h = 0; h < 2; ++h) {
-            float v[32];
-            ptx::tmem_ld32(tl + kTmA + 64 * wg + 32 * h, v);
-            ptx::tmem_wait_ld();
-            uint32_t wv[16];
+          // half h's high part lands on columns [16h, 16h + 16) (half 0's, read first) and its low part on
+          // [32 + 16h, 32 + 16h + 16) (half 1's): half 0's low part waits until half 1 has been read
+          const uint32_t at = tl + kTmA + 64 * wg;
+          auto split = [&](const float* v, int h, uint32_t* hi, uint32_t* lo) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int r0 = 64 * wg + 32 * h + 2 * e;
-              wv[e] = ptx::pack_bf16(r0 < rv ? v[2 * e] : 0.f, r0 + 1 < rv ? v[2 * e + 1] : 0.f);
+              const float a = r0 < rv ? v[2 * e] : 0.f;
+              const float b2 = r0 + 1 < rv ? v[2 * e + 1] : 0.f;
+              hi[e] = ptx::pack_bf16(a, b2);
+              lo[e] = ptx::pack_bf16(a - __uint_as_float(hi[e] << 16), b2 - __uint_as_float(hi[e] & 0xFFFF0000u));
             }
-            ptx::tmem_st16u(tl + kTmA + 64 * wg + 16 * h, wv);
-          }
+          };
+          float v[32];
+          uint32_t hi[16], lo0[16], lo1[16];
+          ptx::tmem_ld32(at, v);
+          ptx::tmem_wait_ld();
+          split(v, 0, hi, lo0);
+          ptx::tmem_st16u(at, hi);
+          ptx::tmem_ld32(at + 32, v);
+          ptx::tmem_wait_ld();
+          ptx::tmem_st16u(at + 32, lo0);
+          split(v, 1, hi, lo1);
+          ptx::tmem_st16u(at + 16, hi);
+          ptx::tmem_st16u(at + 48, lo1);
           ptx::tmem_wait_st();
         }
       }
@@ -1061,7 +1175,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
-              const uint32_t* box) {
+              const uint32_t* box, CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gd[3], gs[2];
@@ -1071,20 +1185,36 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, c
     bx[i] = box[i];
   }
   for (int i = 0; i + 1 < rank; ++i) gs[i] = strides_bytes[i];
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), gd, gs, bx, es,
+  return fn(m, dt, rank, const_cast<void*>(ptr), gd, gs, bx, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Prepares the decode kernel for head dimension d: its shared-memory size, and a check that the launch
 // allocates the registers that the kernel's register split (setmaxnreg) redistributes.
-cudaError_t prepare_kernel(int d) {
-  const void* kfn = d == 64 ? (const void*)decode_tc_kernel<64> : (const void*)decode_tc_kernel<128>;
+template <bool Q8>
+const void* kernel_of(int d) {
+  return d == 64 ? (const void*)decode_tc_kernel<64, Q8> : (const void*)decode_tc_kernel<128, Q8>;
+}
+cudaError_t prepare_kernel(int d, bool q8) {
+  const void* kfn = q8 ? kernel_of<true>(d) : kernel_of<false>(d);
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, kfn);
   if (e != cudaSuccess) return e;
   if (kRegSplit && fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
-  return cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  return cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              q8 ? Smem<true>::kBytes : Smem<false>::kBytes);
+}
+// Launches the decode kernel of head dimension d and mode q8.
+cudaError_t launch_decode_kernel(int d, bool q8, int grid, const Maps& maps, const Params& p, cudaStream_t st) {
+  if (q8) {
+    if (d == 64) decode_tc_kernel<64, true><<<grid, threads_of<true>(), Smem<true>::kBytes, st>>>(maps, p);
+    else decode_tc_kernel<128, true><<<grid, threads_of<true>(), Smem<true>::kBytes, st>>>(maps, p);
+  } else {
+    if (d == 64) decode_tc_kernel<64, false><<<grid, threads_of<false>(), Smem<false>::kBytes, st>>>(maps, p);
+    else decode_tc_kernel<128, false><<<grid, threads_of<false>(), Smem<false>::kBytes, st>>>(maps, p);
+  }
+  return cudaGetLastError();
 }
 
 // The map of a [rows][width] bf16 array with boxes of h rows: 3D for 128 columns (x: 64 columns, y: rows,
@@ -1104,6 +1234,16 @@ bool make_row_maps(RowMaps* rm, const void* ptr, uint64_t width, uint64_t rows) 
   std::memset(rm, 0, sizeof(RowMaps));
   for (int k = 0; k < 8; ++k)
     if (!make_rows_map(&rm->m[k], ptr, width, rows, 16u * (k + 1))) return false;
+  return true;
+}
+// The same for the int8 codes of an 8-bit token factor: [rows][128] bytes, boxes of 128 bytes × h rows.
+bool make_code_maps(RowMaps* rm, const void* ptr, uint64_t rows) {
+  std::memset(rm, 0, sizeof(RowMaps));
+  const uint64_t d2[2] = {128, rows}, s2[1] = {128};
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t b2[2] = {128, 16u * (k + 1)};
+    if (!make_map(&rm->m[k], ptr, 2, d2, s2, b2, CU_TENSOR_MAP_DATA_TYPE_UINT8)) return false;
+  }
   return true;
 }
 
@@ -1154,6 +1294,7 @@ struct TcPlan {
   const void* tok = nullptr;
   const void* dim = nullptr;
   PlanMaps* d_maps = nullptr;  // the factor and partial maps in device memory
+  bool q8 = false;             // 8-bit token factors
 };
 
 bool tc_shape_ok(const DecodeShape& s) {
@@ -1375,7 +1516,8 @@ constexpr int kRecWords = (int)(sizeof(CtaRec) / sizeof(int));
 // at most `cap` items to `out` and sets every record's item range; returns the item count, or -1 when `cap` is
 // too small, a coordinate does not fit the TMA's 32 bits or a rank lies outside [1, d].
 int64_t build_items(const DecodeShape& s, const int32_t* host_ranks, const int* w, int grid, int off_segs,
-                    int off_sel, CtaRec* recs, Item* out, int64_t cap) {
+                    int off_sel, CtaRec* recs, Item* out, int64_t cap, bool q8) {
+  const uint32_t ring_bytes = q8 ? Smem<true>::kRingBytes : Smem<false>::kRingBytes;
   const int nb = s.nb, cpb = s.n / kChunk, G = s.Hq / s.H, ncb = s.d / 64;
   const int ipt = std::min(s.Bq, 128 / G);
   std::vector<int64_t> row0((size_t)2 * s.H * nb);
@@ -1401,7 +1543,7 @@ int64_t build_items(const DecodeShape& s, const int32_t* host_ranks, const int* 
     auto ring = [&](int map, int64_t y, int rows, int nc) {  // `map`: the item's final map index
       if (y > INT32_MAX || rows < 16 || rows > 128) fits = false;
       const uint32_t bytes = (uint32_t)rows * 128u * nc;
-      const uint32_t pos = head + bytes <= (uint32_t)kRingBytes ? head : 0u;
+      const uint32_t pos = head + bytes <= ring_bytes ? head : 0u;
       uint32_t retire = 0;
       while (oldest < n) {
         const uint32_t tail = pos_of[oldest % kItemSlots];
@@ -1448,7 +1590,8 @@ int64_t build_items(const DecodeShape& s, const int32_t* host_ranks, const int* 
       };
       auto dim_item = [&](int64_t r0, int r) { ring(kMapDim + pad(r) / 16 - 1, r0, pad(r), ncb); };
       auto tok_item = [&](int64_t r0, int r, int cc) {
-        ring(kMapTok + pad(r) / 16 - 1, r0 * cpb + (int64_t)cc * r, pad(r), 2);
+        // bf16: two 64-token column blocks; 8-bit: one 128-byte row of codes per component
+        ring(kMapTok + pad(r) / 16 - 1, r0 * cpb + (int64_t)cc * r, pad(r), q8 ? 1 : 2);
       };
       int c = sg.c0;
       BI bi = info(c / cpb), prev{};
@@ -1520,7 +1663,7 @@ static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& 
   host.resize((size_t)off_items + (size_t)icap * kItemWords);
   recs = reinterpret_cast<CtaRec*>(host.data() + pl->off_rec);
   const int64_t nitems = build_items(s, in.host_ranks, host.data(), grid, off_segs, pl->off_sel, recs,
-                                     reinterpret_cast<Item*>(host.data() + off_items), icap);
+                                     reinterpret_cast<Item*>(host.data() + off_items), icap, in.q8);
   if (nitems < 0 || off_items + nitems * kItemWords > INT32_MAX) return cudaErrorInvalidValue;
   pl->off_items = off_items;
   const int nwords_all = (int)(off_items + nitems * kItemWords);
@@ -1546,14 +1689,16 @@ static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& 
   // as [rows][d]
   const uint64_t rows = (uint64_t)in.total_rows;
   PlanMaps pm;
-  if (!make_row_maps(&pm.tok, in.tok, kChunk, rows * cpb)) return cudaErrorInvalidValue;
+  if (!(in.q8 ? make_code_maps(&pm.tok, in.tok, rows * cpb) : make_row_maps(&pm.tok, in.tok, kChunk, rows * cpb)))
+    return cudaErrorInvalidValue;
   if (!make_row_maps(&pm.dim, in.dim, D, rows)) return cudaErrorInvalidValue;
   if (!make_pacc_map(&pm.pacc, pl->part_acc, pl->nsegs, D)) return cudaErrorInvalidValue;
   if ((e = cudaMalloc((void**)&pl->d_maps, sizeof(PlanMaps))) != cudaSuccess) return e;
   if ((e = cudaMemcpy(pl->d_maps, &pm, sizeof(PlanMaps), cudaMemcpyHostToDevice)) != cudaSuccess) return e;
   pl->tok = in.tok;
   pl->dim = in.dim;
-  return prepare_kernel(D);
+  pl->q8 = in.q8;
+  return prepare_kernel(D, in.q8);
 }
 
 cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, void* out, cudaStream_t st,
@@ -1562,7 +1707,8 @@ cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, v
   const bool same_mask = pl && (mask ? pl->mask.size() == (size_t)s.H * s.nb &&
                                            std::memcmp(pl->mask.data(), mask, pl->mask.size()) == 0
                                      : pl->mask.empty());
-  if (!pl || pl->Bq != s.Bq || pl->Hq != s.Hq || pl->S != s.S || pl->tok != in.tok || !same_mask) {
+  if (!pl || pl->Bq != s.Bq || pl->Hq != s.Hq || pl->S != s.S || pl->tok != in.tok || pl->q8 != in.q8 ||
+      !same_mask) {
     tc_plan_destroy(pl);
     *plan = nullptr;
     pl = new TcPlan();
@@ -1596,11 +1742,7 @@ cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, v
   p.c = s.scale * 1.4426950408889634f;
   cudaError_t e;
   if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
-  if (D == 64)
-    decode_tc_kernel<64><<<pl->grid, kThreads, kSmemBytes, st>>>(maps, p);
-  else
-    decode_tc_kernel<128><<<pl->grid, kThreads, kSmemBytes, st>>>(maps, p);
-  e = cudaGetLastError();
+  e = launch_decode_kernel(D, in.q8, pl->grid, maps, p, st);
   if (e != cudaSuccess) return e;
   if (ev1 && (e = cudaEventRecord(ev1, st)) != cudaSuccess) return e;
   const int* pre = pl->d_work + pl->off_pre;
@@ -1623,7 +1765,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 std::mutex g_noalloc_mu;
 void* g_noalloc_dev_ptr[kNoAllocMaxDevices];  // device address of g_noalloc_scratch, per device
-bool g_noalloc_ready[kNoAllocMaxDevices][2];  // decode kernel prepared on the device, per head dim (64, 128)
+bool g_noalloc_ready[kNoAllocMaxDevices][4];  // decode kernel prepared on the device, per (head dim, 8-bit mode)
 alignas(16) int g_noalloc_host_words[kNoAllocMaxWords];  // work list and records staging, guarded by g_noalloc_mu
 
 }  // namespace
@@ -1656,9 +1798,10 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
     if ((e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch)) != cudaSuccess) return e;
     g_noalloc_dev_ptr[dev] = ptr;
   }
-  if (!g_noalloc_ready[dev][s.d == 64 ? 0 : 1]) {
-    if ((e = prepare_kernel(s.d)) != cudaSuccess) return e;
-    g_noalloc_ready[dev][s.d == 64 ? 0 : 1] = true;
+  const int kind = (s.d == 64 ? 0 : 1) + (in.q8 ? 2 : 0);
+  if (!g_noalloc_ready[dev][kind]) {
+    if ((e = prepare_kernel(s.d, in.q8)) != cudaSuccess) return e;
+    g_noalloc_ready[dev][kind] = true;
   }
   unsigned char* scratch = static_cast<unsigned char*>(g_noalloc_dev_ptr[dev]);
   int sms = 148;
@@ -1678,7 +1821,8 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
     off_items = off_rec + rec_words;
     const int64_t room = ((int64_t)kNoAllocMaxWords - off_items) / kItemWords;
     const int64_t nitems = room > 0 ? build_items(s, in.host_ranks, g_noalloc_host_words, grid, off_segs, -1, recs,
-                                                  reinterpret_cast<Item*>(g_noalloc_host_words + off_items), room)
+                                                  reinterpret_cast<Item*>(g_noalloc_host_words + off_items), room,
+                                                  in.q8)
                                     : -1;
     nwords = nitems < 0 ? -1 : (int)(off_items + nitems * kItemWords);
   }
@@ -1699,7 +1843,8 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
   const int D = s.d, G = s.Hq / s.H;
   PlanMaps pm;
   const uint64_t rows = (uint64_t)in.total_rows;
-  if (!make_row_maps(&pm.tok, in.tok, kChunk, rows * cpb)) return cudaErrorInvalidValue;
+  if (!(in.q8 ? make_code_maps(&pm.tok, in.tok, rows * cpb) : make_row_maps(&pm.tok, in.tok, kChunk, rows * cpb)))
+    return cudaErrorInvalidValue;
   if (!make_row_maps(&pm.dim, in.dim, D, rows)) return cudaErrorInvalidValue;
   if (!make_pacc_map(&pm.pacc, part_acc, nsegs, D)) return cudaErrorInvalidValue;
   std::memcpy(g_noalloc_host_words + off_maps, &pm, sizeof(PlanMaps));
@@ -1727,11 +1872,7 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
   p.ipt = ipt;
   p.S = s.S;
   p.c = s.scale * 1.4426950408889634f;
-  if (D == 64)
-    decode_tc_kernel<64><<<grid, kThreads, kSmemBytes, st>>>(maps, p);
-  else
-    decode_tc_kernel<128><<<grid, kThreads, kSmemBytes, st>>>(maps, p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_decode_kernel(D, in.q8, grid, maps, p, st)) != cudaSuccess) return e;
   return launch_combine(s, part_acc, part_ml, d_work + off_pre, d_work + off_suf, ipt, nrt, out, st);
 }
 

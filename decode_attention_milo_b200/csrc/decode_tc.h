@@ -21,9 +21,10 @@ struct TcInputs {
   uint32_t* status;
   int64_t total_rows;  // rows of the factor arrays (Σ of every block's rank)
   const int32_t* host_ranks;  // [2H][nb]
+  bool q8 = false;            // tok holds int8 codes (8-bit factor object), dim bf16
 };
 
-// The shape check alone (no CUDA call): bf16, d in {64, 128}, n % 128 == 0, GQA group <= 128.
+// The shape check alone (no CUDA call): bf16 (or 8-bit) factors, d in {64, 128}, n % 128 == 0, GQA group <= 128.
 bool tc_shape_ok(const DecodeShape& s);
 bool tc_supported(const DecodeShape& s);
 int tc_launches(const DecodeShape& s);

@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "decode_tc.h"
 #include "internal.h"
+#include "quant.h"
 
 struct milo_factors {
   int device = 0;
@@ -47,6 +48,11 @@ struct milo_factors {
 namespace {
 
 size_t esize(int dtype) { return dtype == MILO_BF16 ? 2 : 4; }
+// element sizes of the two factor arrays (an 8-bit object has int8 tok and bf16 dim)
+size_t tok_esize(int dtype) { return dtype == MILO_I8 ? 1 : esize(dtype); }
+size_t dim_esize(int dtype) { return dtype == MILO_I8 ? 2 : esize(dtype); }
+// the decode reads q, the suffix and out in bf16 for bf16 and 8-bit objects
+bool bf16_io(int dtype) { return dtype == MILO_BF16 || dtype == MILO_I8; }
 
 milo_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return MILO_OK;
@@ -81,7 +87,7 @@ void free_all(milo_factors* f) {
 // shared memory (224 KB at this limit, within the 227 KB a CTA may use).
 constexpr int kMaxAllocBlocks = 8192;
 
-bool valid_dtype(int32_t dt) { return dt == MILO_F32 || dt == MILO_BF16; }
+bool valid_dtype(int32_t dt) { return dt == MILO_F32 || dt == MILO_BF16 || dt == MILO_I8; }
 
 milo_status check_layer_shape(int32_t dtype, int32_t H, int64_t T, int32_t d, int32_t n, int32_t r_min) {
   if (!valid_dtype(dtype) || H <= 0 || T <= 0 || n <= 0 || r_min < 1) return MILO_ERR_INVALID_ARGUMENT;
@@ -119,6 +125,7 @@ static milo_status compress_impl(const void* K, const void* V, int32_t dtype, in
   if (!out) return MILO_ERR_INVALID_ARGUMENT;
   *out = nullptr;
   if (!K || !V) return MILO_ERR_INVALID_ARGUMENT;
+  if (dtype == MILO_I8) return MILO_ERR_INVALID_ARGUMENT;  // the cache itself is f32 or bf16
   milo_status st = check_layer_shape(dtype, num_kv_heads, context, head_dim, block_size, r_min);
   if (st != MILO_OK) return st;
   if (!(budget > 0.0) || !isfinite(budget) || max_sweeps < 0 || (flags & ~MILO_KEEP_INTERMEDIATES))
@@ -303,7 +310,7 @@ milo_status milo_factors_import(int32_t dtype, int32_t num_kv_heads, int64_t con
     return cuda_status(err);
   };
   if (e != cudaSuccess) return fail(e);
-  const size_t tb = rows * block_size * esize(dtype), db = rows * head_dim * esize(dtype);
+  const size_t tb = rows * block_size * tok_esize(dtype), db = rows * head_dim * dim_esize(dtype);
   if ((e = cudaMalloc((void**)&f->ranks, (size_t)P * nb * sizeof(int32_t))) != cudaSuccess) return fail(e);
   if ((e = cudaMalloc((void**)&f->row_offsets, offs.size() * sizeof(int64_t))) != cudaSuccess) return fail(e);
   if ((e = cudaMalloc(&f->tok, tb + 256)) != cudaSuccess) return fail(e);
@@ -325,6 +332,89 @@ milo_status milo_factors_import(int32_t dtype, int32_t num_kv_heads, int64_t con
   if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return fail(e);
   f->host_ranks.assign(host_ranks, host_ranks + (size_t)P * nb);
   f->host_ranks_valid = true;
+  *out = f;
+  return MILO_OK;
+}
+
+milo_status milo_factors_quantize(const milo_factors* fc, void* stream, milo_factors** out) {
+  if (!out) return MILO_ERR_INVALID_ARGUMENT;
+  *out = nullptr;
+  if (!fc) return MILO_ERR_INVALID_ARGUMENT;
+  if (fc->dtype != MILO_BF16) return MILO_ERR_UNSUPPORTED;
+  milo_factors* src = const_cast<milo_factors*>(fc);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int P = 2 * src->H, nb = src->nb;
+  {
+    std::lock_guard<std::mutex> lock(src->mu);
+    if (!src->host_ranks_valid) {
+      MILO_CUDA(cudaEventSynchronize(src->ready));
+      MILO_CUDA(cudaMemcpy(src->host_ranks.data(), src->ranks, src->host_ranks.size() * sizeof(int32_t),
+                           cudaMemcpyDeviceToHost));
+      src->host_ranks_valid = true;
+    }
+  }
+  // ranks of the 8-bit object: one more component per block below full rank (the asymmetric form)
+  std::vector<int32_t> qr(src->host_ranks.size());
+  std::vector<int64_t> qoff((size_t)P * (nb + 1));
+  int64_t total = 0;
+  for (int p = 0; p < P; ++p) {
+    for (int b = 0; b < nb; ++b) {
+      const int32_t r = src->host_ranks[(size_t)p * nb + b];
+      qr[(size_t)p * nb + b] = r < src->d ? r + 1 : r;
+      qoff[(size_t)p * (nb + 1) + b] = total;
+      total += qr[(size_t)p * nb + b];
+    }
+    qoff[(size_t)p * (nb + 1) + nb] = total;
+  }
+  milo_factors* f = new (std::nothrow) milo_factors();
+  if (!f) return MILO_ERR_OUT_OF_MEMORY;
+  f->H = src->H;
+  f->T = src->T;
+  f->d = src->d;
+  f->n = src->n;
+  f->nb = nb;
+  f->r_min = src->r_min;
+  f->total_rows = total;
+  // pools keep a common row count only if they stay equal after the extra components
+  int64_t pool0 = qoff[nb];
+  bool same = true;
+  for (int p = 1; p < P; ++p) same = same && qoff[(size_t)p * (nb + 1) + nb] - qoff[(size_t)p * (nb + 1)] == pool0;
+  f->pool_rows = same ? (int)pool0 : 0;
+  f->R = f->pool_rows;
+  f->rule = src->rule;
+  f->scope = src->scope;
+  f->dtype = MILO_I8;
+  f->host_ranks = qr;
+  f->host_ranks_valid = true;
+  auto fail = [&](cudaError_t err) {
+    free_all(f);
+    delete f;
+    return cuda_status(err);
+  };
+  cudaError_t e = cudaGetDevice(&f->device);
+  if (e != cudaSuccess) return fail(e);
+  const size_t rows = (size_t)f->total_rows;
+  const size_t tb = rows * f->n, db = rows * f->d * 2;
+  if ((e = cudaMalloc((void**)&f->ranks, (size_t)P * nb * sizeof(int32_t))) != cudaSuccess) return fail(e);
+  if ((e = cudaMalloc((void**)&f->row_offsets, (size_t)P * (nb + 1) * sizeof(int64_t))) != cudaSuccess) return fail(e);
+  if ((e = cudaMalloc(&f->tok, tb + 256)) != cudaSuccess) return fail(e);
+  if ((e = cudaMalloc(&f->dim, db + 256)) != cudaSuccess) return fail(e);
+  if ((e = cudaMalloc((void**)&f->status, sizeof(uint32_t))) != cudaSuccess) return fail(e);
+  if ((e = cudaMemsetAsync(f->status, 0, sizeof(uint32_t), s)) != cudaSuccess) return fail(e);
+  if ((e = cudaMemsetAsync(f->tok, 0, tb + 256, s)) != cudaSuccess) return fail(e);
+  if ((e = cudaMemsetAsync(f->dim, 0, db + 256, s)) != cudaSuccess) return fail(e);
+  if ((e = cudaMemcpy(f->ranks, qr.data(), qr.size() * sizeof(int32_t), cudaMemcpyHostToDevice)) != cudaSuccess)
+    return fail(e);
+  if ((e = cudaMemcpy(f->row_offsets, qoff.data(), qoff.size() * sizeof(int64_t), cudaMemcpyHostToDevice)) !=
+      cudaSuccess)
+    return fail(e);
+  if ((e = cudaStreamWaitEvent(s, src->ready, 0)) != cudaSuccess) return fail(e);
+  milo::QuantShape qs{P, nb, f->n, f->d};
+  milo::QuantBuffers qb{src->tok, src->dim, src->ranks, src->row_offsets, f->tok, f->dim, f->ranks, f->row_offsets,
+                        f->status};
+  if ((e = milo::launch_quantize(qs, qb, s)) != cudaSuccess) return fail(e);
+  if ((e = cudaEventCreateWithFlags(&f->ready, cudaEventDisableTiming)) != cudaSuccess) return fail(e);
+  if ((e = cudaEventRecord(f->ready, s)) != cudaSuccess) return fail(e);
   *out = f;
   return MILO_OK;
 }
@@ -400,8 +490,9 @@ milo_status milo_decode_worklist(const int32_t* host_ranks, int32_t num_kv_heads
 int32_t milo_decode_launches(const milo_factors* f, int32_t batch, int32_t num_q_heads, int32_t suffix_len) {
   if (!f || batch <= 0 || num_q_heads <= 0 || suffix_len < 0 || num_q_heads % f->H != 0)
     return -(int32_t)MILO_ERR_INVALID_ARGUMENT;
-  milo::DecodeShape ds{f->H, f->nb, f->n, f->d, batch, num_q_heads, suffix_len, f->dtype == MILO_BF16, 1.f};
-  if (f->dtype == MILO_BF16 && milo::tc_supported(ds)) return milo::tc_launches(ds);
+  milo::DecodeShape ds{f->H, f->nb, f->n, f->d, batch, num_q_heads, suffix_len, bf16_io(f->dtype), 1.f};
+  if (bf16_io(f->dtype) && milo::tc_supported(ds)) return milo::tc_launches(ds);
+  if (f->dtype == MILO_I8) return -(int32_t)MILO_ERR_UNSUPPORTED;
   return suffix_len > 0 ? 3 : 2;
 }
 
@@ -430,20 +521,22 @@ static milo_status decode_impl(const void* q, int32_t batch, int32_t num_q_heads
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   MILO_CUDA(cudaStreamIsCapturing(s, &cap));
   if (cap == cudaStreamCaptureStatusNone) MILO_CUDA(cudaStreamWaitEvent(s, f->ready, 0));
-  milo::DecodeShape ds{f->H, f->nb, f->n, f->d, batch, num_q_heads, suffix_len, f->dtype == MILO_BF16, sc};
+  milo::DecodeShape ds{f->H, f->nb, f->n, f->d, batch, num_q_heads, suffix_len, bf16_io(f->dtype), sc};
   milo::DecodeBuffers db{q, K_suffix, V_suffix, f->ranks, f->row_offsets, f->tok, f->dim, nullptr, out, f->status};
-  if (f->dtype == MILO_BF16 && milo::tc_supported(ds)) {
+  if (bf16_io(f->dtype) && milo::tc_supported(ds)) {
     if (!f->host_ranks_valid) {
       MILO_CUDA(cudaStreamSynchronize(s));
       MILO_CUDA(cudaMemcpy(f->host_ranks.data(), f->ranks, f->host_ranks.size() * sizeof(int32_t),
                            cudaMemcpyDeviceToHost));
       f->host_ranks_valid = true;
     }
-    milo::TcInputs in{q,        K_suffix, V_suffix,     f->tok,       f->dim,
-                      f->ranks, f->row_offsets, f->status, f->total_rows, f->host_ranks.data()};
+    milo::TcInputs in{q,        K_suffix,       V_suffix,  f->tok,        f->dim,
+                      f->ranks, f->row_offsets, f->status, f->total_rows, f->host_ranks.data(),
+                      f->dtype == MILO_I8};
     return cuda_status(milo::tc_decode(&f->tc_plan, ds, in, out, s, ev0, ev1, mask));
   }
-  if (mask) return MILO_ERR_UNSUPPORTED;  // block selection runs on the bf16 tensor-core decode
+  // block selection and 8-bit factors run on the tensor-core decode only
+  if (mask || f->dtype == MILO_I8) return MILO_ERR_UNSUPPORTED;
   const size_t need = milo::simt_decode_partials_floats(ds);
   if (need > f->partials_floats) {
     MILO_CUDA(cudaStreamSynchronize(s));
@@ -474,8 +567,8 @@ milo_status milo_decode_attn_noalloc(const void* q, int32_t batch, int32_t num_q
   if (!(scale == scale) || isinf(scale)) return MILO_ERR_INVALID_ARGUMENT;
   if (batch > 65535 || num_q_heads > 4096 || suffix_len > (1 << 20)) return MILO_ERR_INVALID_ARGUMENT;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)f->d);
-  milo::DecodeShape ds{f->H, f->nb, f->n, f->d, batch, num_q_heads, suffix_len, f->dtype == MILO_BF16, sc};
-  if (f->dtype != MILO_BF16 || !milo::tc_supported(ds)) return MILO_ERR_UNSUPPORTED;
+  milo::DecodeShape ds{f->H, f->nb, f->n, f->d, batch, num_q_heads, suffix_len, bf16_io(f->dtype), sc};
+  if (!bf16_io(f->dtype) || !milo::tc_supported(ds)) return MILO_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   std::lock_guard<std::mutex> lock(f->mu);
   if (!f->host_ranks_valid) {
@@ -488,8 +581,9 @@ milo_status milo_decode_attn_noalloc(const void* q, int32_t batch, int32_t num_q
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   MILO_CUDA(cudaStreamIsCapturing(s, &cap));
   if (cap == cudaStreamCaptureStatusNone) MILO_CUDA(cudaStreamWaitEvent(s, f->ready, 0));
-  milo::TcInputs in{q,        K_suffix, V_suffix,     f->tok,       f->dim,
-                    f->ranks, f->row_offsets, f->status, f->total_rows, f->host_ranks.data()};
+  milo::TcInputs in{q,        K_suffix,       V_suffix,  f->tok,        f->dim,
+                    f->ranks, f->row_offsets, f->status, f->total_rows, f->host_ranks.data(),
+                    f->dtype == MILO_I8};
   bool too_large = false;
   const cudaError_t e = milo::tc_decode_noalloc(ds, in, out, s, &too_large);
   if (too_large) return MILO_ERR_UNSUPPORTED;

@@ -39,7 +39,9 @@
  *   so that X_b ≈ U_b · B_bᵀ.  The blocks of a pool are consecutive and the
  *   pools follow each other (pool p starts at row p * pool_rows when every pool
  *   has the same rank sum).  Factor elements have the dtype of the compressed
- *   cache.
+ *   cache, except in 8-bit objects (MILO_I8, made by milo_factors_quantize):
+ *   there tok holds int8 codes and dim holds bf16, and every block carries one
+ *   more component than it was compressed with (see milo_factors_quantize).
  */
 #ifndef MILO_H_
 #define MILO_H_
@@ -50,7 +52,7 @@
 extern "C" {
 #endif
 
-#define MILO_ABI_VERSION 2
+#define MILO_ABI_VERSION 3
 
 typedef enum {
   MILO_OK = 0,
@@ -63,7 +65,8 @@ typedef enum {
   MILO_ERR_OUT_OF_MEMORY = 7
 } milo_status;
 
-typedef enum { MILO_F32 = 0, MILO_BF16 = 1 } milo_dtype;
+/* MILO_I8 describes factor objects only: int8 token factors, bf16 dimension factors. */
+typedef enum { MILO_F32 = 0, MILO_BF16 = 1, MILO_I8 = 2 } milo_dtype;
 
 /* milo_compress flags */
 #define MILO_KEEP_INTERMEDIATES 1u /* keep fp32 eigenpairs, fp64 entropies and quotas */
@@ -311,13 +314,42 @@ milo_status milo_factors_status(const milo_factors* f, uint32_t* host_bits);
  * factors computed elsewhere or saved earlier.  host_ranks [2H][nb], each in
  * [1, d]; host_tok [rows][n] and host_dim [rows][d] in `dtype`, rows = Σ of all
  * ranks, pools in order (their sums may differ, as with a layer-wide budget);
- * host_tok holds each block's 128-token slabs as described above.
+ * host_tok holds each block's 128-token slabs as described above.  With
+ * dtype MILO_I8, host_tok is int8 codes and host_dim bf16 (the form
+ * milo_factors_quantize writes, each rank counting the extra component).
  * Synchronises `stream`.
  */
 milo_status milo_factors_import(int32_t dtype, int32_t num_kv_heads, int64_t context,
                                 int32_t head_dim, int32_t block_size, int32_t r_min,
                                 const int32_t* host_ranks, const void* host_tok,
                                 const void* host_dim, void* stream, milo_factors** out);
+
+/*
+ * milo_factors_quantize — 8-bit storage of a bf16 factor object's token factors.
+ * Source: §5.3 (the compressed caches compose with asymmetric INT8 and KIVI
+ * quantisation for further memory savings).  The page names no scheme; this is
+ * asymmetric INT8 per rank channel of each block (KIVI's per-channel rule for
+ * keys, applied to the token factors U_b and P_b alike):
+ *   channel j of block b, values x_t over the block's n tokens:
+ *     lo = min x_t, a = (max x_t − lo)/255, code c_t = round((x_t − lo)/a) − 128
+ *     in [−128, 127], rounded half to even, all in fp32; a = 0 gives c_t = −128;
+ *   the scales and minima are folded into the bf16 dimension factor with one
+ *   extra component per block whose codes are all 1:
+ *     dim row j = a_j·B_b[:, j] (j < r),  dim row r = Σ_j (lo_j + 128·a_j)·B_b[:, j],
+ *   so that codes·dimᵀ is the dequantized block exactly.
+ *   A block stored at full rank d, where one more component would exceed the
+ *   head dimension, takes the symmetric form: a = max |x_t| / 127,
+ *   c_t = round(x_t / a) in [−127, 127] (a = 0 gives 0), dim row j = a_j·B_b[:, j].
+ * The new object has dtype MILO_I8, ranks r_b + 1 (r_b at full rank), row_offsets
+ * the running sums of those ranks, tok of int8 codes in the slab layout above
+ * (an extra row all 1 where there is one) and dim in bf16; milo_decode_attn,
+ * _select and _noalloc take it as they take a bf16 object (q, suffix and out stay
+ * bf16).  Token-factor bytes halve.
+ *   f    bf16 factor object (MILO_ERR_UNSUPPORTED for other dtypes); not modified.
+ *   out  receives the new object; destroy it with milo_factors_destroy.
+ * Synchronises once on f's factors to read their ranks; allocates the new object.
+ */
+milo_status milo_factors_quantize(const milo_factors* f, void* stream, milo_factors** out);
 
 /* Frees f and everything it owns (synchronises the device first). NULL is a no-op. */
 void milo_factors_destroy(milo_factors* f);

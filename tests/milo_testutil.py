@@ -110,7 +110,12 @@ def factor_arrays(f) -> dict:
     out = dict(desc=d)
     out["ranks"] = device_view(d["ranks"], (H2, nb), "<i4").cpu().numpy()
     out["row_offsets"] = device_view(d["row_offsets"], (H2, nb + 1), "<i8").cpu().numpy()
-    if bf:
+    if d["dtype"] == 2:  # 8-bit object: int8 codes, bf16 dimension factors
+        out["codes"] = device_view(d["tok"], (total * n,), "|i1").cpu().numpy()
+        out["tok"] = out["codes"].astype(np.float64)
+        dim = device_view(d["dim"], (total, dd), "<i2").cpu().numpy().view(np.uint16)
+        out["dim"] = from_storage(dim, "bf16")
+    elif bf:
         tok = device_view(d["tok"], (total * n,), "<i2").cpu().numpy().view(np.uint16)
         dim = device_view(d["dim"], (total, dd), "<i2").cpu().numpy().view(np.uint16)
         out["tok"], out["dim"] = from_storage(tok, "bf16"), from_storage(dim, "bf16")
@@ -124,4 +129,41 @@ def factor_arrays(f) -> dict:
     if d["eigvecs"]:
         out["eigvecs"] = device_view(d["eigvecs"], (H2, nb, dd, dd), "<f4").cpu().numpy().astype(np.float64)
     torch.cuda.synchronize()
+    return out
+
+
+def layer_from_arrays(got: dict) -> dict:
+    """Oracle layer (pools of U, B per block) from a factor object's host arrays (factor_arrays)."""
+    d = got["desc"]
+    H, nb, n = d["num_kv_heads"], d["num_blocks"], d["block_size"]
+    pools = []
+    for p in range(2 * H):
+        U, B = [], []
+        for b in range(nb):
+            r0, r1 = int(got["row_offsets"][p, b]), int(got["row_offsets"][p, b + 1])
+            U.append(untok_slabs(got["tok"][r0 * n:r1 * n], n, r1 - r0))
+            B.append(got["dim"][r0:r1].T)
+        pools.append(dict(U=U, B=B, ranks=got["ranks"][p]))
+    return dict(K=pools[0::2], V=pools[1::2])
+
+
+def pack_factors_8bit(qlayer: dict):
+    """Oracle 8-bit layer (oracle.quantize_layer) → (ranks, int8 codes in slab order, bf16 dim) for import."""
+    H = len(qlayer["K"])
+    pools = []
+    for h in range(H):
+        pools += [qlayer["K"][h], qlayer["V"][h]]
+    ranks = np.array([p["ranks"] for p in pools], dtype=np.int32)
+    tok = np.concatenate([tok_slabs(u) for p in pools for u in p["U"]], axis=0)
+    assert np.array_equal(tok, np.rint(tok)) and tok.min() >= -128 and tok.max() <= 127
+    dim = np.concatenate([b.T for p in pools for b in p["B"]], axis=0)
+    return ranks, tok.astype(np.int8), to_storage(dim, "bf16")
+
+
+def stored_layer_8bit(qlayer: dict) -> dict:
+    """The 8-bit layer as stored: codes exact, the folded dimension factors rounded to bf16."""
+    c = cast_fn("bf16")
+    out = dict(qlayer)
+    for t in ("K", "V"):
+        out[t] = [dict(p, B=[c(b) for b in p["B"]]) for p in qlayer[t]]
     return out

@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol():
     assert {"milo_compress", "milo_decode_attn"} <= names
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.milo_abi_version() == 2
+    assert lib.milo_abi_version() == 3
     assert lib.milo_status_string(0) == b"ok"
     assert lib.milo_status_string(3).startswith(b"budget")
 
@@ -50,6 +50,7 @@ def _compress(lib, **kw):
     (dict(budget=0.0), 1), (dict(budget=float("nan")), 1), (dict(sweeps=-1), 1), (dict(flags=8), 1),
     (dict(budget=0.001), 3),
     (dict(T=8193 * 512, H=1), 2),  # more blocks per pool than the allocation step holds in shared memory
+    (dict(dtype=2), 1),            # 8-bit describes factor objects only, never the cache
 ])
 def test_compress_rejects_bad_arguments(kw, code):
     assert _compress(milo.load_library(), **kw) == code
@@ -170,3 +171,19 @@ def test_python_decode_checks_shapes_before_the_library():
         for fn in (milo.decode_attn, milo.decode_attn_noalloc):
             with pytest.raises(ValueError):
                 fn(args["q"], f, args["K_suf"], args["V_suf"], out=args["out"])
+
+
+def test_quantize_rejects_bad_arguments():
+    lib = milo.load_library()
+    out = ctypes.c_void_p(123)
+    assert lib.milo_factors_quantize(None, None, ctypes.byref(out)) == 1
+    assert out.value is None
+    assert lib.milo_factors_quantize(None, None, None) == 1
+
+
+def test_import_checks_array_sizes_for_8bit():
+    import numpy as np
+    ranks = np.full((2, 2), 5, dtype=np.int32)  # one KV head, two blocks of 512: 20 rows
+    with pytest.raises(ValueError):  # bf16-sized codes for an 8-bit object
+        milo.import_factors(milo.I8, 1, 1024, 64, 512, 4, ranks, np.zeros((20, 512), np.uint16),
+                            np.zeros((20, 64), np.uint16))
