@@ -36,7 +36,7 @@ METRIC = "compressed-KV decode tokens/s at Qwen2.5-7B shape; achieved HBM GB/s v
 # DRAM bytes (read + written) of one launch of the main decode kernel, measured with ncu, per workload, keyed by
 # the SHA-256 prefix of the kernel's source file at the time of the capture.  A different digest means the
 # kernel has changed since the counters were taken, and the line reports traffic as null.
-DECODE_TRAFFIC = {}
+DECODE_TRAFFIC = {("qwen2.5-7b-layer", "082a5a68d461"): 42515968 + 22528}
 
 
 def _source_digest() -> str:
@@ -55,7 +55,7 @@ def _args():
     p.add_argument("--workload", default="qwen2.5-7b-layer")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="bound of the CPU oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--profile", choices=["decode", "compress"], default=None,
+    p.add_argument("--profile", choices=["decode", "decode8", "compress"], default=None,
                    help="run only N calls of one phase on the workload (for profiler captures), no JSON contract")
     p.add_argument("--calls", type=int, default=6)
     return p.parse_args()
@@ -235,6 +235,53 @@ def _algorithmic_bytes(ranks, wl, esize):
     suffix = 2 * wl.batch * wl.kv_heads * wl.suffix * wl.head_dim * esize
     qo = 2 * wl.batch * wl.q_heads * wl.head_dim * esize
     return factors + suffix + qo
+
+
+def _algorithmic_bytes_8bit(qranks, wl):
+    """The same for 8-bit factor objects: one byte per token-factor element, bf16 dimension factors, at the
+    8-bit object's ranks (one more component per block below full rank)."""
+    factors = int(qranks.sum()) * (wl.block_size * 1 + wl.head_dim * 2)
+    suffix = 2 * wl.batch * wl.kv_heads * wl.suffix * wl.head_dim * 2
+    qo = 2 * wl.batch * wl.q_heads * wl.head_dim * 2
+    return factors + suffix + qo
+
+
+def _decode_8bit(torch, milo, wl, sets, qs, ks, vs, outs, steps, peak):
+    """8-bit factor storage (milo_factors_quantize): quantise time per layer and the decode kernel over the
+    8-bit copies, timed like the main kernel (library events around it, eager launches over the copies)."""
+    qsets, qms = [], []
+    for f in sets:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        qsets.append(milo.quantize(f))
+        e1.record()
+        torch.cuda.synchronize()
+        qms.append(e0.elapsed_time(e1))
+    copies = len(qsets)
+    for c in range(copies):
+        milo.decode_attn(qs[c], qsets[c], ks[c], vs[c], out=outs[c])
+    torch.cuda.synchronize()
+    n = min(steps, 300)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for a_, b_ in evs:
+        a_.record()
+        b_.record()
+    for s_ in range(n):
+        c = s_ % copies
+        milo.decode_attn_profiled(qs[c], qsets[c], ks[c], vs[c], outs[c], evs[s_][0], evs[s_][1])
+    torch.cuda.synchronize()
+    kms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    qranks = qsets[0].ranks()
+    nbytes = _algorithmic_bytes_8bit(qranks, wl)
+    ok = all(f.status()[0] == 0 for f in qsets)
+    for f in qsets:
+        f.close()
+    achieved = nbytes / (kms / 1e3) / 1e9
+    return {"kernel": "decode_tc_kernel (8-bit mode)", "kernel_ms": kms, "bytes_per_step": nbytes,
+            "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "decode_tokens_per_s": wl.batch / (kms / 1e3), "quantize_ms": statistics.median(qms), "status_ok": ok,
+            "note": "token factors as int8 codes (asymmetric per rank channel, symmetric at full rank), dimension "
+                    "factors bf16; same timing as the main kernel"}
 
 
 def _oracle_layer(wl, L):
@@ -540,6 +587,8 @@ def run_milo(a):
         milo.decode_attn_profiled(qs[c], sets[c], ks[c], vs[c], outs[c], evs[s_][0], evs[s_][1])
     torch.cuda.synchronize()
     kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    peak, peak_kind = _peaks()
+    dec8 = _decode_8bit(torch, milo, wl, sets, qs, ks, vs, outs, steps, peak) if dt == "bf16" else None
 
     # --- end to end through the public API: pinned host inputs, copies inside the timed region.  Steps
     # alternate between two streams with their own device buffers, so the host-to-device copies of one
@@ -578,7 +627,6 @@ def run_milo(a):
     h2d = hq.numel() * hq.element_size() + (2 * hk.numel() * hk.element_size() if S else 0)
     d2h = hout.numel() * hout.element_size()
 
-    peak, peak_kind = _peaks()
     achieved = step_bytes / (kernel_ms / 1e3) / 1e9
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -604,6 +652,7 @@ def run_milo(a):
             "compress": {"compressions_per_s": 1e3 / statistics.median(comp), "ms": statistics.median(comp),
                          "unit": "whole-layer compressions/s",
                          "roofline": _compress_roofline(torch, wl, esize, comp_ranks, sweeps, kern, peak)},
+            "decode_8bit": dec8,
             "gpu_launches": kernels_per_call * steps,
             "gpu_launches_note": f"{kernels_per_call} kernels per decode call x {steps} steps of one timed window "
                                  f"({windows} windows timed, the median reported)",
@@ -639,6 +688,10 @@ def run_profile(a):
             f.close()
     else:
         f = milo.compress(Kd, Vd, wl.block_size, beta, wl.r_min)
+        if a.profile == "decode8":
+            f8 = milo.quantize(f)
+            f.close()
+            f = f8
         q = dev(L["q"])
         ks = dev(L["K_suf"]) if wl.suffix else None
         vs = dev(L["V_suf"]) if wl.suffix else None
