@@ -10,7 +10,8 @@ Low-rank Compression", a section summary of the paper):
   §4.2  block-wise low-rank compression of keys and values, block by block;
   §4.3  entropy-driven rank allocation under a fixed total budget;
   §4.4  workflow: encode (partition, entropy, low-rank store), then decode;
-  §5.3  composition with asymmetric INT8 quantisation (oracle/quant.py).
+  §5.3  composition with asymmetric INT8 quantisation (oracle/quant.py);
+  §3, §4.5  pre-RoPE key factors, reconstructed and rotated at decode (oracle/rope.py).
 
 Every function states the passage it follows and the reading taken where the
 page is silent.
@@ -38,4 +39,5 @@ from .milo import (  # noqa: F401
 from .hestenes import hestenes_svd  # noqa: F401
 from .quant import (dequantize_channel, quantize_block, quantize_channel, quantize_channel_symmetric,  # noqa: F401
                     quantize_layer, quantize_pool)
+from .rope import apply_rope, decode_attention_rope, inv_freq, rotated_prefix_keys  # noqa: F401
 from .tiefree import cut_gap, greedy_cut_gap, tiefree_taus  # noqa: F401
