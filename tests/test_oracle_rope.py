@@ -48,8 +48,8 @@ def test_scores_depend_on_relative_position_only():
     rng = np.random.default_rng(2)
     a, b = rng.standard_normal((1, 32)), rng.standard_normal((1, 32))
     for m, n in [(5, 3), (1000, 17), (70000, 69999)]:
-        lhs = float(oracle.apply_rope(a, [m], 1e6) @ oracle.apply_rope(b, [n], 1e6).T)
-        rhs = float(oracle.apply_rope(a, [m - n], 1e6) @ b.T)
+        lhs = float((oracle.apply_rope(a, [m], 1e6) @ oracle.apply_rope(b, [n], 1e6).T)[0, 0])
+        rhs = float((oracle.apply_rope(a, [m - n], 1e6) @ b.T)[0, 0])
         assert math.isclose(lhs, rhs, rel_tol=1e-9, abs_tol=1e-9)
 
 
