@@ -75,6 +75,8 @@ def load_library(path: str | None = None):
     L.milo_decode_attn_profiled.argtypes = [vp, i32, i32, vp, vp, vp, i32, f32, vp, vp, vp, vp]
     L.milo_decode_attn_select.restype = i32
     L.milo_decode_attn_select.argtypes = [vp, i32, i32, vp, vp, vp, i32, f32, vp, vp, vp]
+    L.milo_decode_attn_rope.restype = i32
+    L.milo_decode_attn_rope.argtypes = [vp, i32, i32, vp, vp, vp, i32, f32, f64, vp, vp, vp]
     L.milo_decode_attn_noalloc.restype = i32
     L.milo_decode_attn_noalloc.argtypes = [vp, i32, i32, vp, vp, vp, i32, f32, vp, vp]
     L.milo_decode_launches.restype = i32
@@ -93,7 +95,7 @@ def load_library(path: str | None = None):
     L.milo_factors_quantize.argtypes = [vp, vp, ctypes.POINTER(vp)]
     L.milo_factors_destroy.restype = None
     L.milo_factors_destroy.argtypes = [vp]
-    if L.milo_abi_version() != 3:
+    if L.milo_abi_version() != 4:
         raise RuntimeError("libmilo.so ABI version mismatch")
     _lib = L
     return L
@@ -293,6 +295,26 @@ def decode_attn_select(q, factors: Factors, block_mask, K_suf=None, V_suf=None, 
         _dev_ptr(q, "q"), B, Hq, factors.handle, _dev_ptr(K_suf, "K_suf") if S else None,
         _dev_ptr(V_suf, "V_suf") if S else None, S, float(scale), m.ctypes.data_as(ctypes.c_void_p),
         _dev_ptr(out, "out"), _stream_ptr(stream)), "milo_decode_attn_select")
+    return out
+
+
+def decode_attn_rope(q, factors: Factors, K_suf=None, V_suf=None, theta: float = 1e6, block_mask=None,
+                     scale: float = 0.0, out=None, stream=None):
+    """decode_attn over factors of pre-RoPE keys: every key block is rebuilt and rotated at its absolute
+    positions (base theta) before the scores; q and the suffix are post-RoPE.  See milo_decode_attn_rope."""
+    B, Hq, S, out = _decode_args(q, factors, K_suf, V_suf, out)
+    m = None
+    if block_mask is not None:
+        H = factors.shape()[0]
+        nb = factors.describe()["num_blocks"]
+        m = np.ascontiguousarray(np.asarray(block_mask) != 0, dtype=np.uint8)
+        if m.shape != (H, nb):
+            raise ValueError(f"block_mask must be [{H}][{nb}], got {m.shape}")
+    _check(load_library().milo_decode_attn_rope(
+        _dev_ptr(q, "q"), B, Hq, factors.handle, _dev_ptr(K_suf, "K_suf") if S else None,
+        _dev_ptr(V_suf, "V_suf") if S else None, S, float(scale), float(theta),
+        m.ctypes.data_as(ctypes.c_void_p) if m is not None else None, _dev_ptr(out, "out"), _stream_ptr(stream)),
+        "milo_decode_attn_rope")
     return out
 
 

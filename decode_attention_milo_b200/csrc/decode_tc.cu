@@ -34,6 +34,7 @@
 
 #include "common.cuh"
 #include "decode_tc.h"
+#include "rope.h"
 #include "tc_ptx.cuh"
 
 namespace milo {
@@ -164,6 +165,7 @@ struct RowMaps {
 struct Maps {
   CUtensorMap ksuf, vsuf;  // suffix keys and values, boxes of 128 rows
   CUtensorMap qpre, qsuf;  // query rows of a prefix row tile / of one query
+  CUtensorMap krope;       // dense-key mode: the rotated prefix keys [H·T][d], boxes of 128 rows
 };
 // The maps of a plan's factors and partials, in device memory (128-byte aligned), written once per plan.
 struct PlanMaps {
@@ -171,9 +173,9 @@ struct PlanMaps {
   CUtensorMap pacc;  // partial accumulators [segments · 128][d] fp32, boxes of 128 rows × 32 columns
 };
 // An item's map index: [0, 16) counts CUtensorMaps from the start of PlanMaps, [16, 20) from the start of Maps.
-constexpr int kMapTok = 0, kMapDim = 8, kMapKsuf = 16, kMapVsuf = 17, kMapQpre = 18, kMapQsuf = 19;
+constexpr int kMapTok = 0, kMapDim = 8, kMapKsuf = 16, kMapVsuf = 17, kMapQpre = 18, kMapQsuf = 19, kMapKrope = 20;
 static_assert(sizeof(RowMaps) == 8 * sizeof(CUtensorMap), "row maps hold 8 boxes");
-static_assert(sizeof(Maps) == 4 * sizeof(CUtensorMap), "call maps in the order of the item map index");
+static_assert(sizeof(Maps) == 5 * sizeof(CUtensorMap), "call maps in the order of the item map index");
 
 // One CTA's work, built on the host: its segments and the rank / row offset of every block they touch, in
 // the order the roles walk them.  The CTA copies it to shared memory with one coalesced load at start, so
@@ -321,11 +323,15 @@ __device__ __forceinline__ void st_tile8(uint32_t tile, int row, int col, uint32
   ptx::st_shared_v4(addr, a, b, c, d);
 }
 
-template <int D, bool Q8>
-__global__ void __launch_bounds__(threads_of<Q8>(), 1)
+// MODE: kModeRank (bf16 factors, rank-space scores), kMode8bit (int8 token factors), kModeDenseKeys (the scores
+// of the prefix against dense rotated keys, values in rank space).
+constexpr int kModeRank = 0, kMode8bit = 1, kModeDenseKeys = 2;
+template <int D, int MODE>
+__global__ void __launch_bounds__(threads_of<MODE == kMode8bit>(), 1)
     decode_tc_kernel(const __grid_constant__ Maps maps,
                      const Params p) {
   constexpr int NCB = D / 64;
+  constexpr bool Q8 = MODE == kMode8bit, DK = MODE == kModeDenseKeys;
   using L = Smem<Q8>;
   constexpr int kNThreads = threads_of<Q8>();
   extern __shared__ uint8_t smem_raw[];
@@ -626,9 +632,11 @@ __global__ void __launch_bounds__(threads_of<Q8>(), 1)
           bounds_ok = false;
           break;
         }
+        // dense-key mode: no q̃ (the prefix scores are Q·Kᵀ like the suffix's), Q is read by every G2
+        auto g2k = [&]() -> bool { return DK ? g2s() : g2(bi.rk); };
         if (ok) {
-          ok = wait_q() && g1(bi.rk);
-          if (ok && !w.has_next()) commit(B_QEMPTY);  // last read of Q in this segment
+          ok = wait_q() && (DK || g1(bi.rk));
+          if (!DK && ok && !w.has_next()) commit(B_QEMPTY);  // last read of Q in this segment
         }
         while (true) {
           const int n = w.chunks();
@@ -648,12 +656,14 @@ __global__ void __launch_bounds__(threads_of<Q8>(), 1)
             if (next_is_last) commit(B_QEMPTY);
             return true;
           };
-          sync_wg(kSigQt);
-          ++use_c;
+          if (!DK) {
+            sync_wg(kSigQt);
+            ++use_c;
+          }
           if (ok) {
-            ok = g2(bi.rk);
-            if (ok && n >= 2) ok = g2(bi.rk);
-            else if (ok && next) ok = g1_next();
+            ok = g2k();
+            if (ok && n >= 2) ok = g2k();
+            else if (!DK && ok && next) ok = g1_next();
           }
           if (have_prev) {
             sync_wg(kSigAt);
@@ -664,8 +674,8 @@ __global__ void __launch_bounds__(threads_of<Q8>(), 1)
             if (ok) {
               ok = g3(bi.rv, j == 0, s);
               if (ok && j + 1 == n) commit(B_ATFULL);
-              if (ok && j + 2 < n) ok = g2(bi.rk);
-              else if (ok && j + 2 == n && next) ok = g1_next();
+              if (ok && j + 2 < n) ok = g2k();
+              else if (!DK && ok && j + 2 == n && next) ok = g1_next();
             }
           }
           if (!next) break;
@@ -678,6 +688,7 @@ __global__ void __launch_bounds__(threads_of<Q8>(), 1)
         if (!bounds_ok) break;
         sync_wg(kSigAt);
         if (ok) ok = g4(bi.rv, kb == 0);
+        if (DK && ok) commit(B_QEMPTY);  // every G2 of the segment has read Q
       } else {
         const int n = sg.c1 - sg.c0;
         if (ok) {
@@ -1036,7 +1047,7 @@ __global__ void __launch_bounds__(threads_of<Q8>(), 1)
             bounds_ok = fail_bounds();
             break;
           }
-          ok = convert_qt(active, bi.rk) && ok;  // q̃ of this block to smem
+          if (!DK) ok = convert_qt(active, bi.rk) && ok;  // q̃ of this block to smem
         }
         if (have_prev) ok = convert_at(active, prev.rv) && ok;  // the previous block's ã for its G4
         if (done) break;
@@ -1192,30 +1203,34 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, c
 
 // Prepares the decode kernel for head dimension d: its shared-memory size, and a check that the launch
 // allocates the registers that the kernel's register split (setmaxnreg) redistributes.
-template <bool Q8>
+template <int MODE>
 const void* kernel_of(int d) {
-  return d == 64 ? (const void*)decode_tc_kernel<64, Q8> : (const void*)decode_tc_kernel<128, Q8>;
+  return d == 64 ? (const void*)decode_tc_kernel<64, MODE> : (const void*)decode_tc_kernel<128, MODE>;
 }
-cudaError_t prepare_kernel(int d, bool q8) {
-  const void* kfn = q8 ? kernel_of<true>(d) : kernel_of<false>(d);
+cudaError_t prepare_kernel(int d, int mode) {
+  const void* kfn = mode == kMode8bit ? kernel_of<kMode8bit>(d)
+                    : mode == kModeDenseKeys ? kernel_of<kModeDenseKeys>(d) : kernel_of<kModeRank>(d);
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, kfn);
   if (e != cudaSuccess) return e;
   if (kRegSplit && fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
   return cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              q8 ? Smem<true>::kBytes : Smem<false>::kBytes);
+                              mode == kMode8bit ? Smem<true>::kBytes : Smem<false>::kBytes);
 }
-// Launches the decode kernel of head dimension d and mode q8.
-cudaError_t launch_decode_kernel(int d, bool q8, int grid, const Maps& maps, const Params& p, cudaStream_t st) {
-  if (q8) {
-    if (d == 64) decode_tc_kernel<64, true><<<grid, threads_of<true>(), Smem<true>::kBytes, st>>>(maps, p);
-    else decode_tc_kernel<128, true><<<grid, threads_of<true>(), Smem<true>::kBytes, st>>>(maps, p);
-  } else {
-    if (d == 64) decode_tc_kernel<64, false><<<grid, threads_of<false>(), Smem<false>::kBytes, st>>>(maps, p);
-    else decode_tc_kernel<128, false><<<grid, threads_of<false>(), Smem<false>::kBytes, st>>>(maps, p);
-  }
+template <int MODE>
+void launch_mode(int d, int grid, const Maps& maps, const Params& p, cudaStream_t st) {
+  constexpr bool q8 = MODE == kMode8bit;
+  if (d == 64) decode_tc_kernel<64, MODE><<<grid, threads_of<q8>(), Smem<q8>::kBytes, st>>>(maps, p);
+  else decode_tc_kernel<128, MODE><<<grid, threads_of<q8>(), Smem<q8>::kBytes, st>>>(maps, p);
+}
+// Launches the decode kernel of head dimension d in `mode`.
+cudaError_t launch_decode_kernel(int d, int mode, int grid, const Maps& maps, const Params& p, cudaStream_t st) {
+  if (mode == kMode8bit) launch_mode<kMode8bit>(d, grid, maps, p, st);
+  else if (mode == kModeDenseKeys) launch_mode<kModeDenseKeys>(d, grid, maps, p, st);
+  else launch_mode<kModeRank>(d, grid, maps, p, st);
   return cudaGetLastError();
 }
+int mode_of(const TcInputs& in) { return in.q8 ? kMode8bit : in.rope_keys ? kModeDenseKeys : kModeRank; }
 
 // The map of a [rows][width] bf16 array with boxes of h rows: 3D for 128 columns (x: 64 columns, y: rows,
 // z: the two 64-column blocks), 2D for 64 columns.
@@ -1275,6 +1290,7 @@ bool make_call_maps(Maps* M, const DecodeShape& s, const TcInputs& in, int ipt) 
     M->ksuf = M->qpre;  // never read
     M->vsuf = M->qpre;
   }
+  M->krope = M->qpre;  // replaced in the dense-key mode
   return true;
 }
 
@@ -1295,6 +1311,8 @@ struct TcPlan {
   const void* dim = nullptr;
   PlanMaps* d_maps = nullptr;  // the factor and partial maps in device memory
   bool q8 = false;             // 8-bit token factors
+  bool rope = false;           // pre-RoPE key factors: the decode scores the rotated keys below
+  void* krope = nullptr;       // [H][T][d] bf16 rotated reconstructed keys (dense-key mode)
 };
 
 bool tc_shape_ok(const DecodeShape& s) {
@@ -1304,7 +1322,7 @@ bool tc_shape_ok(const DecodeShape& s) {
 
 bool tc_supported(const DecodeShape& s) { return tc_shape_ok(s) && encode_fn() != nullptr; }
 
-int tc_launches(const DecodeShape&) { return 2; }
+int tc_launches(const DecodeShape&, bool rope_keys) { return rope_keys ? 3 : 2; }
 
 void tc_plan_destroy(TcPlan* plan) {
   if (!plan) return;
@@ -1312,6 +1330,7 @@ void tc_plan_destroy(TcPlan* plan) {
   cudaFree(plan->part_acc);
   cudaFree(plan->part_ml);
   cudaFree(plan->d_maps);
+  cudaFree(plan->krope);
   delete plan;
 }
 
@@ -1516,7 +1535,8 @@ constexpr int kRecWords = (int)(sizeof(CtaRec) / sizeof(int));
 // at most `cap` items to `out` and sets every record's item range; returns the item count, or -1 when `cap` is
 // too small, a coordinate does not fit the TMA's 32 bits or a rank lies outside [1, d].
 int64_t build_items(const DecodeShape& s, const int32_t* host_ranks, const int* w, int grid, int off_segs,
-                    int off_sel, CtaRec* recs, Item* out, int64_t cap, bool q8) {
+                    int off_sel, CtaRec* recs, Item* out, int64_t cap, int mode) {
+  const bool q8 = mode == kMode8bit, dk = mode == kModeDenseKeys;
   const uint32_t ring_bytes = q8 ? Smem<true>::kRingBytes : Smem<false>::kRingBytes;
   const int nb = s.nb, cpb = s.n / kChunk, G = s.Hq / s.H, ncb = s.d / 64;
   const int ipt = std::min(s.Bq, 128 / G);
@@ -1564,6 +1584,7 @@ int64_t build_items(const DecodeShape& s, const int32_t* host_ranks, const int* 
     struct BI {
       int rk, rv;
       int64_t rowk, rowv;
+      int b;  // the block's index in its pool
     };
     for (int si = w[k]; si < w[k + 1]; ++si) {
       const Seg& sg = segs[si];
@@ -1584,7 +1605,7 @@ int64_t build_items(const DecodeShape& s, const int32_t* host_ranks, const int* 
       auto info = [&](int vb) {
         const int b = sel ? sel[(size_t)sg.h * nb + vb] : vb;
         const size_t ik = (size_t)(2 * sg.h) * nb + b, iv = (size_t)(2 * sg.h + 1) * nb + b;
-        const BI r{host_ranks[ik], host_ranks[iv], row0[ik], row0[iv]};
+        const BI r{host_ranks[ik], host_ranks[iv], row0[ik], row0[iv], b};
         if (r.rk < 1 || r.rk > s.d || r.rv < 1 || r.rv > s.d) fits = false;
         return r;
       };
@@ -1593,23 +1614,28 @@ int64_t build_items(const DecodeShape& s, const int32_t* host_ranks, const int* 
         // bf16: two 64-token column blocks; 8-bit: one 128-byte row of codes per component
         ring(kMapTok + pad(r) / 16 - 1, r0 * cpb + (int64_t)cc * r, pad(r), q8 ? 1 : 2);
       };
+      // the keys of chunk cc of a block: its K factor slab, or (dense-key mode) 128 rows of the rotated keys
+      auto key_item = [&](const BI& x, int cc) {
+        if (dk) ring(kMapKrope, ((int64_t)sg.h * s.nb + x.b) * s.n + (int64_t)cc * kChunk, kChunk, ncb);
+        else tok_item(x.rowk, x.rk, cc);
+      };
       int c = sg.c0;
       BI bi = info(c / cpb), prev{};
       bool have_prev = false;
-      dim_item(bi.rowk, bi.rk);
+      if (!dk) dim_item(bi.rowk, bi.rk);
       while (true) {
         const int blk = c / cpb, cc0 = c - blk * cpb;
         const int nch = std::min(sg.c1, (blk + 1) * cpb) - c;
         const bool next = c + nch < sg.c1;
         const BI bn = next ? info(blk + 1) : BI{};
-        tok_item(bi.rowk, bi.rk, cc0);
-        if (nch >= 2) tok_item(bi.rowk, bi.rk, cc0 + 1);
-        else if (next) dim_item(bn.rowk, bn.rk);
+        key_item(bi, cc0);
+        if (nch >= 2) key_item(bi, cc0 + 1);
+        else if (next && !dk) dim_item(bn.rowk, bn.rk);
         if (have_prev) dim_item(prev.rowv, prev.rv);
         for (int j = 0; j < nch; ++j) {
           tok_item(bi.rowv, bi.rv, cc0 + j);
-          if (j + 2 < nch) tok_item(bi.rowk, bi.rk, cc0 + j + 2);
-          else if (j + 2 == nch && next) dim_item(bn.rowk, bn.rk);
+          if (j + 2 < nch) key_item(bi, cc0 + j + 2);
+          else if (j + 2 == nch && next && !dk) dim_item(bn.rowk, bn.rk);
         }
         if (!next) break;
         prev = bi;
@@ -1663,7 +1689,7 @@ static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& 
   host.resize((size_t)off_items + (size_t)icap * kItemWords);
   recs = reinterpret_cast<CtaRec*>(host.data() + pl->off_rec);
   const int64_t nitems = build_items(s, in.host_ranks, host.data(), grid, off_segs, pl->off_sel, recs,
-                                     reinterpret_cast<Item*>(host.data() + off_items), icap, in.q8);
+                                     reinterpret_cast<Item*>(host.data() + off_items), icap, mode_of(in));
   if (nitems < 0 || off_items + nitems * kItemWords > INT32_MAX) return cudaErrorInvalidValue;
   pl->off_items = off_items;
   const int nwords_all = (int)(off_items + nitems * kItemWords);
@@ -1698,7 +1724,11 @@ static cudaError_t build_plan(TcPlan* pl, const DecodeShape& s, const TcInputs& 
   pl->tok = in.tok;
   pl->dim = in.dim;
   pl->q8 = in.q8;
-  return prepare_kernel(D, in.q8);
+  pl->rope = in.rope_keys;
+  if (in.rope_keys &&
+      (e = cudaMalloc(&pl->krope, (size_t)s.H * s.nb * s.n * s.d * 2)) != cudaSuccess)
+    return e;
+  return prepare_kernel(D, mode_of(in));
 }
 
 cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, void* out, cudaStream_t st,
@@ -1708,7 +1738,7 @@ cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, v
                                            std::memcmp(pl->mask.data(), mask, pl->mask.size()) == 0
                                      : pl->mask.empty());
   if (!pl || pl->Bq != s.Bq || pl->Hq != s.Hq || pl->S != s.S || pl->tok != in.tok || pl->q8 != in.q8 ||
-      !same_mask) {
+      pl->rope != in.rope_keys || !same_mask) {
     tc_plan_destroy(pl);
     *plan = nullptr;
     pl = new TcPlan();
@@ -1722,6 +1752,14 @@ cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, v
   const int D = s.d, G = s.Hq / s.H;
   Maps maps;
   if (!make_call_maps(&maps, s, in, pl->ipt)) return cudaErrorInvalidValue;
+  if (in.rope_keys) {
+    // the prefix keys, rebuilt from their pre-RoPE factors and rotated, as [H·T][d] rows
+    if (!make_rows_map(&maps.krope, pl->krope, D, (uint64_t)s.H * s.nb * s.n, kChunk)) return cudaErrorInvalidValue;
+    const RopeShape rs{s.H, s.nb, s.n, s.d, in.rope_theta};
+    const RopeBuffers rb{in.tok, in.dim, in.ranks, in.row_offsets, pl->krope, in.status};
+    cudaError_t re = launch_rope_keys(rs, rb, st);
+    if (re != cudaSuccess) return re;
+  }
   Params p;
   p.recs = reinterpret_cast<const CtaRec*>(pl->d_work + pl->off_rec);
   p.items = reinterpret_cast<const Item*>(pl->d_work + pl->off_items);
@@ -1742,7 +1780,7 @@ cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, v
   p.c = s.scale * 1.4426950408889634f;
   cudaError_t e;
   if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
-  e = launch_decode_kernel(D, in.q8, pl->grid, maps, p, st);
+  e = launch_decode_kernel(D, mode_of(in), pl->grid, maps, p, st);
   if (e != cudaSuccess) return e;
   if (ev1 && (e = cudaEventRecord(ev1, st)) != cudaSuccess) return e;
   const int* pre = pl->d_work + pl->off_pre;
@@ -1800,7 +1838,7 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
   }
   const int kind = (s.d == 64 ? 0 : 1) + (in.q8 ? 2 : 0);
   if (!g_noalloc_ready[dev][kind]) {
-    if ((e = prepare_kernel(s.d, in.q8)) != cudaSuccess) return e;
+    if ((e = prepare_kernel(s.d, mode_of(in))) != cudaSuccess) return e;
     g_noalloc_ready[dev][kind] = true;
   }
   unsigned char* scratch = static_cast<unsigned char*>(g_noalloc_dev_ptr[dev]);
@@ -1822,7 +1860,7 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
     const int64_t room = ((int64_t)kNoAllocMaxWords - off_items) / kItemWords;
     const int64_t nitems = room > 0 ? build_items(s, in.host_ranks, g_noalloc_host_words, grid, off_segs, -1, recs,
                                                   reinterpret_cast<Item*>(g_noalloc_host_words + off_items), room,
-                                                  in.q8)
+                                                  mode_of(in))
                                     : -1;
     nwords = nitems < 0 ? -1 : (int)(off_items + nitems * kItemWords);
   }
@@ -1872,7 +1910,7 @@ cudaError_t tc_decode_noalloc(const DecodeShape& s, const TcInputs& in, void* ou
   p.ipt = ipt;
   p.S = s.S;
   p.c = s.scale * 1.4426950408889634f;
-  if ((e = launch_decode_kernel(D, in.q8, grid, maps, p, st)) != cudaSuccess) return e;
+  if ((e = launch_decode_kernel(D, mode_of(in), grid, maps, p, st)) != cudaSuccess) return e;
   return launch_combine(s, part_acc, part_ml, d_work + off_pre, d_work + off_suf, ipt, nrt, out, st);
 }
 

@@ -22,12 +22,16 @@ struct TcInputs {
   int64_t total_rows;  // rows of the factor arrays (Σ of every block's rank)
   const int32_t* host_ranks;  // [2H][nb]
   bool q8 = false;            // tok holds int8 codes (8-bit factor object), dim bf16
+  // Pre-RoPE key factors: the prefix keys are rebuilt and rotated (base rope_theta) into rope_keys
+  // ([H][T][d] bf16 scratch) before the decode, which then scores them densely.
+  bool rope_keys = false;
+  double rope_theta = 0.0;
 };
 
 // The shape check alone (no CUDA call): bf16 (or 8-bit) factors, d in {64, 128}, n % 128 == 0, GQA group <= 128.
 bool tc_shape_ok(const DecodeShape& s);
 bool tc_supported(const DecodeShape& s);
-int tc_launches(const DecodeShape& s);
+int tc_launches(const DecodeShape& s, bool rope_keys = false);
 // ev0 / ev1 (optional) are recorded on `st` right before and right after the main decode kernel.
 // mask (optional, host [H][nb], nonzero = attended): block selection; the plan is rebuilt when it changes.
 cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, void* out, cudaStream_t st,

@@ -499,13 +499,15 @@ int32_t milo_decode_launches(const milo_factors* f, int32_t batch, int32_t num_q
 static milo_status decode_impl(const void* q, int32_t batch, int32_t num_q_heads, const milo_factors* fc,
                                const void* K_suffix, const void* V_suffix, int32_t suffix_len, float scale,
                                void* out, void* stream, cudaEvent_t ev0, cudaEvent_t ev1,
-                               const uint8_t* mask = nullptr) {
+                               const uint8_t* mask = nullptr, double rope_theta = 0.0) {
   if (!fc || !q || !out || batch <= 0 || num_q_heads <= 0 || suffix_len < 0) return MILO_ERR_INVALID_ARGUMENT;
   milo_factors* f = const_cast<milo_factors*>(fc);
   if (num_q_heads % f->H != 0) return MILO_ERR_INVALID_ARGUMENT;
   if (suffix_len > 0 && (!K_suffix || !V_suffix)) return MILO_ERR_INVALID_ARGUMENT;
   if (!(scale == scale) || isinf(scale)) return MILO_ERR_INVALID_ARGUMENT;
   if (batch > 65535 || num_q_heads > 4096 || suffix_len > (1 << 20)) return MILO_ERR_INVALID_ARGUMENT;
+  if (rope_theta != 0.0 && !(rope_theta > 1.0 && isfinite(rope_theta))) return MILO_ERR_INVALID_ARGUMENT;
+  if (rope_theta != 0.0 && f->dtype != MILO_BF16) return MILO_ERR_UNSUPPORTED;  // bf16 key factors only
   if (mask && suffix_len == 0) {  // a head with no selected block and no suffix has nothing to attend
     for (int h = 0; h < f->H; ++h) {
       bool any = false;
@@ -532,11 +534,11 @@ static milo_status decode_impl(const void* q, int32_t batch, int32_t num_q_heads
     }
     milo::TcInputs in{q,        K_suffix,       V_suffix,  f->tok,        f->dim,
                       f->ranks, f->row_offsets, f->status, f->total_rows, f->host_ranks.data(),
-                      f->dtype == MILO_I8};
+                      f->dtype == MILO_I8, rope_theta > 0.0, rope_theta};
     return cuda_status(milo::tc_decode(&f->tc_plan, ds, in, out, s, ev0, ev1, mask));
   }
-  // block selection and 8-bit factors run on the tensor-core decode only
-  if (mask || f->dtype == MILO_I8) return MILO_ERR_UNSUPPORTED;
+  // block selection, 8-bit factors and pre-RoPE keys run on the tensor-core decode only
+  if (mask || f->dtype == MILO_I8 || rope_theta > 0.0) return MILO_ERR_UNSUPPORTED;
   const size_t need = milo::simt_decode_partials_floats(ds);
   if (need > f->partials_floats) {
     MILO_CUDA(cudaStreamSynchronize(s));
@@ -596,6 +598,14 @@ milo_status milo_decode_attn_select(const void* q, int32_t batch, int32_t num_q_
   if (!host_block_mask) return MILO_ERR_INVALID_ARGUMENT;
   return decode_impl(q, batch, num_q_heads, f, K_suffix, V_suffix, suffix_len, scale, out, stream, nullptr,
                      nullptr, host_block_mask);
+}
+
+milo_status milo_decode_attn_rope(const void* q, int32_t batch, int32_t num_q_heads, const milo_factors* f,
+                                  const void* K_suffix, const void* V_suffix, int32_t suffix_len, float scale,
+                                  double rope_theta, const uint8_t* host_block_mask, void* out, void* stream) {
+  if (!(rope_theta > 1.0)) return MILO_ERR_INVALID_ARGUMENT;
+  return decode_impl(q, batch, num_q_heads, f, K_suffix, V_suffix, suffix_len, scale, out, stream, nullptr,
+                     nullptr, host_block_mask, rope_theta);
 }
 
 milo_status milo_decode_attn_profiled(const void* q, int32_t batch, int32_t num_q_heads, const milo_factors* f,

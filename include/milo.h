@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define MILO_ABI_VERSION 3
+#define MILO_ABI_VERSION 4
 
 typedef enum {
   MILO_OK = 0,
@@ -219,6 +219,32 @@ milo_status milo_decode_attn_select(const void* q, int32_t batch, int32_t num_q_
                                     const milo_factors* f, const void* K_suffix, const void* V_suffix,
                                     int32_t suffix_len, float scale, const uint8_t* host_block_mask,
                                     void* out, void* stream);
+
+/*
+ * milo_decode_attn_rope — milo_decode_attn for factors of keys compressed before
+ * the rotary embedding.  Source: §3 and Figure 1 (pre-RoPE keys are more
+ * low-rank, which suits block-wise compression) and §4.4–§4.5 (inference
+ * reconstructs the selected blocks before attention).  The rank-space identity
+ * does not hold for rotated keys (the rotation depends on the token), so this
+ * call first rebuilds every key block K_b = U_b·B_bᵀ and rotates each token t of
+ * the prefix at its absolute position t: dimension i < d/2 pairs with i + d/2
+ * and the pair turns by t·rope_theta^(−2i/d),
+ *   y_i = x_i·cos φ − x_{i+d/2}·sin φ,  y_{i+d/2} = x_{i+d/2}·cos φ + x_i·sin φ,
+ * into a [H][T][d] bf16 scratch held by the factor object; the decode then
+ * scores q against those keys densely, with the values in rank space as in
+ * milo_decode_attn.  q and the suffix keys are taken as already rotated at
+ * their own positions.
+ *   rope_theta       rotary base, > 1 (the Qwen2.5 models use 1e6).
+ *   host_block_mask  NULL (every block) or host [H][nb] as in milo_decode_attn_select.
+ * bf16 factor objects only (MILO_ERR_UNSUPPORTED for fp32 and 8-bit objects).
+ * Three launches per call.  The first call for a shape allocates the scratch
+ * (H·T·d·2 bytes) besides the usual work list.  Other arguments, results and
+ * errors as milo_decode_attn.
+ */
+milo_status milo_decode_attn_rope(const void* q, int32_t batch, int32_t num_q_heads,
+                                  const milo_factors* f, const void* K_suffix, const void* V_suffix,
+                                  int32_t suffix_len, float scale, double rope_theta,
+                                  const uint8_t* host_block_mask, void* out, void* stream);
 
 /*
  * milo_decode_attn_profiled — milo_decode_attn that also records two caller-created

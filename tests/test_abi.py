@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol():
     assert {"milo_compress", "milo_decode_attn"} <= names
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.milo_abi_version() == 3
+    assert lib.milo_abi_version() == 4
     assert lib.milo_status_string(0) == b"ok"
     assert lib.milo_status_string(3).startswith(b"budget")
 
@@ -187,3 +187,11 @@ def test_import_checks_array_sizes_for_8bit():
     with pytest.raises(ValueError):  # bf16-sized codes for an 8-bit object
         milo.import_factors(milo.I8, 1, 1024, 64, 512, 4, ranks, np.zeros((20, 512), np.uint16),
                             np.zeros((20, 64), np.uint16))
+
+
+def test_rope_decode_rejects_bad_arguments():
+    lib = milo.load_library()
+    # no factor object, and a rotary base that is not > 1 (checked before anything else runs)
+    assert lib.milo_decode_attn_rope(None, 1, 1, None, None, None, 0, 0.0, 1e6, None, None, None) == 1
+    assert lib.milo_decode_attn_rope(None, 1, 1, None, None, None, 0, 0.0, 1.0, None, None, None) == 1
+    assert lib.milo_decode_attn_rope(None, 1, 1, None, None, None, 0, 0.0, float("nan"), None, None, None) == 1
