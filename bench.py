@@ -284,6 +284,35 @@ def _decode_8bit(torch, milo, wl, sets, qs, ks, vs, outs, steps, peak):
                     "factors bf16; same timing as the main kernel"}
 
 
+def _decode_rope(torch, milo, wl, sets, qs, ks, vs, outs, steps, peak, ranks):
+    """Pre-RoPE key factors (milo_decode_attn_rope): the whole call (key rebuild and rotation, decode,
+    combine), timed with CUDA events around each eager call over the copies."""
+    copies = len(sets)
+    for c in range(copies):
+        milo.decode_attn_rope(qs[c], sets[c], ks[c], vs[c], theta=1e6, out=outs[c])
+    torch.cuda.synchronize()
+    n = min(steps, 200)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for s_ in range(n):
+        c = s_ % copies
+        evs[s_][0].record()
+        milo.decode_attn_rope(qs[c], sets[c], ks[c], vs[c], theta=1e6, out=outs[c])
+        evs[s_][1].record()
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    ok = all(f.status()[0] == 0 for f in sets)
+    keys = wl.kv_heads * wl.context * wl.head_dim * 2
+    kf = int(ranks[0::2].sum()) * (wl.block_size + wl.head_dim) * 2
+    vf = int(ranks[1::2].sum()) * (wl.block_size + wl.head_dim) * 2
+    rest = 2 * wl.batch * wl.kv_heads * wl.suffix * wl.head_dim * 2 + 2 * wl.batch * wl.q_heads * wl.head_dim * 2
+    nbytes = kf + 2 * keys + vf + rest  # rebuild reads the key factors, writes the keys; decode reads them back
+    achieved = nbytes / (ms / 1e3) / 1e9
+    return {"call_ms": ms, "bytes_per_step": nbytes, "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "decode_tokens_per_s": wl.batch / (ms / 1e3), "status_ok": ok,
+            "note": "3 launches per call (key rebuild and rotation, decode over dense rotated keys, combine); "
+                    "bytes: key factors read, rotated keys written and read back, value factors, suffix, q, out"}
+
+
 def _oracle_layer(wl, L):
     """The oracle's compression of the workload's layer (fp64, stored factors as the decode reads them)."""
     import oracle
@@ -589,6 +618,7 @@ def run_milo(a):
     kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
     peak, peak_kind = _peaks()
     dec8 = _decode_8bit(torch, milo, wl, sets, qs, ks, vs, outs, steps, peak) if dt == "bf16" else None
+    decr = _decode_rope(torch, milo, wl, sets, qs, ks, vs, outs, steps, peak, ranks) if dt == "bf16" else None
 
     # --- end to end through the public API: pinned host inputs, copies inside the timed region.  Steps
     # alternate between two streams with their own device buffers, so the host-to-device copies of one
@@ -653,6 +683,7 @@ def run_milo(a):
                          "unit": "whole-layer compressions/s",
                          "roofline": _compress_roofline(torch, wl, esize, comp_ranks, sweeps, kern, peak)},
             "decode_8bit": dec8,
+            "decode_pre_rope": decr,
             "gpu_launches": kernels_per_call * steps,
             "gpu_launches_note": f"{kernels_per_call} kernels per decode call x {steps} steps of one timed window "
                                  f"({windows} windows timed, the median reported)",

@@ -1335,16 +1335,17 @@ void tc_plan_destroy(TcPlan* plan) {
 }
 
 // Estimated time of one work atom, used to balance the work list across CTAs.  The weights come from a
-// least-squares fit of per-CTA run times on B200 against their work: a 128-token chunk costs about the
-// same whatever its ranks (softmax and MMA issue dominate its bytes), the first chunk of a block adds the
-// q̃ and ã round trips (G1, conversions, G4), the first chunk of a suffix unit adds a segment's partial.
-constexpr double kChunkNs = 1000.0, kBlockNs = 3000.0, kUnitNs = 1700.0, kBytesPerNs = 150.0;
+// least-squares fit of per-CTA run times on B200 against their work (about 0.9 µs per prefix chunk, 0.8 µs
+// per suffix chunk, 2.6 µs per block visited and per segment): a 128-token chunk costs about the same
+// whatever its ranks (softmax and MMA issue dominate its bytes), the first chunk of a block adds the q̃ and
+// ã round trips (G1, conversions, G4), the first chunk of a suffix unit adds a segment's partial.
+constexpr double kChunkNs = 750.0, kSufChunkNs = 370.0, kBlockNs = 2600.0, kUnitNs = 2600.0, kBytesPerNs = 150.0;
 inline double prefix_atom_ns(int rk, int rv, int cc, int d) {
   const double bytes = 2.0 * (rk + rv) * kChunk + (cc == 0 ? 2.0 * (rk + rv) * d : 0.0);
   return bytes / kBytesPerNs + kChunkNs + (cc == 0 ? kBlockNs : 0.0);
 }
 inline double suffix_atom_ns(int c, int d) {
-  return 2.0 * 2.0 * kChunk * d / kBytesPerNs + kChunkNs + (c == 0 ? kUnitNs : 0.0);
+  return 2.0 * 2.0 * kChunk * d / kBytesPerNs + kSufChunkNs + (c == 0 ? kUnitNs : 0.0);
 }
 
 // The decode work list, written into `w` without heap allocation: atoms (one 128-token chunk of one KV head's
