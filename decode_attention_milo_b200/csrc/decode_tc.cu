@@ -399,6 +399,10 @@ __global__ void __launch_bounds__(threads_of<MODE == kMode8bit>(), 1)
     const Item* items = p.items + sh->rec.item0;
     const int nitems = sh->rec.nitems;
     const CUtensorMap* gmap0 = reinterpret_cast<const CUtensorMap*>(p.gmaps);
+    // Everything before this point reads the library's own tables; the loads below read the caller's q,
+    // suffix and factors, which the kernel before this one on the stream may still be writing (the launch is
+    // a programmatic dependent): wait for that grid first.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const CUtensorMap* pmap0 = reinterpret_cast<const CUtensorMap*>(&maps);
     auto load_item = [&](int i) -> uint4 {
       return i < nitems ? __ldg(reinterpret_cast<const uint4*>(items + i)) : make_uint4(0, 0, 0, 0);
@@ -972,7 +976,12 @@ __global__ void __launch_bounds__(threads_of<MODE == kMode8bit>(), 1)
     const bool storer = warp == kSoftWarp0 && lane == 0;
     bool store_pending = false;
     auto soft_sync = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(kSoftBar), "r"(256) : "memory"); };
+    bool dep_done = false;  // the previous combine on this stream (if any) has finished reading the partials
     auto write_partial = [&](const Seg& sg, bool active, float m_used, float l) -> bool {
+      if (!dep_done) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        dep_done = true;
+      }
       const bool got = wait_bar(bar(B_ACCDONE), (accdone_n - 1) & 1, sh, p.status);
       if (got) ptx::tc_fence_after();
       if (active) {
@@ -1103,6 +1112,9 @@ __global__ void __launch_bounds__(D) combine_tc_kernel(const float* __restrict__
   // launched as a programmatic dependent of the decode kernel: its launch overlaps the decode's last CTAs, and
   // this waits until the decode grid has completed and its partials are visible
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the next decode call on this stream may start its set-up and loads now; it waits for this grid before it
+  // writes the partials read here
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int p0 = pre_range[2 * (h * nrt + rt)], p1 = pre_range[2 * (h * nrt + rt) + 1];
   const int s0 = suf_range[2 * (i * H + h)], s1 = suf_range[2 * (i * H + h) + 1];
   const int npre = p1 - p0, nall = npre + (s1 - s0);
@@ -1217,18 +1229,32 @@ cudaError_t prepare_kernel(int d, int mode) {
   return cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               mode == kMode8bit ? Smem<true>::kBytes : Smem<false>::kBytes);
 }
+// Launched with programmatic stream serialization: when the operation before it on the stream is a kernel (the
+// previous decode call's combine, say), this grid's launch and set-up (barriers, TMEM, its work record) overlap
+// that kernel, and the producer waits for it (griddepcontrol.wait) before loading any caller data; the softmax
+// warps wait again before the first partial write.  Not in the dense-key mode, whose keys the kernel right
+// before it writes.
 template <int MODE>
-void launch_mode(int d, int grid, const Maps& maps, const Params& p, cudaStream_t st) {
+cudaError_t launch_mode(int d, int grid, const Maps& maps, const Params& p, cudaStream_t st) {
   constexpr bool q8 = MODE == kMode8bit;
-  if (d == 64) decode_tc_kernel<64, MODE><<<grid, threads_of<q8>(), Smem<q8>::kBytes, st>>>(maps, p);
-  else decode_tc_kernel<128, MODE><<<grid, threads_of<q8>(), Smem<q8>::kBytes, st>>>(maps, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads_of<q8>());
+  cfg.dynamicSmemBytes = Smem<q8>::kBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = MODE == kModeDenseKeys ? 0 : 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (d == 64) return cudaLaunchKernelEx(&cfg, decode_tc_kernel<64, MODE>, maps, p);
+  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<128, MODE>, maps, p);
 }
 // Launches the decode kernel of head dimension d in `mode`.
 cudaError_t launch_decode_kernel(int d, int mode, int grid, const Maps& maps, const Params& p, cudaStream_t st) {
-  if (mode == kMode8bit) launch_mode<kMode8bit>(d, grid, maps, p, st);
-  else if (mode == kModeDenseKeys) launch_mode<kModeDenseKeys>(d, grid, maps, p, st);
-  else launch_mode<kModeRank>(d, grid, maps, p, st);
-  return cudaGetLastError();
+  if (mode == kMode8bit) return launch_mode<kMode8bit>(d, grid, maps, p, st);
+  if (mode == kModeDenseKeys) return launch_mode<kModeDenseKeys>(d, grid, maps, p, st);
+  return launch_mode<kModeRank>(d, grid, maps, p, st);
 }
 int mode_of(const TcInputs& in) { return in.q8 ? kMode8bit : in.rope_keys ? kModeDenseKeys : kModeRank; }
 

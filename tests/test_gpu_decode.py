@@ -168,3 +168,30 @@ def test_decode_large_batch_7b():
     wl, dt, lay, f, q, Ks, Vs = _setup("qwen2.5-7b-layer", batch=300)
     out, want = _run(wl, dt, lay, f, q, Ks, Vs, sample=[0, 17, 18, 151, 287, 288, 299])
     assert_close(out, want, TOL[dt], "batch 300")
+
+
+def test_back_to_back_calls_with_inputs_written_just_before():
+    """Each call's q is written by a kernel right before it on the same stream, and the calls follow each
+    other with no synchronisation (the decode is launched as a programmatic dependent of the kernel before
+    it, and reuses the partials the previous call's combine reads): twelve such calls equal the same calls
+    run one at a time."""
+    import torch
+    import decode_attention_milo_b200 as milo
+    wl, dt, lay, f, q, Ks, Vs = _setup("qwen2.5-7b-layer")
+    tq, tk, tv = to_torch(q, dt), to_torch(Ks, dt), to_torch(Vs, dt)
+    scales = [1.0 + 0.25 * k for k in range(12)]
+    ref = []
+    for sc in scales:
+        qq = tq * sc
+        torch.cuda.synchronize()
+        ref.append(milo.decode_attn(qq, f, tk, tv))
+        torch.cuda.synchronize()
+    buf = torch.empty_like(tq)
+    outs = []
+    for sc in scales:
+        torch.mul(tq, sc, out=buf)  # a kernel that writes q right before the decode on the same stream
+        outs.append(milo.decode_attn(buf, f, tk, tv))
+    torch.cuda.synchronize()
+    for k, (a, b) in enumerate(zip(outs, ref)):
+        assert torch.equal(a, b), k
+    assert f.status()[0] == 0
