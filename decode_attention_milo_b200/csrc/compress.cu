@@ -26,6 +26,10 @@ constexpr int kThreads = 256;
 // the latency of each round: 16 warps, 4 column pairs per warp per round (d = 128).
 constexpr int kJThreads = 512;
 constexpr float kJacobiTol = 1e-5f;  // relative orthogonality |a_p·a_q| / (|a_p||a_q|)
+// A sweep whose largest relative off-diagonal stays below this ends the iteration: cyclic Jacobi converges
+// quadratically, so what remains after it is of order 1e-7, below kJacobiTol, and the next sweep would
+// rotate nothing.
+constexpr float kJacobiExit = 3e-4f;
 
 template <typename T>
 __device__ __forceinline__ const T* pool_block(const T* K, const T* V, int p, int b, int64_t T_, int n,
@@ -279,12 +283,11 @@ __global__ void __launch_bounds__(kEThreads, 3) eig_kernel(const float* __restri
     ss = warp_sum(ss);
     if (lane == 0) nrm[j] = ss;
   }
-  __syncthreads();
   bool converged = false;
   int sweeps_run = 0;
   for (int sweep = 0; sweep < max_sweeps; ++sweep) {
     ++sweeps_run;
-    int rotated = 0;
+    int rotated = 0, big = 0;  // big: some relative off-diagonal of this sweep reached kJacobiExit
     for (int s = 0; s < D - 1; ++s) {
 #pragma unroll 1
       for (int g0 = 0; g0 < PP; g0 += PG) {
@@ -315,7 +318,9 @@ __global__ void __launch_bounds__(kEThreads, 3) eig_kernel(const float* __restri
         for (int t = 0; t < PG; ++t) {
           const int p = pj[t], q = qj[t];
           const float al = nrm[p], be = nrm[q];
-          if (ga[t] != 0.f && fabsf(ga[t]) > kJacobiTol * sqrtf(al) * sqrtf(be)) {
+          const float nn = sqrtf(al) * sqrtf(be), ag = fabsf(ga[t]);
+          big |= ag > 0.f && ag >= kJacobiExit * nn;
+          if (ga[t] != 0.f && ag > kJacobiTol * nn) {
             const float zeta = (be - al) / (2.f * ga[t]);
             const float tn = (zeta >= 0.f ? 1.f : -1.f) / (fabsf(zeta) + sqrtf(1.f + zeta * zeta));
             const float c = 1.f / sqrtf(1.f + tn * tn);
@@ -347,7 +352,8 @@ __global__ void __launch_bounds__(kEThreads, 3) eig_kernel(const float* __restri
       ss = warp_sum(ss);
       if (lane == 0) nrm[j] = ss;
     }
-    if (!__syncthreads_or(rotated)) {
+    const int any_rotated = __syncthreads_or(rotated), any_big = __syncthreads_or(big);
+    if (!any_rotated || !any_big) {
       converged = true;
       break;
     }

@@ -26,7 +26,7 @@ struct CompressBuffers {
   const void* V;
   float* gram;        // [2H][nb][d][d]
   float* eigvals;     // [2H][nb][d]
-  int32_t* sweeps;    // [2H][nb] Jacobi sweeps run per block (the last one found no pair to rotate)
+  int32_t* sweeps;    // [2H][nb] Jacobi sweeps run per block (the last one converged)
   float* eigvecs;     // [2H][nb][d][d]
   double* entropy;    // [2H][nb]
   double* quotas;     // [2H][nb]

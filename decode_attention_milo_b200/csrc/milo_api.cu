@@ -176,9 +176,11 @@ static milo_status compress_impl(const void* K, const void* V, int32_t dtype, in
     return cuda_status(err);
   };
   if (e != cudaSuccess) return fail(e);
+  // stream-ordered allocations: no device-wide synchronisation per array (the object's users order after
+  // its ready event; milo_factors_destroy synchronises before freeing)
 #define ALLOC(ptr, bytes)                                   \
   do {                                                      \
-    e = cudaMalloc((void**)&(ptr), (bytes));                \
+    e = cudaMallocAsync((void**)&(ptr), (bytes), s);        \
     if (e != cudaSuccess) return fail(e);                   \
   } while (0)
   ALLOC(f->ranks, nblk * sizeof(int32_t));

@@ -110,7 +110,8 @@ typedef struct {
   const double* quotas;       /* device [2H][nb], real quotas before rounding          */
   /* present for objects made by milo_compress (NULL for imported ones): */
   const int32_t* sweeps;      /* device [2H][nb], Jacobi sweeps run per block (the last  */
-                              /* one rotated no pair; max_sweeps means no convergence)    */
+                              /* one rotated no pair or left every relative off-diagonal  */
+                              /* below 3e-4; max_sweeps means no convergence)             */
 } milo_factors_desc;
 
 /*
