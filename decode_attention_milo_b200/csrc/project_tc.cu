@@ -38,8 +38,8 @@ constexpr int kPThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 conversion
 constexpr int kPStages = 3;
 constexpr uint64_t kPWaitNs = 1000000000ull;
 
-enum PBar { P_FULL = 0, P_EMPTY = P_FULL + kPStages, P_AREADY = P_EMPTY + kPStages, P_TFULL, P_TEMPTY = P_TFULL + 2,
-            P_DONE = P_TEMPTY + 2, P_COUNT };
+enum PBar { P_FULL = 0, P_EMPTY = P_FULL + kPStages, P_AREADY = P_EMPTY + kPStages, P_AFREE = P_AREADY + 2,
+            P_TFULL = P_AFREE + 2, P_TEMPTY = P_TFULL + 2, P_DONE = P_TEMPTY + 2, P_COUNT };
 
 // Warp-collective bounded wait; false after kPWaitNs (the status flag is set).
 __device__ __noinline__ bool pwait(uint32_t bar, uint32_t parity, uint32_t* status) {
@@ -69,7 +69,8 @@ __device__ __forceinline__ uint64_t pdesc(uint32_t tile, int k) {
 
 template <int D>
 __global__ void __launch_bounds__(kPThreads) project_tc_kernel(const __grid_constant__ ProjMaps maps, int64_t T_,
-                                                              int n, int nb, const float* __restrict__ eigvecs,
+                                                              int n, int nb, int nblocks,
+                                                              const float* __restrict__ eigvecs,
                                                               const int32_t* __restrict__ ranks,
                                                               const int64_t* __restrict__ row_offsets,
                                                               __nv_bfloat16* __restrict__ tok,
@@ -81,22 +82,20 @@ __global__ void __launch_bounds__(kPThreads) project_tc_kernel(const __grid_cons
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t base = ptx::smem_u32(smem);
-  const uint32_t a_hi = base, a_lo = base + kATile, ring = base + 2 * kATile;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kATile + kPStages * kStage);
+  // two A buffers (hi, lo each), then the X ring
+  auto a_hi = [&](int ab) { return base + (uint32_t)(2 * ab) * kATile; };
+  auto a_lo = [&](int ab) { return base + (uint32_t)(2 * ab + 1) * kATile; };
+  const uint32_t ring = base + 4 * kATile;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 4 * kATile + kPStages * kStage);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + P_COUNT);
   auto bar = [&](int i) { return ptx::smem_u32(&bars[i]); };
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int b = blockIdx.x, p = blockIdx.y;
-  const int r = ranks[(int64_t)p * nb + b];
-  const int64_t row0 = row_offsets[(int64_t)p * (nb + 1) + b];
-  if (r < 1 || r > D) {  // uniform across the CTA: nothing was started yet
-    if (threadIdx.x == 0) atomicOr(status, kStatusCompressBounds);
-    return;
-  }
   if (threadIdx.x == 0) {
-    // the A operand and the accumulator releases get one arrival from each of the four epilogue warps
-    for (int i = 0; i < P_COUNT; ++i)
-      ptx::mbar_init(bar(i), i == P_AREADY || i == P_TEMPTY || i == P_TEMPTY + 1 ? 4 : 1);
+    // the A operands and the accumulator releases get one arrival from each of the four epilogue warps
+    for (int i = 0; i < P_COUNT; ++i) {
+      const bool four = i == P_AREADY || i == P_AREADY + 1 || i == P_TEMPTY || i == P_TEMPTY + 1;
+      ptx::mbar_init(bar(i), four ? 4 : 1);
+    }
     ptx::fence_mbar_init();
   }
   if (warp == 1) {
@@ -108,45 +107,75 @@ __global__ void __launch_bounds__(kPThreads) project_tc_kernel(const __grid_cons
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int tiles = n / 128;
-  const int64_t xrow0 = (int64_t)(p >> 1) * T_ + (int64_t)b * n;  // first row of X_b in [H·T][d]
-  const CUtensorMap* xmap = (p & 1) ? &maps.v : &maps.k;
+  // the CTA's blocks: flat index u = blockIdx.x + k·gridDim.x over (pool p = u / nb, block b = u % nb)
+  const int nmine = nblocks > (int)blockIdx.x ? (nblocks - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  struct Blk {
+    int p, b, r;
+    int64_t row0;
+  };
+  auto blk = [&](int k) {
+    Blk x;
+    const int u = (int)blockIdx.x + k * (int)gridDim.x;
+    x.p = u / nb;
+    x.b = u % nb;
+    x.r = ranks[(int64_t)x.p * nb + x.b];
+    x.row0 = row_offsets[(int64_t)x.p * (nb + 1) + x.b];
+    if (x.r < 1 || x.r > D) {  // every role clamps alike, so that the pipeline keeps its shape
+      if (threadIdx.x == 0) atomicOr(status, kStatusCompressBounds);
+      x.r = x.r < 1 ? 1 : D;
+    }
+    return x;
+  };
 
   if (warp == 0) {
-    // ---- producer: tile s = tokens [128 s, 128 s + 128) of X_b
-    for (int s = 0; s < tiles; ++s) {
-      const int slot = s % kPStages;
-      if (s >= kPStages && !pwait(bar(P_EMPTY + slot), ((s / kPStages) - 1) & 1, status)) break;
-      if (lane == 0) {
-        const uint32_t dst = ring + slot * kStage;
-        ptx::mbar_arrive_expect_tx(bar(P_FULL + slot), kStage);
-        if (D == 128) ptx::tma_load_3d(dst, xmap, bar(P_FULL + slot), 0, (int)(xrow0 + 128 * s), 0);
-        else ptx::tma_load_2d(dst, xmap, bar(P_FULL + slot), 0, (int)(xrow0 + 128 * s));
+    // ---- producer: tile s of block k = tokens [128 s, 128 s + 128) of X_b, global tile g = k·tiles + s
+    bool ok = true;
+    int g = 0;
+    for (int k = 0; k < nmine && ok; ++k) {
+      const Blk x = blk(k);
+      const int64_t xrow0 = (int64_t)(x.p >> 1) * T_ + (int64_t)x.b * n;  // first row of X_b in [H·T][d]
+      const CUtensorMap* xmap = (x.p & 1) ? &maps.v : &maps.k;
+      for (int s = 0; s < tiles && ok; ++s, ++g) {
+        const int slot = g % kPStages;
+        if (g >= kPStages && !(ok = pwait(bar(P_EMPTY + slot), ((g / kPStages) - 1) & 1, status))) break;
+        if (lane == 0) {
+          const uint32_t dst = ring + slot * kStage;
+          ptx::mbar_arrive_expect_tx(bar(P_FULL + slot), kStage);
+          if (D == 128) ptx::tma_load_3d(dst, xmap, bar(P_FULL + slot), 0, (int)(xrow0 + 128 * s), 0);
+          else ptx::tma_load_2d(dst, xmap, bar(P_FULL + slot), 0, (int)(xrow0 + 128 * s));
+        }
+        __syncwarp();
       }
-      __syncwarp();
     }
     // drain: the CTA's copies have landed before it can exit
-    for (int s = std::max(0, tiles - kPStages); s < tiles; ++s)
-      pwait(bar(P_FULL + s % kPStages), (s / kPStages) & 1, status);
+    for (int h = std::max(0, g - kPStages); h < g; ++h) pwait(bar(P_FULL + h % kPStages), (h / kPStages) & 1, status);
   } else if (warp == 1) {
     // ---- MMA issuer: Uᵀ tile = A_hi · Xᵀ + A_lo · Xᵀ, M = 128 rank rows, N = 128 tokens, K = d
     constexpr uint32_t idesc = ptx::idesc_bf16(128, 128, false, false);
-    bool ok = pwait(bar(P_AREADY), 0, status);
-    ptx::tc_fence_after();
-    for (int s = 0; s < tiles && ok; ++s) {
-      const int slot = s % kPStages, buf = s & 1;
-      if (s >= 2) ok = pwait(bar(P_TEMPTY + buf), ((s >> 1) - 1) & 1, status);
-      if (ok) ok = pwait(bar(P_FULL + slot), (s / kPStages) & 1, status);
+    bool ok = true;
+    int g = 0;
+    for (int k = 0; k < nmine && ok; ++k) {
+      const int ab = k & 1;
+      ok = pwait(bar(P_AREADY + ab), (k >> 1) & 1, status);
       ptx::tc_fence_after();
-      if (ok && lane == 0) {
-        const uint32_t xs = ring + slot * kStage, d_t = tmem + 128u * buf;
+      for (int s = 0; s < tiles && ok; ++s, ++g) {
+        const int slot = g % kPStages, buf = g & 1;
+        if (g >= 2) ok = pwait(bar(P_TEMPTY + buf), ((g >> 1) - 1) & 1, status);
+        if (ok) ok = pwait(bar(P_FULL + slot), (g / kPStages) & 1, status);
+        ptx::tc_fence_after();
+        if (ok && lane == 0) {
+          const uint32_t xs = ring + slot * kStage, d_t = tmem + 128u * buf;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          ptx::umma_bf16(d_t, pdesc(a_hi, k), pdesc(xs, k), idesc, k > 0 ? 1u : 0u);
-          ptx::umma_bf16(d_t, pdesc(a_lo, k), pdesc(xs, k), idesc, 1u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            ptx::umma_bf16(d_t, pdesc(a_hi(ab), kk), pdesc(xs, kk), idesc, kk > 0 ? 1u : 0u);
+            ptx::umma_bf16(d_t, pdesc(a_lo(ab), kk), pdesc(xs, kk), idesc, 1u);
+          }
+          ptx::umma_commit(bar(P_EMPTY + slot));  // the stage may be reloaded once these MMAs have read it
+          ptx::umma_commit(bar(P_TFULL + buf));   // the accumulator is complete
         }
-        ptx::umma_commit(bar(P_EMPTY + slot));  // the stage may be reloaded once these MMAs have read it
-        ptx::umma_commit(bar(P_TFULL + buf));   // the accumulator is complete
+        __syncwarp();
       }
+      if (ok && lane == 0) ptx::umma_commit(bar(P_AFREE + ab));  // block k's A buffer may be rewritten
       __syncwarp();
     }
     // drain: every MMA issued has completed before TMEM is freed (the epilogue normally waited already)
@@ -154,62 +183,96 @@ __global__ void __launch_bounds__(kPThreads) project_tc_kernel(const __grid_cons
     __syncwarp();
     pwait(bar(P_DONE), 0, status);
   } else {
-    // ---- warps 2..5: A operand and dimension-side factor, then the epilogue of every tile
-    const int ew = warp - 2;  // 0..3
-    const int quarter = warp & 3;  // a warp reads TMEM lanes [32 (warp % 4), 32 (warp % 4) + 32)
-    const float* ev = eigvecs + ((int64_t)p * nb + b) * D * D;
-    // rows j = ew, ew + 4, ...: lane handles columns [4 lane, 4 lane + 4) of each 128-column block
-    for (int j = ew; j < 128; j += 4) {
+    // ---- warps 2..5: each block's A operand and dimension-side factor (one block ahead of the MMAs), then
+    // the epilogue of its tiles
+    const int ew = warp - 2;        // 0..3
+    const int quarter = warp & 3;   // a warp reads TMEM lanes [32 (warp % 4), 32 (warp % 4) + 32)
+    bool ok = true;
+    auto convert = [&](int k) {
+      const Blk x = blk(k);
+      const int ab = k & 1;
+      // the MMAs of block k − 2 have read this buffer
+      if (k >= 2) ok = ok && pwait(bar(P_AFREE + ab), ((k >> 1) - 1) & 1, status);
+      if (ok) {
+        const float* ev = eigvecs + ((int64_t)x.p * nb + x.b) * D * D;
+        // rows j = ew, ew + 4, ...: lane handles columns [4 lane, 4 lane + 4) of each 128-column block; the
+        // loads of kRows rows are issued together so that their latencies overlap
+        constexpr int kRows = 8;
+        for (int j0 = ew; j0 < 128; j0 += 4 * kRows) {
+          float4 vv[kRows][(D + 127) / 128];
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 128) {
-        const int c = c0 + 4 * lane;
-        if (c >= D) continue;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (j < r) v = *reinterpret_cast<const float4*>(ev + (int64_t)j * D + c);
-        const uint32_t h01 = ptx::pack_bf16(v.x, v.y), h23 = ptx::pack_bf16(v.z, v.w);
-        const uint32_t l01 = ptx::pack_bf16(v.x - __uint_as_float(h01 << 16), v.y - __uint_as_float(h01 & 0xFFFF0000u));
-        const uint32_t l23 = ptx::pack_bf16(v.z - __uint_as_float(h23 << 16), v.w - __uint_as_float(h23 & 0xFFFF0000u));
-        // K-major SW128 position of (row j, column c): column block c / 64, 16-byte chunk ((c % 64) / 8) ^ (j % 8)
-        const uint32_t off = (uint32_t)(c >> 6) * 16384u + (uint32_t)j * 128u +
-                             ((uint32_t)(((c & 63) >> 3) ^ (j & 7)) << 4) + (uint32_t)(c & 7) * 2u;
-        asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(a_hi + off), "r"(h01), "r"(h23) : "memory");
-        asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(a_lo + off), "r"(l01), "r"(l23) : "memory");
-        if (j < r) {
-          uint2 w;
-          w.x = h01;
-          w.y = h23;
-          *reinterpret_cast<uint2*>(dim + (row0 + j) * D + c) = w;
+          for (int q = 0; q < kRows; ++q) {
+            const int j = j0 + 4 * q;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 128) {
+              const int c = c0 + 4 * lane;
+              vv[q][c0 / 128] = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (c < D && j < x.r) vv[q][c0 / 128] = __ldg(reinterpret_cast<const float4*>(ev + (int64_t)j * D + c));
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < kRows; ++q) {
+          const int j = j0 + 4 * q;
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 128) {
+            const int c = c0 + 4 * lane;
+            if (c >= D) continue;
+            const float4 v = vv[q][c0 / 128];
+            const uint32_t h01 = ptx::pack_bf16(v.x, v.y), h23 = ptx::pack_bf16(v.z, v.w);
+            const uint32_t l01 =
+                ptx::pack_bf16(v.x - __uint_as_float(h01 << 16), v.y - __uint_as_float(h01 & 0xFFFF0000u));
+            const uint32_t l23 =
+                ptx::pack_bf16(v.z - __uint_as_float(h23 << 16), v.w - __uint_as_float(h23 & 0xFFFF0000u));
+            // K-major SW128 position of (row j, column c): column block c / 64, 16-byte chunk ((c % 64) / 8) ^ (j % 8)
+            const uint32_t off = (uint32_t)(c >> 6) * 16384u + (uint32_t)j * 128u +
+                                 ((uint32_t)(((c & 63) >> 3) ^ (j & 7)) << 4) + (uint32_t)(c & 7) * 2u;
+            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(a_hi(ab) + off), "r"(h01), "r"(h23) : "memory");
+            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(a_lo(ab) + off), "r"(l01), "r"(l23) : "memory");
+            if (j < x.r) {
+              uint2 w;
+              w.x = h01;
+              w.y = h23;
+              *reinterpret_cast<uint2*>(dim + (x.row0 + j) * D + c) = w;
+            }
+          }
+          }
         }
       }
-    }
-    ptx::fence_async_smem();
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(bar(P_AREADY));
+      ptx::fence_async_smem();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(P_AREADY + ab));
+    };
     // epilogue: lane j of this warp's quarter holds rank component j = 32 quarter + lane; 128 tokens per tile
     const int j = 32 * quarter + lane;
     const uint32_t tl = tmem + ((uint32_t)(32 * quarter) << 16);
-    for (int s = 0; s < tiles; ++s) {
-      const int buf = s & 1;
-      if (!pwait(bar(P_TFULL + buf), (s >> 1) & 1, status)) break;
-      ptx::tc_fence_after();
-      __nv_bfloat16* dst = tok + row0 * n + (int64_t)s * (r * 128) + (int64_t)j * 128;
+    int g = 0;
+    if (nmine > 0) convert(0);
+    for (int k = 0; k < nmine && ok; ++k) {
+      if (k + 1 < nmine) convert(k + 1);  // the next block's operand is ready before this block's epilogue
+      const Blk x = blk(k);
+      for (int s = 0; s < tiles; ++s, ++g) {
+        const int buf = g & 1;
+        if (!ok || !(ok = pwait(bar(P_TFULL + buf), (g >> 1) & 1, status))) break;
+        ptx::tc_fence_after();
+        __nv_bfloat16* dst = tok + x.row0 * n + (int64_t)s * (x.r * 128) + (int64_t)j * 128;
 #pragma unroll 1
-      for (int c32 = 0; c32 < 128; c32 += 32) {
-        float v[32];
-        ptx::tmem_ld32(tl + 128u * buf + c32, v);
-        ptx::tmem_wait_ld();
-        if (j < r) {
-          uint32_t w[16];
+        for (int c32 = 0; c32 < 128; c32 += 32) {
+          float v[32];
+          ptx::tmem_ld32(tl + 128u * buf + c32, v);
+          ptx::tmem_wait_ld();
+          if (j < x.r) {
+            uint32_t w[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) w[e] = ptx::pack_bf16(v[2 * e], v[2 * e + 1]);
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c32);
+            for (int e = 0; e < 16; ++e) w[e] = ptx::pack_bf16(v[2 * e], v[2 * e + 1]);
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c32);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) d4[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+            for (int q = 0; q < 4; ++q) d4[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+          }
         }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(P_TEMPTY + buf));
       }
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(P_TEMPTY + buf));
     }
   }
   ptx::tc_fence_before();
@@ -242,7 +305,7 @@ bool pmap(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims, con
 
 template <int D>
 constexpr int proj_smem() {
-  return (2 + kPStages) * 16384 * (D / 64) + 8 * P_COUNT + 16 + 1024;
+  return (4 + kPStages) * 16384 * (D / 64) + 8 * P_COUNT + 16 + 1024;
 }
 
 }  // namespace
@@ -266,21 +329,26 @@ cudaError_t launch_project_tc(const CompressShape& s, const void* K, const void*
     const cuuint32_t b2[2] = {64, 128};
     if (!pmap(&maps.k, K, 2, d2, s2, b2) || !pmap(&maps.v, V, 2, d2, s2, b2)) return cudaErrorInvalidValue;
   }
-  const dim3 grid(s.nb, 2 * s.H);
+  const int64_t nblocks = 2LL * s.H * s.nb;
+  if (nblocks > 0x7fffffff) return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const unsigned grid = (unsigned)std::min<int64_t>(nblocks, sms);  // one persistent CTA per SM
   cudaError_t e;
   if (s.d == 128) {
     if ((e = cudaFuncSetAttribute(project_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   proj_smem<128>())) != cudaSuccess)
       return e;
     project_tc_kernel<128><<<grid, kPThreads, proj_smem<128>(), st>>>(
-        maps, s.T, s.n, s.nb, eigvecs, ranks, row_offsets, static_cast<__nv_bfloat16*>(tok),
+        maps, s.T, s.n, s.nb, (int)nblocks, eigvecs, ranks, row_offsets, static_cast<__nv_bfloat16*>(tok),
         static_cast<__nv_bfloat16*>(dim), status);
   } else {
     if ((e = cudaFuncSetAttribute(project_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   proj_smem<64>())) != cudaSuccess)
       return e;
     project_tc_kernel<64><<<grid, kPThreads, proj_smem<64>(), st>>>(
-        maps, s.T, s.n, s.nb, eigvecs, ranks, row_offsets, static_cast<__nv_bfloat16*>(tok),
+        maps, s.T, s.n, s.nb, (int)nblocks, eigvecs, ranks, row_offsets, static_cast<__nv_bfloat16*>(tok),
         static_cast<__nv_bfloat16*>(dim), status);
   }
   return cudaGetLastError();
