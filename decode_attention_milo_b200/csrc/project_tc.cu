@@ -9,11 +9,12 @@
 // The kernel computes the transpose, Uᵀ = B_rᵀ · X_bᵀ, one 128-token tile at a
 // time, so that a TMEM lane holds one rank component and its columns are the
 // tile's tokens: row j of the 128-token slab the decode reads is then one lane's
-// 128 contiguous values.  One CTA per block:
+// 128 contiguous values.  One persistent CTA per SM walks blocks:
 //  - warps 2..5 convert the fp32 eigenvectors (rows 0..r−1, rows r..127 zero)
 //    to a bf16 pair hi + lo (B ≈ hi + lo to about 2^-17 relative), write them as
 //    the K-major A operand (M = 128 rank rows, K = d) in shared memory with the
-//    128-byte swizzle, and store hi as the block's dimension-side factor rows;
+//    128-byte swizzle, into one of two buffers one block ahead of the MMAs, and
+//    store hi as the block's dimension-side factor rows;
 //  - warp 0 streams X_b through a 3-stage ring of 128-token tiles by TMA
 //    (K-major B operand, N = 128 tokens);
 //  - warp 1 issues tcgen05.mma kind::f16, hi and lo per k-step (bf16 products
