@@ -1783,7 +1783,8 @@ cudaError_t tc_decode(TcPlan** plan, const DecodeShape& s, const TcInputs& in, v
     // the prefix keys, rebuilt from their pre-RoPE factors and rotated, as [H·T][d] rows
     if (!make_rows_map(&maps.krope, pl->krope, D, (uint64_t)s.H * s.nb * s.n, kChunk)) return cudaErrorInvalidValue;
     const RopeShape rs{s.H, s.nb, s.n, s.d, in.rope_theta};
-    const RopeBuffers rb{in.tok, in.dim, in.ranks, in.row_offsets, pl->krope, in.status};
+    const CUtensorMap* pmaps = reinterpret_cast<const CUtensorMap*>(pl->d_maps);
+    const RopeBuffers rb{pmaps + kMapTok, pmaps + kMapDim, in.ranks, in.row_offsets, &maps.krope, in.status};
     cudaError_t re = launch_rope_keys(rs, rb, st);
     if (re != cudaSuccess) return re;
   }

@@ -214,6 +214,13 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, uint32_t ssrc
                "r"(ssrc), "r"(x), "r"(y)
                : "memory");
 }
+// The same for a 3D map.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, uint32_t ssrc, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(ssrc), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
