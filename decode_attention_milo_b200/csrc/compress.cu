@@ -212,7 +212,6 @@ __global__ void __launch_bounds__(kEThreads, 3) eig_kernel(const float* __restri
   constexpr int E = D / 32;           // elements per lane of one column
   constexpr int NW = kEThreads / 32;  // warps
   constexpr int PP = (D / 2) / NW;    // column pairs per warp per round
-  constexpr int PG = PP < 4 ? PP : 4; // pairs handled together (their loads and reductions overlap)
   extern __shared__ float smem[];
   float* A = smem;              // column-major [D][D]: the Schur complement, then the columns of L̃
   float* nrm = A + D * D;       // [D] squared column norms during the sweeps
@@ -275,7 +274,10 @@ __global__ void __launch_bounds__(kEThreads, 3) eig_kernel(const float* __restri
     __syncthreads();
   }
   // every column has now been pivoted: the columns of A are the columns of L̃ (in pivot order)
-  // ---- one-sided Jacobi on the columns of L̃ (round-robin pairs), norms carried along
+  // ---- one-sided Jacobi on the columns of L̃ (round-robin pairs), norms carried along.
+  // Eight lanes take one pair, so a warp works on four pairs at once: lane l of group g = lane / 8 holds
+  // the float4 at elements 32e + 4l .. + 3 (e < d/32) of both columns of the group's pair.  The dot product
+  // then reduces over three shuffle levels, and each scalar step of the rotation serves four pairs.
   for (int j = warp; j < D; j += NW) {
     float ss = 0.f;
 #pragma unroll
@@ -283,6 +285,11 @@ __global__ void __launch_bounds__(kEThreads, 3) eig_kernel(const float* __restri
     ss = warp_sum(ss);
     if (lane == 0) nrm[j] = ss;
   }
+  constexpr int IT = PP / 4;  // groups of four pairs per warp per round
+  constexpr float kTol2 = kJacobiTol * kJacobiTol, kExit2 = kJacobiExit * kJacobiExit;
+  const int g = lane / 8, lq = lane % 8;
+  const unsigned gmask = 0xffu << (8 * g);
+  float4* A4 = reinterpret_cast<float4*>(A);
   bool converged = false;
   int sweeps_run = 0;
   for (int sweep = 0; sweep < max_sweeps; ++sweep) {
@@ -290,56 +297,57 @@ __global__ void __launch_bounds__(kEThreads, 3) eig_kernel(const float* __restri
     int rotated = 0, big = 0;  // big: some relative off-diagonal of this sweep reached kJacobiExit
     for (int s = 0; s < D - 1; ++s) {
 #pragma unroll 1
-      for (int g0 = 0; g0 < PP; g0 += PG) {
-        float ap[PG][E], aq[PG][E], ga[PG];
-        int pj[PG], qj[PG];
+      for (int it = 0; it < IT; ++it) {
+        // round-robin pair k of round s without a division: (s, D-1) for k = 0, else (s+k, s-k) mod D-1
+        const int k = warp + (4 * it + g) * NW, m = D - 1;
+        int pp = s + k, qq = s - k;
+        if (pp >= m) pp -= m;
+        if (qq < 0) qq += m;
+        const int p = k == 0 ? s : pp, q = k == 0 ? m : qq;
+        float4 ap[E], aq[E];
+        float ga = 0.f;
 #pragma unroll
-        for (int t = 0; t < PG; ++t) {
-          // round-robin pair k of round s without a division: (s, D-1) for k = 0, else (s+k, s-k) mod D-1
-          const int k = warp + (g0 + t) * NW, m = D - 1;
-          int pp = s + k, qq = s - k;
-          if (pp >= m) pp -= m;
-          if (qq < 0) qq += m;
-          pj[t] = k == 0 ? s : pp;
-          qj[t] = k == 0 ? m : qq;
-          ga[t] = 0.f;
+        for (int e = 0; e < E; ++e) {
+          ap[e] = A4[p * (D / 4) + 8 * e + lq];
+          aq[e] = A4[q * (D / 4) + 8 * e + lq];
+          ga = fmaf(ap[e].x, aq[e].x, ga);
+          ga = fmaf(ap[e].y, aq[e].y, ga);
+          ga = fmaf(ap[e].z, aq[e].z, ga);
+          ga = fmaf(ap[e].w, aq[e].w, ga);
+        }
+        // the butterfly leaves the same sum in all eight lanes, so the group takes one branch below
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) ga += __shfl_xor_sync(0xffffffffu, ga, o);
+        const float al = nrm[p], be = nrm[q], ag2 = ga * ga;
+        big |= ga != 0.f && ag2 >= kExit2 * al * be;
+        if (ga != 0.f && ag2 > kTol2 * al * be) {
+          // tan θ = sign(ζ) / (|ζ| + sqrt(1 + ζ²)), ζ = (β − α) / 2γ; cos θ from the hardware reciprocal square
+          // root with one Newton–Raphson step (y ← y·(1.5 − 0.5·x·y²)), so that cos² + sin² = 1 to fp32
+          // rounding; the angle itself needs no more than approximate divisions
+          const float zeta = __fdividef(be - al, 2.f * ga);
+          const float z2 = fmaf(zeta, zeta, 1.f);
+          const float tn = copysignf(__fdividef(1.f, fabsf(zeta) + z2 * rsqrtf(z2)), zeta);
+          const float x = fmaf(tn, tn, 1.f);
+          float c = rsqrtf(x);
+          c = c * fmaf(-0.5f * x * c, c, 1.5f);
+          const float sn = c * tn, tau = __fdividef(sn, 1.f + c);
+          // the rotation written as a correction of each column (a_p − s(a_q + τa_p), a_q + s(a_p − τa_q),
+          // τ = s / (1 + c)): its rounding scales with the correction, not with the column, so that the many
+          // small late rotations do not drift the column norms (the eigenvalues)
 #pragma unroll
           for (int e = 0; e < E; ++e) {
-            ap[t][e] = A[pj[t] * D + lane + 32 * e];
-            aq[t][e] = A[qj[t] * D + lane + 32 * e];
-            ga[t] = fmaf(ap[t][e], aq[t][e], ga[t]);
+            const float4 u = ap[e], v = aq[e];
+            A4[p * (D / 4) + 8 * e + lq] = make_float4(u.x - sn * fmaf(tau, u.x, v.x), u.y - sn * fmaf(tau, u.y, v.y),
+                                                      u.z - sn * fmaf(tau, u.z, v.z), u.w - sn * fmaf(tau, u.w, v.w));
+            A4[q * (D / 4) + 8 * e + lq] = make_float4(v.x + sn * fmaf(-tau, v.x, u.x), v.y + sn * fmaf(-tau, v.y, u.y),
+                                                      v.z + sn * fmaf(-tau, v.z, u.z), v.w + sn * fmaf(-tau, v.w, u.w));
           }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-          for (int t = 0; t < PG; ++t) ga[t] += __shfl_xor_sync(0xffffffffu, ga[t], o);
-#pragma unroll
-        for (int t = 0; t < PG; ++t) {
-          const int p = pj[t], q = qj[t];
-          const float al = nrm[p], be = nrm[q];
-          const float nn = sqrtf(al) * sqrtf(be), ag = fabsf(ga[t]);
-          big |= ag > 0.f && ag >= kJacobiExit * nn;
-          if (ga[t] != 0.f && ag > kJacobiTol * nn) {
-            const float zeta = (be - al) / (2.f * ga[t]);
-            const float tn = (zeta >= 0.f ? 1.f : -1.f) / (fabsf(zeta) + sqrtf(1.f + zeta * zeta));
-            const float c = 1.f / sqrtf(1.f + tn * tn);
-            const float sn = c * tn, tau = sn / (1.f + c);
-            // the rotation written as a correction of each column (a_p − s(a_q + τa_p), a_q + s(a_p − τa_q),
-            // τ = s / (1 + c)): its rounding scales with the correction, not with the column, so that the many
-            // small late rotations do not drift the column norms (the eigenvalues)
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-              A[p * D + lane + 32 * e] = ap[t][e] - sn * fmaf(tau, ap[t][e], aq[t][e]);
-              A[q * D + lane + 32 * e] = aq[t][e] + sn * fmaf(-tau, aq[t][e], ap[t][e]);
-            }
-            __syncwarp();
-            if (lane == 0) {
-              nrm[p] = al - tn * ga[t];
-              nrm[q] = be + tn * ga[t];
-            }
-            rotated = 1;
+          __syncwarp(gmask);  // every lane of the group has read nrm[p], nrm[q]
+          if (lq == 0) {
+            nrm[p] = al - tn * ga;
+            nrm[q] = be + tn * ga;
           }
+          rotated = 1;
         }
       }
       __syncthreads();
