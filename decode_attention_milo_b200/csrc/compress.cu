@@ -264,12 +264,18 @@ __global__ void __launch_bounds__(kEThreads, 3) eig_kernel(const float* __restri
     }
     __syncthreads();
     if (threadIdx.x == 0) done[p] = 1;
-    // Schur complement of the remaining indices: A[i][j] -= L̃[i][k] L̃[j][k]
-    for (int e = threadIdx.x; e < D * D; e += kEThreads) {
-      const int j = e / D, i = e % D;
-      if (j == p || i == p) continue;
-      const float li = A[p * D + i], lj = A[p * D + j];
-      if (li != 0.f && lj != 0.f) A[e] = fmaf(-li, lj, A[e]);
+    // Schur complement of the remaining indices: A[i][j] -= L̃[i][k] L̃[j][k].  A thread keeps one row i
+    // (A[j·D + i] is row i of column j) and walks the columns j ≡ tid / D (mod kEThreads / D); eliminated rows
+    // and columns hold 0 in column p and are skipped (a column skip is uniform across the warp)
+    {
+      const int i = threadIdx.x % D;
+      const float li = A[p * D + i];
+      if (i != p && li != 0.f) {
+        for (int j = threadIdx.x / D; j < D; j += kEThreads / D) {
+          const float lj = A[p * D + j];
+          if (j != p && lj != 0.f) A[j * D + i] = fmaf(-li, lj, A[j * D + i]);
+        }
+      }
     }
     __syncthreads();
   }
@@ -285,6 +291,7 @@ __global__ void __launch_bounds__(kEThreads, 3) eig_kernel(const float* __restri
     ss = warp_sum(ss);
     if (lane == 0) nrm[j] = ss;
   }
+  __syncthreads();  // a pair reads norms that other warps wrote
   constexpr int IT = PP / 4;  // groups of four pairs per warp per round
   constexpr float kTol2 = kJacobiTol * kJacobiTol, kExit2 = kJacobiExit * kJacobiExit;
   const int g = lane / 8, lq = lane % 8;
@@ -305,16 +312,18 @@ __global__ void __launch_bounds__(kEThreads, 3) eig_kernel(const float* __restri
         if (qq < 0) qq += m;
         const int p = k == 0 ? s : pp, q = k == 0 ? m : qq;
         float4 ap[E], aq[E];
-        float ga = 0.f;
+        float gx[E];  // one partial dot product per float4, so that the FMA chains are short
 #pragma unroll
         for (int e = 0; e < E; ++e) {
           ap[e] = A4[p * (D / 4) + 8 * e + lq];
           aq[e] = A4[q * (D / 4) + 8 * e + lq];
-          ga = fmaf(ap[e].x, aq[e].x, ga);
-          ga = fmaf(ap[e].y, aq[e].y, ga);
-          ga = fmaf(ap[e].z, aq[e].z, ga);
-          ga = fmaf(ap[e].w, aq[e].w, ga);
+          gx[e] = fmaf(ap[e].w, aq[e].w, fmaf(ap[e].z, aq[e].z, fmaf(ap[e].y, aq[e].y, ap[e].x * aq[e].x)));
         }
+#pragma unroll
+        for (int w = 1; w < E; w *= 2)
+#pragma unroll
+          for (int e = 0; e + w < E; e += 2 * w) gx[e] += gx[e + w];
+        float ga = gx[0];
         // the butterfly leaves the same sum in all eight lanes, so the group takes one branch below
 #pragma unroll
         for (int o = 4; o > 0; o >>= 1) ga += __shfl_xor_sync(0xffffffffu, ga, o);

@@ -10,11 +10,11 @@
 // time, so that a TMEM lane holds one rank component and its columns are the
 // tile's tokens: row j of the 128-token slab the decode reads is then one lane's
 // 128 contiguous values.  One persistent CTA per SM walks blocks:
-//  - warps 2..5 convert the fp32 eigenvectors (rows 0..r−1, rows r..127 zero)
+//  - warps 6..13 convert the fp32 eigenvectors (rows 0..r−1, rows r..127 zero)
 //    to a bf16 pair hi + lo (B ≈ hi + lo to about 2^-17 relative), write them as
 //    the K-major A operand (M = 128 rank rows, K = d) in shared memory with the
-//    128-byte swizzle, into one of two buffers one block ahead of the MMAs, and
-//    store hi as the block's dimension-side factor rows;
+//    128-byte swizzle, into one of two buffers up to two blocks ahead of the
+//    MMAs, and store hi as the block's dimension-side factor rows;
 //  - warp 0 streams X_b through a 3-stage ring of 128-token tiles by TMA
 //    (K-major B operand, N = 128 tokens);
 //  - warp 1 issues tcgen05.mma kind::f16, hi and lo per k-step (bf16 products
@@ -35,7 +35,8 @@
 namespace milo {
 namespace {
 
-constexpr int kPThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 conversion and epilogue
+constexpr int kPConvWarps = 8;  // warps 6..13: the eigenvector conversion
+constexpr int kPThreads = 32 * (6 + kPConvWarps);  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue, then conversion
 constexpr int kPStages = 3;
 constexpr uint64_t kPWaitNs = 1000000000ull;
 
@@ -92,10 +93,11 @@ __global__ void __launch_bounds__(kPThreads) project_tc_kernel(const __grid_cons
   auto bar = [&](int i) { return ptx::smem_u32(&bars[i]); };
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
-    // the A operands and the accumulator releases get one arrival from each of the four epilogue warps
+    // an A operand gets one arrival from each conversion warp, an accumulator release one from each of the
+    // four epilogue warps
     for (int i = 0; i < P_COUNT; ++i) {
-      const bool four = i == P_AREADY || i == P_AREADY + 1 || i == P_TEMPTY || i == P_TEMPTY + 1;
-      ptx::mbar_init(bar(i), four ? 4 : 1);
+      const bool conv = i == P_AREADY || i == P_AREADY + 1, epi = i == P_TEMPTY || i == P_TEMPTY + 1;
+      ptx::mbar_init(bar(i), conv ? kPConvWarps : epi ? 4 : 1);
     }
     ptx::fence_mbar_init();
   }
@@ -183,11 +185,10 @@ __global__ void __launch_bounds__(kPThreads) project_tc_kernel(const __grid_cons
     if (lane == 0) ptx::umma_commit(bar(P_DONE));
     __syncwarp();
     pwait(bar(P_DONE), 0, status);
-  } else {
-    // ---- warps 2..5: each block's A operand and dimension-side factor (one block ahead of the MMAs), then
-    // the epilogue of its tiles
-    const int ew = warp - 2;        // 0..3
-    const int quarter = warp & 3;   // a warp reads TMEM lanes [32 (warp % 4), 32 (warp % 4) + 32)
+  } else if (warp >= 6) {
+    // ---- warps 6..13: each block's A operand and dimension-side factor, up to two blocks ahead of the MMAs
+    // (the epilogue warps never wait for a conversion)
+    const int cw = warp - 6;
     bool ok = true;
     auto convert = [&](int k) {
       const Blk x = blk(k);
@@ -196,14 +197,14 @@ __global__ void __launch_bounds__(kPThreads) project_tc_kernel(const __grid_cons
       if (k >= 2) ok = ok && pwait(bar(P_AFREE + ab), ((k >> 1) - 1) & 1, status);
       if (ok) {
         const float* ev = eigvecs + ((int64_t)x.p * nb + x.b) * D * D;
-        // rows j = ew, ew + 4, ...: lane handles columns [4 lane, 4 lane + 4) of each 128-column block; the
-        // loads of kRows rows are issued together so that their latencies overlap
+        // rows j = cw, cw + kPConvWarps, ...: lane handles columns [4 lane, 4 lane + 4) of each 128-column
+        // block; the loads of kRows rows are issued together so that their latencies overlap
         constexpr int kRows = 8;
-        for (int j0 = ew; j0 < 128; j0 += 4 * kRows) {
+        for (int j0 = cw; j0 < 128; j0 += kPConvWarps * kRows) {
           float4 vv[kRows][(D + 127) / 128];
 #pragma unroll
           for (int q = 0; q < kRows; ++q) {
-            const int j = j0 + 4 * q;
+            const int j = j0 + kPConvWarps * q;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 128) {
               const int c = c0 + 4 * lane;
@@ -213,7 +214,7 @@ __global__ void __launch_bounds__(kPThreads) project_tc_kernel(const __grid_cons
           }
 #pragma unroll
           for (int q = 0; q < kRows; ++q) {
-          const int j = j0 + 4 * q;
+          const int j = j0 + kPConvWarps * q;
 #pragma unroll
           for (int c0 = 0; c0 < D; c0 += 128) {
             const int c = c0 + 4 * lane;
@@ -243,13 +244,16 @@ __global__ void __launch_bounds__(kPThreads) project_tc_kernel(const __grid_cons
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(P_AREADY + ab));
     };
-    // epilogue: lane j of this warp's quarter holds rank component j = 32 quarter + lane; 128 tokens per tile
+    for (int k = 0; k < nmine && ok; ++k) convert(k);
+  } else {
+    // ---- warps 2..5, the epilogue: lane j of this warp's quarter holds rank component j = 32 quarter + lane;
+    // 128 tokens per tile
+    const int quarter = warp & 3;  // a warp reads TMEM lanes [32 (warp % 4), 32 (warp % 4) + 32)
+    bool ok = true;
     const int j = 32 * quarter + lane;
     const uint32_t tl = tmem + ((uint32_t)(32 * quarter) << 16);
     int g = 0;
-    if (nmine > 0) convert(0);
     for (int k = 0; k < nmine && ok; ++k) {
-      if (k + 1 < nmine) convert(k + 1);  // the next block's operand is ready before this block's epilogue
       const Blk x = blk(k);
       for (int s = 0; s < tiles; ++s, ++g) {
         const int buf = g & 1;
