@@ -55,7 +55,7 @@ def _args():
     p.add_argument("--workload", default="qwen2.5-7b-layer")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="bound of the CPU oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--profile", choices=["decode", "decode8", "compress"], default=None,
+    p.add_argument("--profile", choices=["decode", "decode8", "rope", "compress"], default=None,
                    help="run only N calls of one phase on the workload (for profiler captures), no JSON contract")
     p.add_argument("--calls", type=int, default=6)
     return p.parse_args()
@@ -728,7 +728,10 @@ def run_profile(a):
         vs = dev(L["V_suf"]) if wl.suffix else None
         out = torch.empty_like(q)
         for _ in range(a.calls):
-            milo.decode_attn(q, f, ks, vs, out=out)
+            if a.profile == "rope":
+                milo.decode_attn_rope(q, f, ks, vs, theta=1e6, out=out)
+            else:
+                milo.decode_attn(q, f, ks, vs, out=out)
         torch.cuda.synchronize()
         assert f.status()[0] == 0
         f.close()
