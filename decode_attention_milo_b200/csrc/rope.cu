@@ -10,14 +10,14 @@
 //   (i, i + d/2) by φ_i = pos·θ^(−2i/d), pos = t (the token's absolute position),
 // and written as bf16 [H][T][d], the dense key layout the decode kernel reads.
 //
-// One CTA of 128 threads per (KV head, block, 128-token chunk), three resident per SM:
+// One CTA of 256 threads per (KV head, block, 128-token chunk), three resident per SM:
 //   - one thread loads the chunk's token-factor slab [r][128 tokens] and the block's dimension factor
 //     [r][d] with one TMA box each (height r rounded up to 16; the rows past r are cleared in shared memory);
 //   - the same thread issues K_chunk = U·Bᵀ as one tcgen05 MMA chain (M = 128 tokens, N = d, K = r, both
 //     operands MN-major) into d TMEM columns;
-//   - each thread then owns TMEM lane t = one token: it reads the pairs (i, i + d/2), rotates them with the
-//     angle reduced in fp64 before the fp32 sine and cosine, and writes the bf16 row into a 128-byte-swizzled
-//     tile in shared memory (the token-factor buffer, free once the MMA has completed);
+//   - two threads then share TMEM lane t = one token, each half of its pairs (i, i + d/2): they rotate them
+//     with the angle reduced in fp64 before the fp32 sine and cosine, and write the bf16 values into a
+//     128-byte-swizzled tile in shared memory (the token-factor buffer, free once the MMA has completed);
 //   - one TMA store writes the 128 × d tile to the output.
 // Every wait is bounded (1 s): on expiry the kernel records kStatusDecodeTimeout and skips the rest.
 #include <cuda.h>
@@ -30,7 +30,7 @@
 namespace milo {
 namespace {
 
-constexpr int kRThreads = 128;
+constexpr int kRThreads = 256;  // two threads per token in the epilogue, each half of the pairs
 constexpr uint64_t kRWaitNs = 1000000000ull;
 constexpr int kUBytes = 2 * 128 * 128;  // token-factor box [2 column blocks][≤ 128 rows][128 B], later the output tile
 template <int D>
@@ -85,6 +85,7 @@ __global__ void __launch_bounds__(kRThreads) rope_keys_kernel(const __grid_const
   const uint32_t b_full = ptx::smem_u32(&bars[0]), b_done = ptx::smem_u32(&bars[1]);
   __shared__ double s_freq[P];  // θ^(−2i/d)
   const int warp = threadIdx.x / 32, t = threadIdx.x;
+  const int tok = t & 127, half = t >> 7;  // epilogue: TMEM lane (token) and half of the pairs
   const int cpb = n / 128;
   const int c = blockIdx.x % cpb, b = (blockIdx.x / cpb) % nb, h = blockIdx.x / (cpb * nb);
   const int r = __ldg(ranks + (size_t)(2 * h) * nb + b);
@@ -146,13 +147,14 @@ __global__ void __launch_bounds__(kRThreads) rope_keys_kernel(const __grid_const
   ok = __syncthreads_and(ok);
   ptx::tc_fence_after();
 
-  // ---- rotate token t's pairs and stage the bf16 row (the U box is free: the MMA has read it)
+  // ---- rotate token tok's pairs [half·d/4, half·d/4 + d/4) and stage them as bf16 (the U box is free: the MMA
+  // has read it); warp w reads TMEM lanes 32·(w mod 4) .. + 31
   if (ok) {
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    const double pos = (double)((int64_t)b * n + (int64_t)c * 128 + t);
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const double pos = (double)((int64_t)b * n + (int64_t)c * 128 + tok);
     constexpr double kTwoPi = 6.283185307179586, kInvTwoPi = 0.15915494309189535;
 #pragma unroll 1
-    for (int i0 = 0; i0 < P; i0 += 16) {
+    for (int i0 = half * (P / 2); i0 < (half + 1) * (P / 2); i0 += 16) {
       float x1[16], x2[16];
       ptx::tmem_ld16(tl + (uint32_t)i0, x1);
       ptx::tmem_ld16(tl + (uint32_t)(P + i0), x2);
@@ -174,10 +176,10 @@ __global__ void __launch_bounds__(kRThreads) rope_keys_kernel(const __grid_const
         w1[k / 2] = ptx::pack_bf16(y1[0], y1[1]);
         w2[k / 2] = ptx::pack_bf16(y2[0], y2[1]);
       }
-      st_out8(sU, t, i0, w1);
-      st_out8(sU, t, i0 + 8, w1 + 4);
-      st_out8(sU, t, P + i0, w2);
-      st_out8(sU, t, P + i0 + 8, w2 + 4);
+      st_out8(sU, tok, i0, w1);
+      st_out8(sU, tok, i0 + 8, w1 + 4);
+      st_out8(sU, tok, P + i0, w2);
+      st_out8(sU, tok, P + i0 + 8, w2 + 4);
     }
     ptx::fence_async_smem();
   }
