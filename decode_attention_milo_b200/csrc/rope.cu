@@ -19,7 +19,8 @@
 //     with the angle reduced in fp64 before the fp32 sine and cosine, and write the bf16 values into a
 //     128-byte-swizzled tile in shared memory (the token-factor buffer, free once the MMA has completed);
 //   - one TMA store writes the 128 × d tile to the output.
-// Every wait is bounded (1 s): on expiry the kernel records kStatusDecodeTimeout and skips the rest.
+// Every wait is bounded (1 s): on expiry the kernel records kStatusDecodeTimeout, skips the rest, and gives the
+// copies or MMAs it issued one more bounded wait before it frees TMEM and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -120,6 +121,7 @@ __global__ void __launch_bounds__(kRThreads) rope_keys_kernel(const __grid_const
     else ptx::tma_load_2d(sB, bm, b_full, 0, (int)row0);
   }
   bool ok = __syncthreads_and(rwait(b_full, 0, status));
+  if (!ok) rwait(b_full, 0, status);  // after a timeout, one more bounded wait for the copies still in flight
   if (ok) {
     // rows r .. rp-1 of both boxes belong to the next chunk or block (or are past the array): clear them so
     // they add nothing (a whole 128-byte row stays in place under the swizzle)
@@ -143,8 +145,10 @@ __global__ void __launch_bounds__(kRThreads) rope_keys_kernel(const __grid_const
     for (int k = 0; k < rp / 16; ++k) ptx::umma_bf16(tmem, mn_desc(sU, k, cbs), mn_desc(sB, k, cbs), id, k > 0);
     ptx::umma_commit(b_done);
   }
+  const bool issued = ok;
   if (ok) ok = rwait(b_done, 0, status);
   ok = __syncthreads_and(ok);
+  if (issued && !ok) rwait(b_done, 0, status);  // the same for MMAs still in flight, before TMEM is freed
   ptx::tc_fence_after();
 
   // ---- rotate token tok's pairs [half·d/4, half·d/4 + d/4) and stage them as bf16 (the U box is free: the MMA
