@@ -6,8 +6,8 @@
 // from its entropy under a fixed total budget.  Four kernels per layer, all on
 // the caller's stream:
 //   gram     G_b = X_bᵀ X_b in fp32  (bf16 blocks: tensor cores, gram_tc.cu; fp32: here, one CTA per block)
-//   jacobi   one-sided Jacobi on G_b: eigenvalues λ_i = σ_i², eigenvectors B_b,
-//            sorted descending                            (one CTA per block)
+//   eig      pivoted Cholesky of G_b, then one-sided Jacobi on the columns of its factor: eigenvalues
+//            λ_i = σ_i², eigenvectors B_b, sorted descending      (one CTA per block)
 //   alloc    H_b = −Σ p ln p (p = λ/Σλ, fp64), w_b = e^{H_b}, quotas
 //            clamp(lam·w_b, r_min, d) with Σ = R, largest-remainder ranks,
 //            row offsets                                  (one CTA per pool)
@@ -22,9 +22,6 @@ namespace milo {
 namespace {
 
 constexpr int kThreads = 256;
-// Jacobi runs one CTA per block with 128 KB of shared memory (one CTA per SM), so it uses more warps to hide
-// the latency of each round: 16 warps, 4 column pairs per warp per round (d = 128).
-constexpr int kJThreads = 512;
 constexpr float kJacobiTol = 1e-5f;  // relative orthogonality |a_p·a_q| / (|a_p||a_q|)
 // A sweep whose largest relative off-diagonal stays below this ends the iteration: cyclic Jacobi converges
 // quadratically, so what remains after it is of order 1e-7, below kJacobiTol, and the next sweep would
@@ -78,122 +75,7 @@ __global__ void __launch_bounds__(kThreads) gram_kernel(const T* __restrict__ K,
     for (int j = 0; j < MT; ++j) G[(ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
 }
 
-// ---------------------------------------------------------------- jacobi
-// Round-robin (circle method) pairing: round s in [0, D-1), pair k in [0, D/2).
-__device__ __forceinline__ void rr_pair(int D, int s, int k, int& p, int& q) {
-  const int m = D - 1;
-  if (k == 0) {
-    p = s;
-    q = m;
-  } else {
-    p = (s + k) % m;
-    q = (s - k + m) % m;
-  }
-}
-
-template <int D>
-__global__ void __launch_bounds__(kJThreads) jacobi_kernel(const float* __restrict__ gram, int nb, int max_sweeps,
-                                                         float* __restrict__ eigvals, float* __restrict__ eigvecs,
-                                                         int32_t* __restrict__ sweeps_out, uint32_t* status) {
-  constexpr int E = D / 32;  // elements per lane of one column
-  extern __shared__ float smem[];
-  float* A = smem;          // column-major: column j at A[j*D]
-  float* W = smem + D * D;  // accumulated rotations, column-major
-  float* lam = W + D * D;   // D
-  const int blk = blockIdx.x + blockIdx.y * nb;
-  const float* G = gram + (int64_t)blk * D * D;
-  for (int e = threadIdx.x; e < D * D; e += kJThreads) {
-    A[e] = G[e];  // G symmetric: row-major == column-major
-    W[e] = (e / D == e % D) ? 1.f : 0.f;
-  }
-  __syncthreads();
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  constexpr int NW = kJThreads / 32;
-  constexpr int PP = (D / 2) / NW;  // column pairs per warp per round
-  bool converged = false;
-  int sweeps_run = 0;
-  for (int sweep = 0; sweep < max_sweeps; ++sweep) {
-    ++sweeps_run;
-    int rotated = 0;
-    for (int s = 0; s < D - 1; ++s) {
-      // the warp's PP pairs are handled together so that their loads and reductions overlap
-      float ap[PP][E], aq[PP][E], al[PP], be[PP], ga[PP];
-      int pj[PP], qj[PP];
-#pragma unroll
-      for (int t = 0; t < PP; ++t) {
-        rr_pair(D, s, warp + t * NW, pj[t], qj[t]);
-        al[t] = be[t] = ga[t] = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          ap[t][e] = A[pj[t] * D + lane + 32 * e];
-          aq[t][e] = A[qj[t] * D + lane + 32 * e];
-          al[t] = fmaf(ap[t][e], ap[t][e], al[t]);
-          be[t] = fmaf(aq[t][e], aq[t][e], be[t]);
-          ga[t] = fmaf(ap[t][e], aq[t][e], ga[t]);
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-        for (int t = 0; t < PP; ++t) {
-          al[t] += __shfl_xor_sync(0xffffffffu, al[t], o);
-          be[t] += __shfl_xor_sync(0xffffffffu, be[t], o);
-          ga[t] += __shfl_xor_sync(0xffffffffu, ga[t], o);
-        }
-#pragma unroll
-      for (int t = 0; t < PP; ++t) {
-        if (ga[t] != 0.f && fabsf(ga[t]) > kJacobiTol * sqrtf(al[t]) * sqrtf(be[t])) {
-          const float zeta = (be[t] - al[t]) / (2.f * ga[t]);
-          const float tn = (zeta >= 0.f ? 1.f : -1.f) / (fabsf(zeta) + sqrtf(1.f + zeta * zeta));
-          const float c = 1.f / sqrtf(1.f + tn * tn);
-          const float sn = c * tn;
-          const int p = pj[t], q = qj[t];
-#pragma unroll
-          for (int e = 0; e < E; ++e) {
-            A[p * D + lane + 32 * e] = c * ap[t][e] - sn * aq[t][e];
-            A[q * D + lane + 32 * e] = sn * ap[t][e] + c * aq[t][e];
-            const float wp = W[p * D + lane + 32 * e], wq = W[q * D + lane + 32 * e];
-            W[p * D + lane + 32 * e] = c * wp - sn * wq;
-            W[q * D + lane + 32 * e] = sn * wp + c * wq;
-          }
-          rotated = 1;
-        }
-      }
-      __syncthreads();
-    }
-    if (!__syncthreads_or(rotated)) {
-      converged = true;
-      break;
-    }
-  }
-  if (!converged && threadIdx.x == 0) atomicOr(status, kStatusNoConvergence);
-  if (threadIdx.x == 0) sweeps_out[blk] = sweeps_run;
-  // eigenvalue of column j = |G w_j| = norm of A's column j
-  for (int j = warp; j < D; j += kJThreads / 32) {
-    float ss = 0.f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const float v = A[j * D + lane + 32 * e];
-      ss = fmaf(v, v, ss);
-    }
-    ss = warp_sum(ss);
-    if (lane == 0) lam[j] = sqrtf(ss);
-  }
-  __syncthreads();
-  // sort descending by counting (ties: lower column first)
-  for (int j = warp; j < D; j += kJThreads / 32) {
-    const float lj = lam[j];
-    int rank = 0;
-    for (int i = lane; i < D; i += 32) rank += (lam[i] > lj) || (lam[i] == lj && i < j);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
-    if (lane == 0) eigvals[(int64_t)blk * D + rank] = lj;
-    float* dst = eigvecs + ((int64_t)blk * D + rank) * D;
-#pragma unroll
-    for (int e = 0; e < E; ++e) dst[lane + 32 * e] = W[j * D + lane + 32 * e];
-  }
-}
-
+// ---------------------------------------------------------------- eigen-decomposition
 // Eigen-decomposition of G_b by one-sided Jacobi preconditioned with a pivoted Cholesky factor
 // (the preconditioning of Demmel–Veselić and Drmač for Jacobi SVD): G = L̃ L̃ᵀ with L̃ the Cholesky
 // factor under diagonal pivoting, its rows kept in the original index order; then one-sided Jacobi
